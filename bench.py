@@ -1,0 +1,326 @@
+"""Benchmark of the VDN-H3 hybrid attention layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--impl ours|reference]
+
+One step is one call of the whole layer (vdn_hybrid_attn_fwd: mask tables, softmax
+branch, linear states, scan, read, fuse, both output projections) on one batch of
+synthetic inputs resident in HBM.  With N > 1 (launched by torch.distributed.run) every
+rank runs its own independent replica on its own seeded batch: the layer is
+data-parallel over batch elements and has no exchange step, so the ranks share only the
+barrier and the max-over-ranks timing (weak scaling).
+
+The JSON line reports video tokens/s over all ranks, an end-to-end figure through the
+C ABI with pinned host buffers (host->device copies of q, k, v and the text k, v, and the
+device->host copy of y inside the timed region), the roofline of the dominant kernel
+timed live with CUDA events on its launching stream, and the float64 CPU oracle timed on
+a bounded sample on the host cores (rank 0 at N = 1 only).
+
+``--impl reference`` times that CPU oracle alone on the same workload and metric (each
+step a bounded sample, extrapolated to the whole layer).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hybrid_softmax_linear_b200 import synth  # noqa: E402
+
+METRIC = "hybrid-attn layer video tokens/s @1 B200; % of bf16 tensor / HBM roofline"
+UNIT = "video tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def softmax_flops(shape: synth.Shape) -> float:
+    """Algorithmic FLOPs of the softmax branch: 4 D H sum over queries of |keys(q)|."""
+    import hybrid_softmax_linear_b200 as vdn
+    _, gtab = vdn.mask_layout_build(shape)
+    T = shape.tokens_per_frame
+    total = 0
+    for r in gtab:
+        keys = sum(int(r[5 + 2 * i]) - int(r[4 + 2 * i]) for i in range(int(r[2])))
+        total += (int(r[1]) - int(r[0])) * T * keys
+    return 4.0 * shape.head_dim * shape.heads * total
+
+
+def layer_flops(shape: synth.Shape) -> dict:
+    Nv, H, D = shape.n_video, shape.heads, shape.head_dim
+    F, L = shape.frames, shape.text_tokens
+    return {
+        "softmax": softmax_flops(shape),
+        "out_proj": 2.0 * Nv * (2 * H * D) * (H * D),
+        "state_build": 2.0 * (Nv + L) * H * D * D,
+        "read": 2.0 * Nv * H * D * D,
+        "gate": 2.0 * Nv * H * D * D,
+        "scan": float(F * H * (D * D + D)),
+    }
+
+
+def load_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            return json.load(fh), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+def oracle_sample(cfg: int, inp: dict, n_rows: int, seed: int = 11) -> dict:
+    """Time the float64 oracle on a bounded sample of the layer: all per-frame linear
+    states (shared by every query) plus softmax, linear read, fuse and projections for
+    n_rows random query rows (all heads).  Extrapolates to video tokens/s of the whole
+    layer: t = t_states + t_rows * N_v / n_rows."""
+    from oracle import vdn_oracle as vo
+    w = synth.CONFIGS[cfg]
+    s = w.shape
+    F, T, C = s.frames, s.tokens_per_frame, s.chunk_frames
+    o = {n: (synth.bf16_bits_to_f32(a) if a.dtype == np.uint16 else a) for n, a in inp.items()}
+    rows = np.sort(np.random.default_rng(seed).choice(s.n_video, size=n_rows, replace=False))
+    t0 = time.perf_counter()
+    if w.linear == "delta":
+        mem = vo.delta_memory(o["k"], o["v"], o["kt"], o["vt"], o["beta"], F, T, C)
+    else:
+        mem = vo.linear_memory(o["k"], o["v"], o["kt"], o["vt"], F, T, C)
+    t1 = time.perf_counter()
+    o_s = vo.softmax_branch(o["q"], o["k"], o["v"], o["kt"], o["vt"], F, T, C, rows=rows)
+    o_l = vo.delta_read(o["q"], *mem, T, rows) if w.linear == "delta" else vo.linear_read(o["q"], *mem, T, rows)
+    a = vo.hybrid_fuse(o["q"][rows], o_s, o_l, o["w_gate_s"], o["w_gate_l"], o["gamma"], 1e-6)
+    vo.out_proj(a, o["w_os"], o["w_ol"])
+    t2 = time.perf_counter()
+    t_full = (t1 - t0) + (t2 - t1) * s.n_video / n_rows
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        cores = len(os.sched_getaffinity(0))
+    return {"value": s.n_video / t_full, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"all per-frame linear states + {n_rows} random query rows x {s.heads} heads "
+                      f"(softmax, linear read, fuse, projections); extrapolated as "
+                      f"t_states + t_rows*N_v/{n_rows}",
+            "t_states_s": round(t1 - t0, 3), "t_rows_s": round(t2 - t1, 3)}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle as it stands, on rank 0 only."""
+    if rank != 0:
+        return
+    cfg = args.config
+    inp = synth.workload_inputs(cfg)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(cfg, inp, args.ref_rows, seed=100 + i)
+        if i >= args.warmup:
+            vals.append(r)
+    value = statistics.median(v["value"] for v in vals)
+    w = synth.CONFIGS[cfg]
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.shape.n_video / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(cfg),
+            "cpu_baseline": {k: vals[-1][k] for k in ("kind", "cores", "sample")} | {"value": value, "unit": UNIT},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg: int) -> dict:
+    w = synth.CONFIGS[cfg]
+    s = w.shape
+    return {"workload": w.name, "frames": s.frames, "tokens_per_frame": s.tokens_per_frame,
+            "chunk_frames": s.chunk_frames, "text_tokens": s.text_tokens, "heads": s.heads, "head_dim": s.head_dim,
+            "video_tokens": s.n_video, "linear": w.linear, "softmax_fp8": w.softmax_fp8, "batch": 1,
+            "parallelism": "replicas (data-parallel, one batch per rank)",
+            "l2": "inputs larger than L2 (q, k, v are each > 126 MB at this size)"}
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import hybrid_softmax_linear_b200 as vdn
+    from hybrid_softmax_linear_b200.tensors import to_device, to_torch, workspace
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = args.config
+    w = synth.CONFIGS[cfg]
+    s = w.shape
+    kind = vdn.DELTA if w.linear == "delta" else vdn.ELU1
+    cdt = vdn.E4M3 if w.softmax_fp8 else (vdn.F32 if w.dtype == "f32" else vdn.BF16)
+    tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    inp = synth.workload_inputs(cfg, rank)
+    names_in = ["q", "k", "v", "kt", "vt"] + (["beta"] if kind == vdn.DELTA else [])
+    d = {n: to_device(a, dev) for n, a in inp.items()}
+    G_l = inp["w_gate_l"].shape[2]
+    ws = workspace(vdn.hybrid_attn_workspace_size(s, kind, cdt), dev)
+    y = torch.empty((s.n_video, s.hidden), dtype=tdt, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    vdn.workspace_init(ws, stream)
+
+    def step(src):
+        vdn.hybrid_attn_fwd(s, kind, cdt, src["q"], src["k"], src["v"], src["kt"], src["vt"],
+                            src.get("beta") if kind == vdn.DELTA else None, d["w_gate_s"], d["w_gate_l"], G_l,
+                            d["gamma"], 1e-6, d["w_os"], d["w_ol"], y, ws, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step(d)
+    torch.cuda.synchronize(dev)
+    vdn.check_device_status(ws, stream)
+
+    # ---- timed region: K steps, inputs resident in HBM
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    vdn.profile_begin(64 * max(args.steps, 1))
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(d)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    prof = vdn.profile_end()
+    clk = clocks.stop() if clocks else None
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    vdn.check_device_status(ws, stream)
+
+    # ---- end to end through the C ABI with pinned host buffers
+    host_in = {n: to_torch(inp[n]).pin_memory() for n in names_in}
+    dev_in = {n: torch.empty_like(host_in[n], device=dev) for n in names_in}
+    host_y = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_y.numel() * host_y.element_size()
+    e2e_steps = max(1, min(args.steps, 3))
+    barrier()
+    torch.cuda.synchronize(dev)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        for n in names_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        step(dev_in)
+        host_y.copy_(y, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1)) / e2e_steps
+
+    if rank != 0:
+        return
+    per_step_ms = ms / max(args.steps, 1)
+    value = world * s.n_video / (per_step_ms / 1e3)
+    peaks, peak_src = load_peaks()
+    fl = layer_flops(s)
+    sm_key = "softmax_tc" if "softmax_tc" in prof else "softmax_simt"
+    sm_ms, sm_n = prof.get(sm_key, (0.0, 0))
+    sm_avg = sm_ms / max(sm_n, 1)
+    achieved = fl["softmax"] / (sm_avg / 1e3) / 1e12 if sm_avg > 0 else None
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    launches = sum(n for _, n in prof.values())
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic", "config": workload_config(cfg),
+        "roofline": {"kernel": sm_key, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel runs inside a long step)",
+                     "algorithmic_tflop_per_launch": fl["softmax"] / 1e12, "avg_launch_ms": sm_avg},
+        "layer_tflops": sum(v for k, v in fl.items()) / (per_step_ms / 1e3) / 1e12,
+        "per_kernel_ms_per_step": {k: round(v[0] / max(args.steps, 1), 4) for k, v in prof.items()},
+        "gpu_launches": launches,
+        "e2e": {"value": world * s.n_video / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(cfg, inp, args.cpu_rows)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=4, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=48, help="query rows of the CPU oracle sample")
+    ap.add_argument("--ref-rows", type=int, default=32, help="query rows per step of --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import datetime
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

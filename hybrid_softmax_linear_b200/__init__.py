@@ -1,0 +1,221 @@
+"""Python binding of libvdn, the sm_100a implementation of the VDN-H3 hybrid attention
+layer (forward).  Argument marshalling only: every step runs in the library's CUDA
+kernels; torch is used for device memory and streams.
+
+The functions carry the C entry points' names without the ``vdn_`` prefix and accept
+torch tensors (their ``data_ptr()`` is passed) or raw integer device pointers.  A
+non-zero status raises :class:`VdnError` with the library's message.  If libvdn.so is
+missing, :func:`lib` raises: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+__all__ = [
+    "VdnError", "Shape", "lib", "F32", "BF16", "E4M3", "ELU1", "DELTA",
+    "mask_layout_build", "max_groups", "hybrid_attn_workspace_size", "step_workspace_size", "workspace_init",
+    "softmax_branch_fwd", "linear_state_build", "linear_state_scan", "linear_read", "hybrid_fuse", "out_proj",
+    "hybrid_attn_fwd", "hybrid_attn_intermediate", "check_device_status", "debug_unset_flag_wait", "version",
+    "profile_begin", "profile_end",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdn.so")
+
+F32, BF16, E4M3 = 0, 1, 2
+ELU1, DELTA = 0, 1
+STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT", 6: "DEVICE"}
+
+
+class VdnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"vdn status {status} ({STATUS.get(status, '?')}): {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("frames", ctypes.c_int32), ("tokens_per_frame", ctypes.c_int32), ("chunk_frames", ctypes.c_int32),
+                ("text_tokens", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+    @classmethod
+    def of(cls, s) -> "Shape":
+        if isinstance(s, Shape):
+            return s
+        return cls(s.frames, s.tokens_per_frame, s.chunk_frames, s.text_tokens, s.heads, s.head_dim)
+
+
+_lib = None
+_vp, _sz, _i32, _f32, _u32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_float, ctypes.c_uint32
+_SP = ctypes.POINTER(Shape)
+
+_SIGS = {
+    "vdn_version": (ctypes.c_int, []),
+    "vdn_last_error": (ctypes.c_char_p, []),
+    "vdn_mask_layout_build": (ctypes.c_int, [_SP, _vp, _vp, _vp, _sz]),
+    "vdn_max_groups": (_i32, [_SP]),
+    "vdn_hybrid_attn_workspace_size": (_sz, [_SP, ctypes.c_int, ctypes.c_int]),
+    "vdn_step_workspace_size": (_sz, [_SP]),
+    "vdn_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
+    "vdn_softmax_branch_fwd": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp,
+                                              _sz, _vp]),
+    "vdn_linear_state_build": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                              _vp, _vp, _sz, _vp]),
+    "vdn_linear_state_scan": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                             _sz, _vp]),
+    "vdn_linear_read": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                       _vp]),
+    "vdn_hybrid_fuse": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _f32, _vp, _vp]),
+    "vdn_out_proj": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]),
+    "vdn_hybrid_attn_fwd": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                           _i32, _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "vdn_hybrid_attn_intermediate": (_vp, [_SP, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int]),
+    "vdn_check_device_status": (ctypes.c_int, [_vp, _sz, _vp]),
+    "vdn_debug_unset_flag_wait": (ctypes.c_int, [_vp, _sz, _u32, _vp]),
+    "vdn_profile_begin": (ctypes.c_int, [_i32]),
+    "vdn_profile_end": (ctypes.c_int, [_vp, _vp, _i32]),
+}
+
+PROF_KERNELS = 16
+KERNEL_NAMES = {1: "tables", 2: "softmax_simt", 3: "softmax_tc", 4: "state_build", 5: "scan", 6: "read", 7: "fuse",
+                8: "out_proj_simt", 9: "out_proj_tc", 10: "fp8_quant", 11: "delta_stats"}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libvdn.so (built in-tree by ``python -m hybrid_softmax_linear_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libvdn.so not found at {LIB_PATH}; build it with "
+                               "`python -m hybrid_softmax_linear_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _p(x):
+    """Device pointer of a tensor, an int, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _nbytes(ws):
+    return ws.numel() * ws.element_size()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int):
+    if status != 0:
+        raise VdnError(status, lib().vdn_last_error().decode(errors="replace"))
+
+
+def version() -> int:
+    return lib().vdn_version()
+
+
+def max_groups(shape) -> int:
+    return lib().vdn_max_groups(ctypes.byref(Shape.of(shape)))
+
+
+def mask_layout_build(shape, cap: int | None = None):
+    """(frame_tab int32[F, 8], group_tab int32[G, 16]) from the host layout builder."""
+    s = Shape.of(shape)
+    cap = max_groups(s) if cap is None else cap
+    ftab = np.zeros((s.frames, 8), np.int32)
+    gtab = np.zeros((max(cap, 1), 16), np.int32)
+    G = ctypes.c_int32(0)
+    _check(lib().vdn_mask_layout_build(ctypes.byref(s), ftab.ctypes.data, gtab.ctypes.data, ctypes.byref(G), cap))
+    return ftab, gtab[:G.value].copy()
+
+
+def hybrid_attn_workspace_size(shape, kind: int, dtype: int) -> int:
+    return lib().vdn_hybrid_attn_workspace_size(ctypes.byref(Shape.of(shape)), kind, dtype)
+
+
+def step_workspace_size(shape) -> int:
+    return lib().vdn_step_workspace_size(ctypes.byref(Shape.of(shape)))
+
+
+def workspace_init(ws, stream=None):
+    _check(lib().vdn_workspace_init(_p(ws), _nbytes(ws), _stream(stream)))
+
+
+def softmax_branch_fwd(shape, dtype, q, k, v, kt, vt, o_s, ws, scales=None, sm_scale=0.0, lse=None, stream=None):
+    _check(lib().vdn_softmax_branch_fwd(ctypes.byref(Shape.of(shape)), dtype, _p(q), _p(k), _p(v), _p(kt), _p(vt),
+                                        _p(scales), sm_scale, _p(o_s), _p(lse), _p(ws), _nbytes(ws),
+                                        _stream(stream)))
+
+
+def linear_state_build(shape, kind, dtype, k, v, kt, vt, S, z, S_txt, z_txt, ws=None, stream=None):
+    _check(lib().vdn_linear_state_build(ctypes.byref(Shape.of(shape)), kind, dtype, _p(k), _p(v), _p(kt), _p(vt),
+                                        _p(S), _p(z), _p(S_txt), _p(z_txt), _p(ws),
+                                        0 if ws is None else _nbytes(ws), _stream(stream)))
+
+
+def linear_state_scan(shape, kind, S, z, S_txt, z_txt, beta, S_fwd, S_bwd, z_fwd, z_bwd, ws, stream=None):
+    _check(lib().vdn_linear_state_scan(ctypes.byref(Shape.of(shape)), kind, _p(S), _p(z), _p(S_txt), _p(z_txt),
+                                       _p(beta), _p(S_fwd), _p(S_bwd), _p(z_fwd), _p(z_bwd), _p(ws), _nbytes(ws),
+                                       _stream(stream)))
+
+
+def linear_read(shape, kind, dtype, q, S_fwd, S_bwd, z_fwd, z_bwd, o_l, ws, stream=None):
+    _check(lib().vdn_linear_read(ctypes.byref(Shape.of(shape)), kind, dtype, _p(q), _p(S_fwd), _p(S_bwd),
+                                 _p(z_fwd), _p(z_bwd), _p(o_l), _p(ws), _nbytes(ws), _stream(stream)))
+
+
+def hybrid_fuse(shape, dtype, q, o_s, o_l, w_gate_s, w_gate_l, G_l, gamma, eps, a, stream=None):
+    _check(lib().vdn_hybrid_fuse(ctypes.byref(Shape.of(shape)), dtype, _p(q), _p(o_s), _p(o_l), _p(w_gate_s),
+                                 _p(w_gate_l), G_l, _p(gamma), eps, _p(a), _stream(stream)))
+
+
+def out_proj(shape, dtype, a, w_os, w_ol, y, stream=None):
+    _check(lib().vdn_out_proj(ctypes.byref(Shape.of(shape)), dtype, _p(a), _p(w_os), _p(w_ol), _p(y),
+                              _stream(stream)))
+
+
+def hybrid_attn_fwd(shape, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma, eps, w_os, w_ol, y,
+                    ws, stream=None):
+    _check(lib().vdn_hybrid_attn_fwd(ctypes.byref(Shape.of(shape)), kind, dtype, _p(q), _p(k), _p(v), _p(kt),
+                                     _p(vt), _p(beta), _p(w_gate_s), _p(w_gate_l), G_l, _p(gamma), eps, _p(w_os),
+                                     _p(w_ol), _p(y), _p(ws), _nbytes(ws), _stream(stream)))
+
+
+def hybrid_attn_intermediate(shape, kind, dtype, ws, which: int) -> int:
+    """Device address of an intermediate inside ws (0 O_s, 1 O_l, 2 A, 3 S_fwd, 4 S_bwd)."""
+    return lib().vdn_hybrid_attn_intermediate(ctypes.byref(Shape.of(shape)), kind, dtype, _p(ws), which) or 0
+
+
+def check_device_status(ws, stream=None):
+    _check(lib().vdn_check_device_status(_p(ws), _nbytes(ws), _stream(stream)))
+
+
+def profile_begin(max_launches: int = 4096):
+    """Start per-kernel CUDA-event timing of vdn_hybrid_attn_fwd calls."""
+    _check(lib().vdn_profile_begin(max_launches))
+
+
+def profile_end() -> dict:
+    """{kernel name: (total ms, launches)} of the launches recorded since profile_begin."""
+    ms = (ctypes.c_float * PROF_KERNELS)()
+    n = (ctypes.c_int32 * PROF_KERNELS)()
+    _check(lib().vdn_profile_end(ms, n, PROF_KERNELS))
+    return {KERNEL_NAMES.get(k, str(k)): (float(ms[k]), int(n[k])) for k in range(PROF_KERNELS) if n[k] > 0}
+
+
+def debug_unset_flag_wait(ws, max_polls: int, stream=None):
+    _check(lib().vdn_debug_unset_flag_wait(_p(ws), _nbytes(ws), max_polls, _stream(stream)))

@@ -1,0 +1,422 @@
+// The C ABI of libvdn (declared in include/vdn.h): argument checks, workspace plan,
+// and the order in which the layer's kernels are enqueued.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "vdn_internal.cuh"
+
+using namespace vdn;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+vdn_status fail(vdn_status code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+vdn_status ok() {
+  g_err[0] = '\0';
+  return VDN_OK;
+}
+
+vdn_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(VDN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+vdn_status check_shape(const vdn_shape *s) {
+  if (s == nullptr) return fail(VDN_ERR_INVALID_ARG, "shape is NULL");
+  if (s->frames < 1 || s->tokens_per_frame < 1 || s->chunk_frames < 1 || s->text_tokens < 0 || s->heads < 1)
+    return fail(VDN_ERR_INVALID_ARG, "shape out of range (F=%d T=%d C=%d L=%d H=%d)", s->frames,
+                s->tokens_per_frame, s->chunk_frames, s->text_tokens, s->heads);
+  if (s->head_dim != 32 && s->head_dim != 64 && s->head_dim != 128)
+    return fail(VDN_ERR_UNSUPPORTED, "head_dim %d not in {32, 64, 128}", s->head_dim);
+  const int64_t nv = (int64_t)s->frames * s->tokens_per_frame;
+  if (nv + s->text_tokens >= (int64_t)1 << 31 || (int64_t)s->heads * s->head_dim > 65536)
+    return fail(VDN_ERR_INVALID_ARG, "shape too large (F*T + L must stay below 2^31, H*D <= 65536)");
+  return VDN_OK;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+vdn_status need(const void *p, const char *name) {
+  if (p == nullptr) return fail(VDN_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(VDN_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return VDN_OK;
+}
+
+#define VDN_TRY(x)                     \
+  do {                                 \
+    vdn_status _s = (x);               \
+    if (_s != VDN_OK) return _s;       \
+  } while (0)
+
+// sm_100 check, once per device
+vdn_status check_device() {
+  static int cached[64];  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(VDN_ERR_UNSUPPORTED, "device index %d", dev);
+  if (cached[dev] == 0) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  if (cached[dev] != 1) return fail(VDN_ERR_UNSUPPORTED, "libvdn is built for sm_100a (B200) only");
+  return VDN_OK;
+}
+
+vdn_status check_ws(void *ws, size_t ws_bytes, size_t needed) {
+  if (ws == nullptr) return fail(VDN_ERR_WORKSPACE, "workspace is NULL");
+  if (((uintptr_t)ws & (WS_ALIGN - 1)) != 0) return fail(VDN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < needed) return fail(VDN_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, needed);
+  return VDN_OK;
+}
+
+vdn_status check_act_dtype(vdn_dtype dt) {
+  if (dt != VDN_F32 && dt != VDN_BF16) return fail(VDN_ERR_UNSUPPORTED, "dtype %d not supported here", (int)dt);
+  return VDN_OK;
+}
+
+vdn_status check_kind(vdn_lin_kind kind) {
+  if (kind != VDN_LIN_ELU1 && kind != VDN_LIN_DELTA) return fail(VDN_ERR_INVALID_ARG, "unknown kind %d", (int)kind);
+  return VDN_OK;
+}
+
+#define VDN_CUDA(x, what)                               \
+  do {                                                  \
+    cudaError_t _e = (x);                               \
+    if (_e != cudaSuccess) return cuda_fail(_e, what);  \
+  } while (0)
+
+// ---- per-kernel event timing (host state; off unless vdn_profile_begin was called)
+struct Prof {
+  bool on = false;
+  int cap = 0, n = 0;
+  cudaEvent_t *ev = nullptr;  // 2 per launch
+  int *kid = nullptr;
+} g_prof;
+
+void prof_mark(int kid, bool start, cudaStream_t st) {
+  if (!g_prof.on) return;
+  if (start) {
+    if (g_prof.n >= g_prof.cap) return;
+    g_prof.kid[g_prof.n] = kid;
+    cudaEventRecord(g_prof.ev[2 * g_prof.n], st);
+  } else {
+    if (g_prof.n >= g_prof.cap) return;
+    cudaEventRecord(g_prof.ev[2 * g_prof.n + 1], st);
+    ++g_prof.n;
+  }
+}
+
+struct ProfScope {
+  int kid;
+  cudaStream_t st;
+  ProfScope(int k, cudaStream_t s) : kid(k), st(s) { prof_mark(kid, true, st); }
+  ~ProfScope() { prof_mark(kid, false, st); }
+};
+
+float scale_log2_of(float sm_scale, int D) {
+  const float s = sm_scale > 0.f ? sm_scale : 1.f / std::sqrt((float)D);
+  return s * 1.4426950408889634f;
+}
+
+vdn_status softmax_dispatch(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
+                            const void *kt, const void *vt, const float *scales, float sl2, void *o, float *lse,
+                            char *ws, const WsPlan &p, cudaStream_t st) {
+  (void)scales;
+  if (dt == VDN_E4M3) return fail(VDN_ERR_UNSUPPORTED, "e4m3 softmax branch not available");
+  VDN_CUDA(launch_softmax_simt(d, dt, q, k, v, kt, vt, sl2, o, lse, ws, p, st), "softmax branch launch");
+  return VDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int vdn_version(void) { return 100; }
+
+const char *vdn_last_error(void) { return g_err; }
+
+int32_t vdn_max_groups(const vdn_shape *shape) {
+  if (check_shape(shape) != VDN_OK) return 0;
+  return max_groups(shape->frames, shape->chunk_frames);
+}
+
+vdn_status vdn_mask_layout_build(const vdn_shape *shape, int32_t *frame_tab, int32_t *group_tab, int32_t *n_groups,
+                                 size_t group_tab_cap) {
+  VDN_TRY(check_shape(shape));
+  if (frame_tab == nullptr || group_tab == nullptr || n_groups == nullptr)
+    return fail(VDN_ERR_INVALID_ARG, "frame_tab, group_tab and n_groups must be non-NULL");
+  const int cap = group_tab_cap > (size_t)1 << 30 ? 1 << 30 : (int)group_tab_cap;
+  const int G = build_layout(shape->frames, shape->tokens_per_frame, shape->chunk_frames, shape->text_tokens,
+                             frame_tab, group_tab, cap);
+  if (G < 0) return fail(VDN_ERR_INVALID_ARG, "group_tab_cap %zu is below the group count", group_tab_cap);
+  *n_groups = G;
+  return ok();
+}
+
+size_t vdn_hybrid_attn_workspace_size(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype) {
+  if (check_shape(shape) != VDN_OK || check_kind(kind) != VDN_OK) return 0;
+  return plan_workspace(*shape, kind, dtype).total;
+}
+
+size_t vdn_step_workspace_size(const vdn_shape *shape) {
+  if (check_shape(shape) != VDN_OK) return 0;
+  return plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16).step_end;
+}
+
+vdn_status vdn_workspace_init(void *ws, size_t ws_bytes, vdn_stream stream) {
+  VDN_TRY(check_ws(ws, ws_bytes, 256));
+  VDN_CUDA(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream), "workspace init");
+  return ok();
+}
+
+vdn_status vdn_softmax_branch_fwd(const vdn_shape *shape, vdn_dtype dtype, const void *q, const void *k,
+                                  const void *v, const void *kt, const void *vt, const float *scales, float sm_scale,
+                                  void *o_s, float *lse, void *ws, size_t ws_bytes, vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  if (dtype != VDN_F32 && dtype != VDN_BF16 && dtype != VDN_E4M3)
+    return fail(VDN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  VDN_TRY(need(q, "q")); VDN_TRY(need(k, "k")); VDN_TRY(need(v, "v")); VDN_TRY(need(o_s, "o_s"));
+  if (shape->text_tokens > 0) { VDN_TRY(need(kt, "kt")); VDN_TRY(need(vt, "vt")); }
+  if ((dtype == VDN_E4M3) != (scales != nullptr))
+    return fail(VDN_ERR_INVALID_ARG, "scales must be given exactly when dtype is VDN_E4M3");
+  if (!std::isfinite(sm_scale)) return fail(VDN_ERR_INVALID_ARG, "sm_scale is not finite");
+  const WsPlan p = plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16);
+  VDN_TRY(check_ws(ws, ws_bytes, p.step_end));
+  VDN_TRY(check_device());
+  const Dims d = dims_of(*shape);
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(launch_tables(d, (char *)ws, p, st), "tables launch");
+  VDN_TRY(softmax_dispatch(d, dtype, q, k, v, kt, vt, scales, scale_log2_of(sm_scale, d.D), o_s, lse, (char *)ws, p,
+                           st));
+  return ok();
+}
+
+vdn_status vdn_linear_state_build(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *k,
+                                  const void *v, const void *kt, const void *vt, float *S, float *z, float *S_txt,
+                                  float *z_txt, void *ws, size_t ws_bytes, vdn_stream stream) {
+  (void)ws; (void)ws_bytes;
+  VDN_TRY(check_shape(shape));
+  VDN_TRY(check_kind(kind));
+  VDN_TRY(check_act_dtype(dtype));
+  VDN_TRY(need(k, "k")); VDN_TRY(need(v, "v")); VDN_TRY(need(S, "S")); VDN_TRY(need(z, "z"));
+  VDN_TRY(need(S_txt, "S_txt"));
+  if (kind == VDN_LIN_ELU1) VDN_TRY(need(z_txt, "z_txt"));
+  if (shape->text_tokens > 0) { VDN_TRY(need(kt, "kt")); VDN_TRY(need(vt, "vt")); }
+  VDN_TRY(check_device());
+  const Dims d = dims_of(*shape);
+  VDN_CUDA(launch_state_build(d, kind, dtype, k, v, kt, vt, S, z, S_txt, z_txt, (cudaStream_t)stream),
+           "state build launch");
+  return ok();
+}
+
+vdn_status vdn_linear_state_scan(const vdn_shape *shape, vdn_lin_kind kind, const float *S, const float *z,
+                                 const float *S_txt, const float *z_txt, const float *beta, float *S_fwd,
+                                 float *S_bwd, float *z_fwd, float *z_bwd, void *ws, size_t ws_bytes,
+                                 vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  VDN_TRY(check_kind(kind));
+  VDN_TRY(need(S, "S")); VDN_TRY(need(S_txt, "S_txt")); VDN_TRY(need(S_fwd, "S_fwd")); VDN_TRY(need(S_bwd, "S_bwd"));
+  if (kind == VDN_LIN_ELU1) {
+    VDN_TRY(need(z, "z")); VDN_TRY(need(z_txt, "z_txt")); VDN_TRY(need(z_fwd, "z_fwd")); VDN_TRY(need(z_bwd, "z_bwd"));
+  } else {
+    VDN_TRY(need(z, "z (vbar)")); VDN_TRY(need(beta, "beta"));
+  }
+  const WsPlan p = plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16);
+  VDN_TRY(check_ws(ws, ws_bytes, p.step_end));
+  VDN_TRY(check_device());
+  const Dims d = dims_of(*shape);
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(launch_tables(d, (char *)ws, p, st), "tables launch");
+  VDN_CUDA(launch_state_scan(d, kind, S, z, S_txt, z_txt, beta, S_fwd, S_bwd, z_fwd, z_bwd, (char *)ws, p, st),
+           "scan launch");
+  return ok();
+}
+
+vdn_status vdn_linear_read(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *q,
+                           const float *S_fwd, const float *S_bwd, const float *z_fwd, const float *z_bwd, void *o_l,
+                           void *ws, size_t ws_bytes, vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  VDN_TRY(check_kind(kind));
+  VDN_TRY(check_act_dtype(dtype));
+  VDN_TRY(need(q, "q")); VDN_TRY(need(S_fwd, "S_fwd")); VDN_TRY(need(S_bwd, "S_bwd")); VDN_TRY(need(o_l, "o_l"));
+  if (kind == VDN_LIN_ELU1) { VDN_TRY(need(z_fwd, "z_fwd")); VDN_TRY(need(z_bwd, "z_bwd")); }
+  const WsPlan p = plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16);
+  VDN_TRY(check_ws(ws, ws_bytes, p.step_end));
+  VDN_TRY(check_device());
+  const Dims d = dims_of(*shape);
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(launch_tables(d, (char *)ws, p, st), "tables launch");
+  VDN_CUDA(launch_linear_read(d, kind, dtype, q, S_fwd, S_bwd, z_fwd, z_bwd, o_l, (char *)ws, p, st), "read launch");
+  return ok();
+}
+
+vdn_status vdn_hybrid_fuse(const vdn_shape *shape, vdn_dtype dtype, const void *q, const void *o_s, const void *o_l,
+                           const float *w_gate_s, const float *w_gate_l, int32_t G_l, const float *gamma, float eps,
+                           void *a, vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  VDN_TRY(check_act_dtype(dtype));
+  VDN_TRY(need(q, "q")); VDN_TRY(need(o_s, "o_s")); VDN_TRY(need(o_l, "o_l")); VDN_TRY(need(a, "a"));
+  VDN_TRY(need(w_gate_s, "w_gate_s")); VDN_TRY(need(w_gate_l, "w_gate_l")); VDN_TRY(need(gamma, "gamma"));
+  if (G_l != 1 && G_l != shape->head_dim) return fail(VDN_ERR_INVALID_ARG, "G_l must be 1 or D");
+  if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(VDN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  VDN_TRY(check_device());
+  VDN_CUDA(launch_fuse(dims_of(*shape), dtype, q, o_s, o_l, w_gate_s, w_gate_l, G_l, gamma, eps, a,
+                       (cudaStream_t)stream),
+           "fuse launch");
+  return ok();
+}
+
+vdn_status vdn_out_proj(const vdn_shape *shape, vdn_dtype dtype, const void *a, const void *w_os, const void *w_ol,
+                        void *y, vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  VDN_TRY(check_act_dtype(dtype));
+  VDN_TRY(need(a, "a")); VDN_TRY(need(w_os, "w_os")); VDN_TRY(need(w_ol, "w_ol")); VDN_TRY(need(y, "y"));
+  VDN_TRY(check_device());
+  const Dims d = dims_of(*shape);
+  VDN_CUDA(launch_out_proj_simt(d, dtype, a, w_os, w_ol, y, (cudaStream_t)stream), "out-proj launch");
+  return ok();
+}
+
+vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *q,
+                               const void *k, const void *v, const void *kt, const void *vt, const float *beta,
+                               const float *w_gate_s, const float *w_gate_l, int32_t G_l, const float *gamma,
+                               float eps, const void *w_os, const void *w_ol, void *y, void *ws, size_t ws_bytes,
+                               vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  VDN_TRY(check_kind(kind));
+  if (dtype != VDN_F32 && dtype != VDN_BF16 && dtype != VDN_E4M3)
+    return fail(VDN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  VDN_TRY(need(q, "q")); VDN_TRY(need(k, "k")); VDN_TRY(need(v, "v")); VDN_TRY(need(y, "y"));
+  if (shape->text_tokens > 0) { VDN_TRY(need(kt, "kt")); VDN_TRY(need(vt, "vt")); }
+  VDN_TRY(need(w_gate_s, "w_gate_s")); VDN_TRY(need(w_gate_l, "w_gate_l")); VDN_TRY(need(gamma, "gamma"));
+  VDN_TRY(need(w_os, "w_os")); VDN_TRY(need(w_ol, "w_ol"));
+  if (kind == VDN_LIN_DELTA) VDN_TRY(need(beta, "beta"));
+  else if (beta != nullptr) return fail(VDN_ERR_INVALID_ARG, "beta must be NULL for VDN_LIN_ELU1");
+  if (G_l != 1 && G_l != shape->head_dim) return fail(VDN_ERR_INVALID_ARG, "G_l must be 1 or D");
+  if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(VDN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  const WsPlan p = plan_workspace(*shape, kind, dtype);
+  VDN_TRY(check_ws(ws, ws_bytes, p.total));
+  VDN_TRY(check_device());
+  const Dims d = dims_of(*shape);
+  cudaStream_t st = (cudaStream_t)stream;
+  char *w = (char *)ws;
+  const vdn_dtype act = dtype == VDN_E4M3 ? VDN_BF16 : dtype;
+  float *S = (float *)(w + p.S), *z = (float *)(w + p.z), *St = (float *)(w + p.St), *zt = (float *)(w + p.zt);
+  float *Sf = (float *)(w + p.Sf), *Sb = (float *)(w + p.Sb), *zf = (float *)(w + p.zf), *zb = (float *)(w + p.zb);
+  void *Os = w + p.Os, *Ol = w + p.Ol, *A = w + p.A;
+  {
+    ProfScope ps(K_TABLES, st);
+    VDN_CUDA(launch_tables(d, w, p, st), "tables launch");
+  }
+  {
+    ProfScope ps(K_SOFTMAX_SIMT, st);
+    VDN_TRY(softmax_dispatch(d, dtype, q, k, v, kt, vt, nullptr, scale_log2_of(0.f, d.D), Os, nullptr, w, p, st));
+  }
+  {
+    ProfScope ps(K_STATE, st);
+    VDN_CUDA(launch_state_build(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, st),
+             "state build launch");
+  }
+  {
+    ProfScope ps(K_SCAN, st);
+    VDN_CUDA(launch_state_scan(d, kind, S, z, St, zt, beta, Sf, Sb, zf, zb, w, p, st), "scan launch");
+  }
+  {
+    ProfScope ps(K_READ, st);
+    VDN_CUDA(launch_linear_read(d, kind, act, q, Sf, Sb, zf, zb, Ol, w, p, st), "read launch");
+  }
+  {
+    ProfScope ps(K_FUSE, st);
+    VDN_CUDA(launch_fuse(d, act, q, Os, Ol, w_gate_s, w_gate_l, G_l, gamma, eps, A, st), "fuse launch");
+  }
+  {
+    ProfScope ps(K_GEMM_SIMT, st);
+    VDN_CUDA(launch_out_proj_simt(d, act, A, w_os, w_ol, y, st), "out-proj launch");
+  }
+  return ok();
+}
+
+void *vdn_hybrid_attn_intermediate(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, void *ws, int which) {
+  if (check_shape(shape) != VDN_OK || ws == nullptr) return nullptr;
+  const WsPlan p = plan_workspace(*shape, kind, dtype);
+  char *w = (char *)ws;
+  switch (which) {
+    case 0: return w + p.Os;
+    case 1: return w + p.Ol;
+    case 2: return w + p.A;
+    case 3: return w + p.Sf;
+    case 4: return w + p.Sb;
+    case 5: return w + p.ftab;
+    case 6: return w + p.gtab;
+    case 7: return w + p.tiles;
+    case 8: return w + p.meta;
+    default: return nullptr;
+  }
+}
+
+vdn_status vdn_check_device_status(void *ws, size_t ws_bytes, vdn_stream stream) {
+  VDN_TRY(check_ws(ws, ws_bytes, 256));
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(cudaStreamSynchronize(st), "stream synchronize");
+  DevStatus h{};
+  VDN_CUDA(cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost), "status read");
+  VDN_CUDA(cudaMemset(ws, 0, sizeof(h)), "status clear");
+  if (h.code == 0) return ok();
+  const vdn_status code = h.code == VDN_ERR_TIMEOUT ? VDN_ERR_TIMEOUT : VDN_ERR_DEVICE;
+  return fail(code, "device status %u from kernel %u, block %u, detail %u", h.code, h.where, h.block, h.detail);
+}
+
+vdn_status vdn_profile_begin(int32_t max_launches) {
+  if (max_launches < 1 || max_launches > (1 << 20)) return fail(VDN_ERR_INVALID_ARG, "max_launches out of range");
+  if (g_prof.cap < max_launches) {
+    for (int i = 0; i < 2 * g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+    delete[] g_prof.ev;
+    delete[] g_prof.kid;
+    g_prof.ev = new cudaEvent_t[2 * max_launches];
+    g_prof.kid = new int[max_launches];
+    g_prof.cap = 0;
+    for (int i = 0; i < 2 * max_launches; ++i) VDN_CUDA(cudaEventCreate(&g_prof.ev[i]), "event create");
+    g_prof.cap = max_launches;
+  }
+  g_prof.n = 0;
+  g_prof.on = true;
+  return ok();
+}
+
+vdn_status vdn_profile_end(float *ms, int32_t *launches, int32_t n) {
+  if (ms == nullptr || launches == nullptr || n < 1) return fail(VDN_ERR_INVALID_ARG, "bad output arrays");
+  for (int i = 0; i < n; ++i) { ms[i] = 0.f; launches[i] = 0; }
+  g_prof.on = false;
+  for (int i = 0; i < g_prof.n; ++i) {
+    VDN_CUDA(cudaEventSynchronize(g_prof.ev[2 * i + 1]), "event sync");
+    float t = 0.f;
+    VDN_CUDA(cudaEventElapsedTime(&t, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]), "event elapsed");
+    const int k = g_prof.kid[i];
+    if (k >= 0 && k < n) { ms[k] += t; launches[k] += 1; }
+  }
+  g_prof.n = 0;
+  return ok();
+}
+
+vdn_status vdn_debug_unset_flag_wait(void *ws, size_t ws_bytes, uint32_t max_polls, vdn_stream stream) {
+  VDN_TRY(check_ws(ws, ws_bytes, 256));
+  if (max_polls == 0) return fail(VDN_ERR_INVALID_ARG, "max_polls must be >= 1");
+  VDN_TRY(check_device());
+  VDN_CUDA(launch_debug_wait((char *)ws, max_polls, (cudaStream_t)stream), "debug wait launch");
+  return ok();
+}
+
+}  // extern "C"

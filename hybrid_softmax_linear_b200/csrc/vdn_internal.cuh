@@ -1,0 +1,278 @@
+// Internal declarations of libvdn: layout rules (host and device), workspace plan,
+// device status word, element conversions and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/vdn.h"
+
+#define VDN_HD __host__ __device__ __forceinline__
+
+namespace vdn {
+
+// ---------------------------------------------------------------- layout rules
+// Window of a query frame: its chunk and the chunks on either side ("VDN-MiniMax-H3
+// 开源" article, 技术解读 / 局部精确计算 para. 1); chunks start at frame 0.
+VDN_HD void chunk_window(int f, int F, int C, int *lo, int *hi) {
+  int c = f / C;
+  int a = (c - 1) * C, b = (c + 2) * C;
+  *lo = a < 0 ? 0 : a;
+  *hi = b > F ? F : b;
+}
+
+VDN_HD bool is_anchor(int f, int F) { return f == 0 || f == F - 1; }
+
+struct FrameSets {
+  int nseg;
+  int seg[4][2];  // softmax key segments in [text | video] index space
+  int fwd[2];     // forward-memory frames, empty = (0, 0)
+  int bwd[2];     // backward-memory frames, empty = (0, 0)
+  int win[2];
+  int anchor;
+};
+
+// Key sets of query frame f.  Anchors read every frame by softmax and have empty
+// memories; other frames read {0} + window + {F-1} by softmax, the frames in
+// [1, win_lo) through the forward memory and [win_hi, F-1) through the backward one.
+VDN_HD void frame_sets(int f, int F, int T, int C, int L, FrameSets *s) {
+  int lo, hi;
+  s->anchor = is_anchor(f, F) ? 1 : 0;
+  if (s->anchor) { lo = 0; hi = F; } else { chunk_window(f, F, C, &lo, &hi); }
+  s->win[0] = lo; s->win[1] = hi;
+  // candidate token ranges, already in ascending order
+  int cand[4][2];
+  int nc = 0;
+  if (L > 0) { cand[nc][0] = 0; cand[nc][1] = L; ++nc; }
+  if (s->anchor) {
+    cand[nc][0] = L; cand[nc][1] = L + F * T; ++nc;
+  } else {
+    cand[nc][0] = L; cand[nc][1] = L + T; ++nc;                       // frame 0
+    cand[nc][0] = L + lo * T; cand[nc][1] = L + hi * T; ++nc;         // window
+    cand[nc][0] = L + (F - 1) * T; cand[nc][1] = L + F * T; ++nc;     // frame F-1
+  }
+  s->nseg = 0;
+  for (int i = 0; i < 4; ++i) { s->seg[i][0] = 0; s->seg[i][1] = 0; }
+  for (int i = 0; i < nc; ++i) {
+    if (s->nseg > 0 && cand[i][0] <= s->seg[s->nseg - 1][1]) {
+      if (cand[i][1] > s->seg[s->nseg - 1][1]) s->seg[s->nseg - 1][1] = cand[i][1];
+    } else {
+      s->seg[s->nseg][0] = cand[i][0]; s->seg[s->nseg][1] = cand[i][1]; ++s->nseg;
+    }
+  }
+  s->fwd[0] = s->fwd[1] = s->bwd[0] = s->bwd[1] = 0;
+  if (!s->anchor) {
+    int a = 1, b = lo;            // [1, lo): before the window, frame 0 excluded
+    if (b > a) { s->fwd[0] = a; s->fwd[1] = b; }
+    a = hi; b = F - 1;            // [hi, F-1): after the window, frame F-1 excluded
+    if (b > a) { s->bwd[0] = a; s->bwd[1] = b; }
+  }
+}
+
+VDN_HD bool same_sets(const FrameSets &x, const FrameSets &y) {
+  if (x.nseg != y.nseg) return false;
+  for (int i = 0; i < 4; ++i)
+    if (x.seg[i][0] != y.seg[i][0] || x.seg[i][1] != y.seg[i][1]) return false;
+  return x.fwd[0] == y.fwd[0] && x.fwd[1] == y.fwd[1] && x.bwd[0] == y.bwd[0] && x.bwd[1] == y.bwd[1];
+}
+
+VDN_HD int max_groups(int F, int C) { return (F + C - 1) / C + 2; }
+
+// Fills frame_tab [F][8] and group_tab [cap][16]; returns G, or -1 if cap < G.
+VDN_HD int build_layout(int F, int T, int C, int L, int32_t *ftab, int32_t *gtab, int cap) {
+  FrameSets prev, cur;
+  int G = 0;
+  for (int f = 0; f < F; ++f) {
+    frame_sets(f, F, T, C, L, &cur);
+    bool extend = f > 0 && same_sets(cur, prev);
+    if (extend) {
+      gtab[(G - 1) * 16 + 1] = f + 1;
+    } else {
+      if (G >= cap) return -1;
+      int32_t *r = gtab + G * 16;
+      r[0] = f; r[1] = f + 1; r[2] = cur.nseg; r[3] = 0;
+      for (int i = 0; i < 4; ++i) { r[4 + 2 * i] = cur.seg[i][0]; r[5 + 2 * i] = cur.seg[i][1]; }
+      r[12] = cur.fwd[0]; r[13] = cur.fwd[1]; r[14] = cur.bwd[0]; r[15] = cur.bwd[1];
+      ++G;
+    }
+    int32_t *fr = ftab + f * 8;
+    fr[0] = G - 1; fr[1] = cur.win[0]; fr[2] = cur.win[1]; fr[3] = cur.anchor;
+    fr[4] = cur.fwd[0]; fr[5] = cur.fwd[1]; fr[6] = cur.bwd[0]; fr[7] = cur.bwd[1];
+    prev = cur;
+  }
+  return G;
+}
+
+VDN_HD int group_keys(const int32_t *grow) {
+  int n = 0;
+  for (int i = 0; i < grow[2]; ++i) n += grow[5 + 2 * i] - grow[4 + 2 * i];
+  return n;
+}
+
+// ---------------------------------------------------------------- query tiles
+// Query rows are cut into tiles of TILE_M rows that never straddle a group, so every
+// row of a tile shares one key set.  Tiles are listed longest key set first.
+constexpr int TILE_M = 128;
+constexpr int TILE_REC = 4;  // {group, row_lo, row_hi, n_keys}
+
+VDN_HD int64_t max_tiles(int F, int T, int C) {
+  return (int64_t)F * T / TILE_M + max_groups(F, C) + 1;
+}
+
+// ---------------------------------------------------------------- workspace plan
+constexpr size_t WS_ALIGN = 256;
+VDN_HD size_t align_up(size_t x) { return (x + WS_ALIGN - 1) / WS_ALIGN * WS_ALIGN; }
+
+struct WsPlan {
+  // step part (tables, tile list, status)
+  size_t status, ftab, gtab, meta, tiles, step_end;
+  // layer part
+  size_t S, z, St, zt, Sf, Sb, zf, zb, Os, Ol, A, q8, k8, v8, kt8, vt8, scales, amax, total;
+};
+
+// meta: int32[8] = {G, n_tiles, ...}
+inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dtype) {
+  WsPlan p{};
+  size_t F = s.frames, T = s.tokens_per_frame, L = s.text_tokens, H = s.heads, D = s.head_dim;
+  size_t G = (size_t)max_groups(s.frames, s.chunk_frames);
+  size_t Nv = F * T;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+  p.status = take(256);
+  p.ftab = take(F * 8 * 4);
+  p.gtab = take(G * 16 * 4);
+  p.meta = take(64);
+  p.tiles = take((size_t)max_tiles(s.frames, s.tokens_per_frame, s.chunk_frames) * TILE_REC * 4);
+  p.step_end = off;
+  size_t act = (dtype == VDN_F32) ? 4 : 2;
+  // per-frame states: ELU1 S [F][H][D][D]; DELTA kbar [F][H][D] in S, vbar in z
+  p.S = take(kind == VDN_LIN_ELU1 ? F * H * D * D * 4 : F * H * D * 4);
+  p.z = take(F * H * D * 4);
+  p.St = take(H * D * D * 4);
+  p.zt = take(H * D * 4);
+  p.Sf = take(G * H * D * D * 4);
+  p.Sb = take(G * H * D * D * 4);
+  p.zf = take(G * H * D * 4);
+  p.zb = take(G * H * D * 4);
+  p.Os = take(Nv * H * D * act);
+  p.Ol = take(Nv * H * D * act);
+  p.A = take(Nv * 2 * H * D * act);
+  if (dtype == VDN_E4M3) {
+    p.q8 = take(Nv * H * D);
+    p.k8 = take(Nv * H * D);
+    p.v8 = take(Nv * H * D);
+    p.kt8 = take(L * H * D + 16);
+    p.vt8 = take(L * H * D + 16);
+    p.scales = take(3 * H * 4);
+    p.amax = take(3 * H * 4);
+  }
+  p.total = off;
+  return p;
+}
+
+// ---------------------------------------------------------------- device status word
+struct DevStatus {
+  uint32_t code;    // 0 ok, VDN_ERR_TIMEOUT, VDN_ERR_DEVICE
+  uint32_t where;   // kernel id
+  uint32_t block;   // linear block index of the first reporter
+  uint32_t detail;  // kernel-specific
+};
+
+enum KernelId : uint32_t {
+  K_TABLES = 1, K_SOFTMAX_SIMT = 2, K_SOFTMAX_TC = 3, K_STATE = 4, K_SCAN = 5, K_READ = 6,
+  K_FUSE = 7, K_GEMM_SIMT = 8, K_GEMM_TC = 9, K_QUANT = 10, K_DELTA = 11, K_DEBUG_WAIT = 12,
+};
+
+__device__ __forceinline__ void report(DevStatus *st, uint32_t code, uint32_t where, uint32_t detail) {
+  if (atomicCAS(&st->code, 0u, code) == 0u) {
+    st->where = where;
+    st->block = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    st->detail = detail;
+  }
+}
+
+// Bound on device polls of an mbarrier or flag before a kernel gives up (about a
+// second at the polling rates involved).  Settable per call for the wait test.
+constexpr uint32_t DEFAULT_MAX_POLLS = 1u << 26;
+
+// ---------------------------------------------------------------- element access
+template <typename T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
+
+// ---------------------------------------------------------------- launchers
+struct Dims {
+  int F, T, C, L, H, D;
+  __host__ __device__ int64_t Nv() const { return (int64_t)F * T; }
+};
+
+inline Dims dims_of(const vdn_shape &s) {
+  return Dims{s.frames, s.tokens_per_frame, s.chunk_frames, s.text_tokens, s.heads, s.head_dim};
+}
+
+// Group and tile counts from the same rules the device tables kernel runs.
+inline int host_group_count(const Dims &d) {
+  FrameSets prev, cur;
+  int G = 0;
+  for (int f = 0; f < d.F; ++f) {
+    frame_sets(f, d.F, d.T, d.C, d.L, &cur);
+    if (!(f > 0 && same_sets(cur, prev))) ++G;
+    prev = cur;
+  }
+  return G;
+}
+
+inline int host_tile_count(const Dims &d) {
+  FrameSets prev, cur;
+  int64_t n = 0, lo = 0;
+  for (int f = 0; f < d.F; ++f) {
+    frame_sets(f, d.F, d.T, d.C, d.L, &cur);
+    if (f > 0 && !same_sets(cur, prev)) {
+      n += ((int64_t)f * d.T - lo + TILE_M - 1) / TILE_M;
+      lo = (int64_t)f * d.T;
+    }
+    prev = cur;
+  }
+  n += (d.Nv() - lo + TILE_M - 1) / TILE_M;
+  return (int)n;
+}
+
+// tables + tile list into the workspace (device kernel, one block)
+cudaError_t launch_tables(const Dims &d, char *ws, const WsPlan &p, cudaStream_t st);
+
+cudaError_t launch_softmax_simt(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
+                                const void *kt, const void *vt, float scale_log2, void *o, float *lse,
+                                char *ws, const WsPlan &p, cudaStream_t st);
+cudaError_t launch_softmax_tc(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
+                              const void *kt, const void *vt, const float *scales, float scale_log2, void *o,
+                              float *lse, char *ws, const WsPlan &p, cudaStream_t st);
+bool softmax_tc_supported(const Dims &d, vdn_dtype dt);
+
+cudaError_t launch_state_build(const Dims &d, vdn_lin_kind kind, vdn_dtype dt, const void *k, const void *v,
+                               const void *kt, const void *vt, float *S, float *z, float *St, float *zt,
+                               cudaStream_t st);
+cudaError_t launch_state_scan(const Dims &d, vdn_lin_kind kind, const float *S, const float *z, const float *St,
+                              const float *zt, const float *beta, float *Sf, float *Sb, float *zf, float *zb,
+                              char *ws, const WsPlan &p, cudaStream_t st);
+cudaError_t launch_linear_read(const Dims &d, vdn_lin_kind kind, vdn_dtype dt, const void *q, const float *Sf,
+                               const float *Sb, const float *zf, const float *zb, void *o, char *ws,
+                               const WsPlan &p, cudaStream_t st);
+cudaError_t launch_fuse(const Dims &d, vdn_dtype dt, const void *q, const void *os, const void *ol,
+                        const float *wgs, const float *wgl, int G_l, const float *gamma, float eps, void *a,
+                        cudaStream_t st);
+cudaError_t launch_out_proj_simt(const Dims &d, vdn_dtype dt, const void *a, const void *wos, const void *wol,
+                                 void *y, cudaStream_t st);
+cudaError_t launch_out_proj_tc(const Dims &d, const void *a, const void *wos, const void *wol, void *y,
+                               char *ws, const WsPlan &p, cudaStream_t st);
+bool out_proj_tc_supported(const Dims &d);
+cudaError_t launch_debug_wait(char *ws, uint32_t max_polls, cudaStream_t st);
+
+}  // namespace vdn

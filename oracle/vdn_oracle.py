@@ -242,15 +242,14 @@ def linear_memory(k, v, kt, vt, F, T, C):
     S, z = frame_states(k, v, F, T)
     St, zt = text_state(kt, vt)
     H, D = St.shape[0], St.shape[1]
-    num_f = np.zeros((F, H, D, D)); num_b = np.zeros((F, H, D, D))
-    den_f = np.zeros((F, H, D)); den_b = np.zeros((F, H, D))
-    for fq in range(F):
-        fw = np.nonzero(M[fq] == FWD)[0]
-        bw = np.nonzero(M[fq] == BWD)[0]
-        num_f[fq] = 0.5 * St + S[fw].sum(axis=0)
-        num_b[fq] = 0.5 * St + S[bw].sum(axis=0)
-        den_f[fq] = 0.5 * zt + z[fw].sum(axis=0)
-        den_b[fq] = 0.5 * zt + z[bw].sum(axis=0)
+    # sum over the explicit frame set of every query frame: indicator rows times the
+    # stacked per-frame states (one matrix product per memory)
+    w_f = (M == FWD).astype(np.float64)   # w_f[fq, fk] = 1 if fk is in fq's forward set
+    w_b = (M == BWD).astype(np.float64)
+    num_f = 0.5 * St[None] + (w_f @ S.reshape(F, -1)).reshape(F, H, D, D)
+    num_b = 0.5 * St[None] + (w_b @ S.reshape(F, -1)).reshape(F, H, D, D)
+    den_f = 0.5 * zt[None] + (w_f @ z.reshape(F, -1)).reshape(F, H, D)
+    den_b = 0.5 * zt[None] + (w_b @ z.reshape(F, -1)).reshape(F, H, D)
     return num_f, num_b, den_f, den_b
 
 
@@ -260,12 +259,14 @@ def linear_read(q, num_f, num_b, den_f, den_b, T, rows=None):
     halves add up to one ([ART] para. 2-3, R5); 0 where the normaliser is 0 (R7)."""
     N, H, D = q.shape
     rows = np.arange(N) if rows is None else np.asarray(rows)
-    fq = rows // T
-    pq = phi(q[rows])                                                    # [n, H, D]
-    num = np.einsum("nhd,nhde->nhe", pq, num_f[fq] + num_b[fq])
-    den = np.einsum("nhd,nhd->nh", pq, den_f[fq] + den_b[fq])[..., None]
-    safe = np.where(den > 0, den, 1.0)
-    return np.where(den > 0, num / safe, 0.0)
+    out = np.zeros((rows.size, H, D))
+    for f in np.unique(rows // T):
+        sel = np.nonzero(rows // T == f)[0]
+        pq = phi(q[rows[sel]])                                              # [n, H, D]
+        num = np.einsum("nhd,hde->nhe", pq, num_f[f] + num_b[f])
+        den = np.einsum("nhd,hd->nh", pq, den_f[f] + den_b[f])[..., None]
+        out[sel] = np.where(den > 0, num / np.where(den > 0, den, 1.0), 0.0)
+    return out
 
 
 def linear_branch(q, k, v, kt, vt, F, T, C, rows=None):
@@ -354,9 +355,11 @@ def delta_read(q, Sf, Sb, T, rows=None):
     """o = (S_f + S_b)^T q_hat with q_hat = q / ||q|| (R12, R13)."""
     N, H, D = q.shape
     rows = np.arange(N) if rows is None else np.asarray(rows)
-    fq = rows // T
-    qh = l2_normalize(q[rows])
-    return np.einsum("nhde,nhd->nhe", Sf[fq] + Sb[fq], qh)
+    out = np.zeros((rows.size, H, D))
+    for f in np.unique(rows // T):
+        sel = np.nonzero(rows // T == f)[0]
+        out[sel] = np.einsum("hde,nhd->nhe", Sf[f] + Sb[f], l2_normalize(q[rows[sel]]))
+    return out
 
 
 def delta_branch(q, k, v, kt, vt, beta, F, T, C, rows=None):

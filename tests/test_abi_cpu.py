@@ -1,0 +1,116 @@
+"""CPU checks of the C ABI: the library loads without a GPU, exports every entry point
+that include/vdn.h declares, builds layout tables identical to the oracle's, and rejects
+bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import hybrid_softmax_linear_b200 as vdn
+from hybrid_softmax_linear_b200 import synth
+from oracle import vdn_oracle as vo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "vdn.h"), encoding="utf-8").read()
+    return sorted(set(re.findall(r"VDN_API[^;(]*?\b(vdn_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 17
+    L = ctypes.CDLL(vdn.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(vdn._SIGS), "binding and header disagree"
+
+
+def test_version():
+    assert vdn.version() >= 100
+
+
+SHAPES = [(15, 16, 1, 4, 2, 32), (30, 256, 5, 64, 8, 64), (60, 1008, 5, 256, 24, 128), (90, 1008, 5, 512, 40, 128),
+          (87, 1008, 5, 512, 40, 128), (1, 4, 5, 3, 1, 32), (2, 5, 5, 0, 1, 32), (3, 7, 1, 0, 1, 64),
+          (16, 1, 2, 1, 1, 32), (11, 100, 2, 0, 2, 64), (40, 3, 6, 9, 1, 32), (13, 5, 13, 2, 1, 32)]
+
+
+@pytest.mark.parametrize("sh", SHAPES)
+def test_layout_bit_exact_vs_oracle(sh):
+    F, T, C, L, H, D = sh
+    ftab, gtab = vdn.mask_layout_build(synth.Shape(F, T, C, L, H, D))
+    oft, ogt = vo.layout_tables(F, T, C, L)
+    np.testing.assert_array_equal(ftab, oft)
+    np.testing.assert_array_equal(gtab, ogt)
+    assert len(gtab) <= vdn.max_groups(synth.Shape(F, T, C, L, H, D))
+
+
+def test_layout_all_small_shapes_vs_oracle():
+    for F in range(1, 41):
+        for C in range(1, 7):
+            for T, L in ((1, 0), (3, 2)):
+                ftab, gtab = vdn.mask_layout_build(synth.Shape(F, T, C, L, 1, 32))
+                oft, ogt = vo.layout_tables(F, T, C, L)
+                assert np.array_equal(ftab, oft) and np.array_equal(gtab, ogt), (F, C, T, L)
+
+
+def test_layout_capacity_error():
+    s = synth.Shape(90, 1008, 5, 512, 40, 128)
+    with pytest.raises(vdn.VdnError) as e:
+        vdn.mask_layout_build(s, cap=3)
+    assert e.value.status == 1
+
+
+@pytest.mark.parametrize("bad", [(0, 16, 1, 4, 2, 32), (15, 0, 1, 4, 2, 32), (15, 16, 0, 4, 2, 32),
+                                 (15, 16, 1, -1, 2, 32), (15, 16, 1, 4, 0, 32)])
+def test_bad_shape_rejected(bad):
+    with pytest.raises(vdn.VdnError) as e:
+        vdn.mask_layout_build(vdn.Shape(*bad), cap=64)
+    assert e.value.status == 1
+
+
+def test_unsupported_head_dim():
+    with pytest.raises(vdn.VdnError) as e:
+        vdn.mask_layout_build(vdn.Shape(15, 16, 1, 4, 2, 48), cap=64)
+    assert e.value.status == 2
+
+
+def test_workspace_sizes():
+    s = synth.Shape(90, 1008, 5, 512, 40, 128)
+    step = vdn.step_workspace_size(s)
+    full = vdn.hybrid_attn_workspace_size(s, vdn.ELU1, vdn.BF16)
+    assert 0 < step < full
+    # the layer keeps O_s, O_l and A (bf16) plus per-frame and per-group fp32 states
+    nv, hd = 90 * 1008, 40 * 128
+    assert full >= nv * hd * 2 * 4
+    assert vdn.hybrid_attn_workspace_size(s, vdn.DELTA, vdn.E4M3) > 0
+
+
+def test_argument_checks_precede_cuda():
+    """Null pointers and small workspaces are reported without a device."""
+    s = vdn.Shape(15, 16, 1, 4, 2, 32)
+    L = vdn.lib()
+    st = L.vdn_softmax_branch_fwd(ctypes.byref(s), vdn.F32, None, 16, 16, 16, 16, None, 0.0, 16, None, 256, 1 << 20,
+                                  None)
+    assert st == 1 and b"q" in L.vdn_last_error()
+    st = L.vdn_softmax_branch_fwd(ctypes.byref(s), vdn.F32, 16, 16, 16, 16, 16, None, 0.0, 16, None, 256, 16, None)
+    assert st == 3
+    st = L.vdn_softmax_branch_fwd(ctypes.byref(s), vdn.F32, 16, 16, 16, 16, 16, None, 0.0, 16, None, 100, 1 << 20,
+                                  None)
+    assert st == 3  # misaligned workspace
+    st = L.vdn_softmax_branch_fwd(ctypes.byref(s), vdn.F32, 24, 16, 16, 16, 16, None, 0.0, 16, None, 256, 1 << 20,
+                                  None)
+    assert st == 1  # misaligned q
+    st = L.vdn_softmax_branch_fwd(ctypes.byref(s), vdn.F32, 16, 16, 16, 16, 16, 16, 0.0, 16, None, 256, 1 << 20, None)
+    assert st == 1  # scales with a non-fp8 dtype
+    st = L.vdn_hybrid_fuse(ctypes.byref(s), vdn.BF16, 16, 16, 16, 16, 16, 7, 16, 1e-6, 16, None)
+    assert st == 1  # G_l not in {1, D}
+    st = L.vdn_hybrid_attn_fwd(ctypes.byref(s), vdn.ELU1, vdn.F32, 16, 16, 16, 16, 16, 16, 16, 16, 32, 16, 1e-6, 16,
+                               16, 16, 256, 1 << 30, None)
+    assert st == 1  # beta given for ELU1
+    st = L.vdn_hybrid_attn_fwd(ctypes.byref(s), 7, vdn.F32, 16, 16, 16, 16, 16, None, 16, 16, 32, 16, 1e-6, 16, 16,
+                               16, 256, 1 << 30, None)
+    assert st == 1  # unknown kind
