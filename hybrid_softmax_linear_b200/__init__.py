@@ -67,7 +67,7 @@ _SIGS = {
     "vdn_linear_read": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                        _vp]),
     "vdn_hybrid_fuse": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _f32, _vp, _vp]),
-    "vdn_out_proj": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]),
+    "vdn_out_proj": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "vdn_hybrid_attn_fwd": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                            _i32, _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "vdn_hybrid_attn_intermediate": (_vp, [_SP, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int]),
@@ -183,9 +183,9 @@ def hybrid_fuse(shape, dtype, q, o_s, o_l, w_gate_s, w_gate_l, G_l, gamma, eps, 
                                  _p(w_gate_l), G_l, _p(gamma), eps, _p(a), _stream(stream)))
 
 
-def out_proj(shape, dtype, a, w_os, w_ol, y, stream=None):
-    _check(lib().vdn_out_proj(ctypes.byref(Shape.of(shape)), dtype, _p(a), _p(w_os), _p(w_ol), _p(y),
-                              _stream(stream)))
+def out_proj(shape, dtype, a, w_os, w_ol, y, ws, stream=None):
+    _check(lib().vdn_out_proj(ctypes.byref(Shape.of(shape)), dtype, _p(a), _p(w_os), _p(w_ol), _p(y), _p(ws),
+                              _nbytes(ws), _stream(stream)))
 
 
 def hybrid_attn_fwd(shape, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma, eps, w_os, w_ol, y,

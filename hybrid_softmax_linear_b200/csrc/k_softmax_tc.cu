@@ -1,0 +1,369 @@
+// Softmax branch on the 5th-generation tensor cores: block-sparse flash attention over
+// the key set of each query group ("VDN-MiniMax-H3 开源" article, 技术解读 /
+// 局部精确计算: the chunk window, both anchor frames and every text token; the model
+// card calls it the window softmax).
+//
+// One CTA owns 256 query rows of one group and one head, as two 128-row tiles Q0, Q1
+// that share every K/V tile.  Warp 0 streams Q once and the group's K/V tiles (128 keys,
+// text first, then the merged video segments) with TMA into 2-stage rings.  One thread
+// of warp 1 issues tcgen05.mma: S_w = Q_w K_j^T (M=128, N=128) into tensor memory, then,
+// once softmax warpgroup w has written P_w (bf16, over S_w's columns) and rescaled its
+// output, O_w += P_w V_j (A operand from tensor memory, V as an MN-major operand).
+// Warpgroups 0 and 1 (warps 2-5 and 6-9) run the online softmax of Q0 and Q1, one row
+// per thread, so while one warpgroup exponentiates, the tensor cores work for the
+// other.  The running maximum is only moved (and O rescaled) when it grows by more than
+// 2^8; the final normalisation uses the same stale maximum, so the result is exact.
+// Keys past the end of a segment are masked in the last tile of that segment.
+#include "tc_common.cuh"
+
+namespace vdn {
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128;     // rows per Q tile
+constexpr int BN = 128;     // keys per K/V tile
+constexpr int NQ = 2;       // Q tiles per CTA
+constexpr int KST = 2, VST = 2;
+constexpr int THREADS = 320;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int BOXES = D / 64;                 // 64-column (128-byte) boxes per row
+  static constexpr int TILE_BYTES = BM * D * 2;        // one 128 x D bf16 tile
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + NQ * TILE_BYTES;
+  static constexpr int V_OFF = K_OFF + KST * TILE_BYTES;
+  static constexpr int BAR_OFF = V_OFF + VST * TILE_BYTES;
+  static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
+  static constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);
+  static constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);
+  // tensor memory columns
+  static constexpr uint32_t S_COL[2] = {0, 128};
+  static constexpr uint32_t O_COL[2] = {256, 384};
+};
+
+struct alignas(8) Bars {
+  uint64_t q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[NQ], p_full[NQ], o_done, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// The key tiles of a group: text rows first, then video rows, each merged segment of the
+// group cut into 128-key tiles.
+struct KvParts {
+  int n;
+  int text[5], lo[5], hi[5];
+};
+
+__device__ __forceinline__ void kv_parts(const int32_t *g, int L, KvParts &p) {
+  p.n = 0;
+  for (int s = 0; s < g[2]; ++s) {
+    const int lo = g[4 + 2 * s], hi = g[5 + 2 * s];
+    if (lo < L) { p.text[p.n] = 1; p.lo[p.n] = lo; p.hi[p.n] = hi < L ? hi : L; ++p.n; }
+    if (hi > L) { p.text[p.n] = 0; p.lo[p.n] = (lo > L ? lo : L) - L; p.hi[p.n] = hi - L; ++p.n; }
+  }
+}
+
+__device__ __forceinline__ int kv_tiles(const KvParts &p) {
+  int n = 0;
+  for (int i = 0; i < p.n; ++i) n += (p.hi[i] - p.lo[i] + BN - 1) / BN;
+  return n;
+}
+
+// cursor over the tiles: part index and row of the current tile
+struct KvCursor {
+  int part, row;
+  __device__ void init(const KvParts &p) { part = 0; row = p.lo[0]; }
+  __device__ void next(const KvParts &p) {
+    row += BN;
+    if (row >= p.hi[part]) { ++part; if (part < p.n) row = p.lo[part]; }
+  }
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int D>
+__global__ void __launch_bounds__(THREADS, 1)
+    softmax_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
+                      const __grid_constant__ CUtensorMap tmVt, Dims d, float sl2, __nv_bfloat16 *__restrict__ out,
+                      float *__restrict__ lse, const int32_t *__restrict__ gtab, const int32_t *__restrict__ tiles,
+                      DevStatus *st) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  Bars *bars = reinterpret_cast<Bars *>(base + C::BAR_OFF);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int *abort_flag = &bars->abort;
+
+  const int h = blockIdx.x % d.H;
+  const int32_t *tr = tiles + (int64_t)(blockIdx.x / d.H) * TILE_REC;
+  const int g = tr[0], row0 = tr[1], row_end = tr[2];
+  const int32_t *grow = gtab + g * 16;
+  KvParts parts;
+  kv_parts(grow, d.L, parts);
+  const int nkv = kv_tiles(parts);
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int s = 0; s < KST; ++s) { mbar_init(smem_u32(&bars->k_full[s]), 1); mbar_init(smem_u32(&bars->k_empty[s]), 1); }
+    for (int s = 0; s < VST; ++s) { mbar_init(smem_u32(&bars->v_full[s]), 1); mbar_init(smem_u32(&bars->v_empty[s]), 1); }
+    for (int w = 0; w < NQ; ++w) { mbar_init(smem_u32(&bars->s_full[w]), 1); mbar_init(smem_u32(&bars->p_full[w]), 4); }
+    mbar_init(smem_u32(&bars->o_done), 1);
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+    tma_prefetch(&tmQ); tma_prefetch(&tmK); tma_prefetch(&tmV); tma_prefetch(&tmKt); tma_prefetch(&tmVt);
+  }
+  if (warp == 1) { tmem_alloc(smem_u32(&bars->tmem_base), TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      uint32_t armed_k = 0, ph_k = 0, armed_v = 0, ph_v = 0;
+      const uint32_t qb = smem_u32(&bars->q_full);
+      mbar_arrive_expect_tx(qb, NQ * C::TILE_BYTES);
+      for (int w = 0; w < NQ; ++w)
+        for (int c = 0; c < C::BOXES; ++c)
+          tma_load_2d(smem_u32(base + C::Q_OFF + w * C::TILE_BYTES + c * BM * 128), &tmQ, qb, h * D + c * 64,
+                      row0 + w * BM);
+      KvCursor cur;
+      cur.init(parts);
+      for (int j = 0; j < nkv; ++j) {
+        const int ks = j % KST, vs = j % VST;
+        const CUtensorMap *mk = parts.text[cur.part] ? &tmKt : &tmK;
+        const CUtensorMap *mv = parts.text[cur.part] ? &tmVt : &tmV;
+        if (!mbar_wait(smem_u32(&bars->k_empty[ks]), ((j / KST) & 1) ^ 1, abort_flag, st, K_SOFTMAX_TC, 1)) break;
+        const uint32_t kb = smem_u32(&bars->k_full[ks]);
+        mbar_arrive_expect_tx(kb, C::TILE_BYTES);
+        for (int c = 0; c < C::BOXES; ++c)
+          tma_load_2d(smem_u32(base + C::K_OFF + ks * C::TILE_BYTES + c * BN * 128), mk, kb, h * D + c * 64, cur.row);
+        armed_k |= 1u << ks;
+        ph_k = (ph_k & ~(1u << ks)) | (((j / KST) & 1u) << ks);
+        if (!mbar_wait(smem_u32(&bars->v_empty[vs]), ((j / VST) & 1) ^ 1, abort_flag, st, K_SOFTMAX_TC, 2)) break;
+        const uint32_t vb = smem_u32(&bars->v_full[vs]);
+        mbar_arrive_expect_tx(vb, C::TILE_BYTES);
+        for (int c = 0; c < C::BOXES; ++c)
+          tma_load_2d(smem_u32(base + C::V_OFF + vs * C::TILE_BYTES + c * BN * 128), mv, vb, h * D + c * 64, cur.row);
+        armed_v |= 1u << vs;
+        ph_v = (ph_v & ~(1u << vs)) | (((j / VST) & 1u) << vs);
+        cur.next(parts);
+      }
+      // loads issued here land before the block leaves (bounded waits)
+      int no_abort = 0;
+      mbar_wait(qb, 0, &no_abort, st, K_SOFTMAX_TC, 10);
+      for (int s = 0; s < KST; ++s)
+        if (armed_k & (1u << s)) mbar_wait(smem_u32(&bars->k_full[s]), (ph_k >> s) & 1u, &no_abort, st, K_SOFTMAX_TC, 11);
+      for (int s = 0; s < VST; ++s)
+        if (armed_v & (1u << s)) mbar_wait(smem_u32(&bars->v_full[s]), (ph_v >> s) & 1u, &no_abort, st, K_SOFTMAX_TC, 12);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t qa = smem_u32(base + C::Q_OFF);
+      auto issue_s = [&](int w, int j) {
+        const uint32_t kbase = smem_u32(base + C::K_OFF + (j % KST) * C::TILE_BYTES);
+        const uint32_t abase = qa + w * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          mma_ss(tmem + C::S_COL[w], sdesc(abase + off, 16, 1024), sdesc(kbase + off, 16, 1024), C::IDESC_S, kk > 0);
+        }
+        mma_commit(smem_u32(&bars->s_full[w]));
+      };
+      bool ok = mbar_wait(smem_u32(&bars->q_full), 0, abort_flag, st, K_SOFTMAX_TC, 3);
+      if (ok) ok = mbar_wait(smem_u32(&bars->k_full[0]), 0, abort_flag, st, K_SOFTMAX_TC, 4);
+      if (ok) {
+        tc_fence_after();
+        for (int w = 0; w < NQ; ++w) issue_s(w, 0);
+        mma_commit(smem_u32(&bars->k_empty[0]));
+      }
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int vs = j % VST;
+        if (!mbar_wait(smem_u32(&bars->v_full[vs]), (j / VST) & 1, abort_flag, st, K_SOFTMAX_TC, 5)) break;
+        const bool more = j + 1 < nkv;
+        if (more && !mbar_wait(smem_u32(&bars->k_full[(j + 1) % KST]), ((j + 1) / KST) & 1, abort_flag, st,
+                               K_SOFTMAX_TC, 6))
+          break;
+        const uint32_t vbase = smem_u32(base + C::V_OFF + vs * C::TILE_BYTES);
+        for (int w = 0; w < NQ && ok; ++w) {
+          if (!mbar_wait(smem_u32(&bars->p_full[w]), j & 1, abort_flag, st, K_SOFTMAX_TC, 7)) { ok = false; break; }
+          tc_fence_after();
+          // O_w += P_w V_j: P_w (bf16, two per column) sits over the first 64 columns of S_w
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts(tmem + C::O_COL[w], tmem + C::S_COL[w] + kk * 8, sdesc(vbase + kk * 2048, BM * 128, 1024),
+                   C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          if (more) issue_s(w, j + 1);
+        }
+        mma_commit(smem_u32(&bars->v_empty[vs]));
+        if (more) mma_commit(smem_u32(&bars->k_empty[(j + 1) % KST]));
+      }
+      mma_commit(smem_u32(&bars->o_done));
+      mma_commit(smem_u32(&bars->drain));
+      int no_abort = 0;
+      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_SOFTMAX_TC, 8);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int w = (warp - 2) >> 2;          // Q tile of this warpgroup
+    const int quad = warp & 3;              // tensor-memory lane quadrant
+    const int r = quad * 32 + lane;         // row within the Q tile
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + C::S_COL[w];
+    const uint32_t o_addr = tmem + lane_off + C::O_COL[w];
+    float m = -INFINITY, l = 0.f;
+    KvCursor cur;
+    cur.init(parts);
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const int nvalid = min(BN, parts.hi[cur.part] - cur.row);
+      cur.next(parts);
+      if (!mbar_wait(smem_u32(&bars->s_full[w]), j & 1, abort_flag, st, K_SOFTMAX_TC, 9)) { ok = false; break; }
+      tc_fence_after();
+      float s[BN];
+#pragma unroll
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(s_addr + c, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(u[i]);
+      }
+      if (nvalid < BN) {
+#pragma unroll
+        for (int i = 0; i < BN; ++i)
+          if (i >= nvalid) s[i] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < BN; ++i) mx = fmaxf(mx, s[i]);
+      const float m_new = fmaxf(m, mx * sl2);
+      const bool need = __any_sync(0xffffffffu, m_new > m + RESCALE_THRESHOLD);
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2(m - m_new);   // 0 on the first tile (m = -inf)
+        m = m_new;
+      }
+      float rs = 0.f;
+      const float neg_m = -m;
+#pragma unroll
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(fmaf(s[c + 2 * i], sl2, neg_m));
+          const float p1 = ex2(fmaf(s[c + 2 * i + 1], sl2, neg_m));
+          rs += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        tmem_st16(s_addr + (c >> 1), pk);
+      }
+      if (need && j > 0) {
+        // O_w was last written by P V of tile j-1, which completed before S_w of tile j
+#pragma unroll 1
+        for (int c = 0; c < D; c += 16) {
+          uint32_t u[16];
+          tmem_ld16(o_addr + c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          tmem_st16(o_addr + c, u);
+        }
+      }
+      l = l * alpha + rs;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[w]));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && mbar_wait(smem_u32(&bars->o_done), 0, abort_flag, st, K_SOFTMAX_TC, 13)) {
+      tc_fence_after();
+      const int row = row0 + w * BM + r;
+      const bool valid = row < row_end;
+      const float inv = 1.f / l;
+      __nv_bfloat16 *orow = out + ((int64_t)row * d.H + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(o_addr + c, u);
+        tmem_wait_ld();
+        if (valid) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 o;
+            o.x = pack_bf16(__uint_as_float(u[8 * v + 0]) * inv, __uint_as_float(u[8 * v + 1]) * inv);
+            o.y = pack_bf16(__uint_as_float(u[8 * v + 2]) * inv, __uint_as_float(u[8 * v + 3]) * inv);
+            o.z = pack_bf16(__uint_as_float(u[8 * v + 4]) * inv, __uint_as_float(u[8 * v + 5]) * inv);
+            o.w = pack_bf16(__uint_as_float(u[8 * v + 6]) * inv, __uint_as_float(u[8 * v + 7]) * inv);
+            dst[v] = o;
+          }
+        }
+      }
+      if (valid && lse != nullptr) lse[(int64_t)row * d.H + h] = (m + __log2f(l)) * 0.69314718055994530942f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+template <int D>
+cudaError_t launch_t(const Dims &d, const void *q, const void *k, const void *v, const void *kt, const void *vt,
+                     float sl2, void *o, float *lse, char *ws, const WsPlan &p, cudaStream_t st) {
+  using C = Cfg<D>;
+  const uint64_t HD = (uint64_t)d.H * D;
+  CUtensorMap mq, mk, mv, mkt, mvt;
+  uint64_t strides[1] = {HD * 2};
+  uint32_t box[2] = {64, BM};
+  uint64_t dims_v[2] = {HD, (uint64_t)d.Nv()};
+  uint64_t dims_t[2] = {HD, (uint64_t)(d.L > 0 ? d.L : 1)};
+  const void *kt_base = d.L > 0 ? kt : k, *vt_base = d.L > 0 ? vt : v;  // unused when there is no text
+  if (!encode_tmap(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mkt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kt_base, dims_t, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mvt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vt_base, dims_t, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(softmax_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int ntiles = host_tile_count(d);
+  softmax_tc_kernel<D><<<ntiles * d.H, THREADS, C::SMEM, st>>>(
+      mq, mk, mv, mkt, mvt, d, sl2, (__nv_bfloat16 *)o, lse, (const int32_t *)(ws + p.gtab),
+      (const int32_t *)(ws + p.tiles), (DevStatus *)(ws + p.status));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool softmax_tc_supported(const Dims &d, vdn_dtype dt) {
+  return dt == VDN_BF16 && (d.D == 64 || d.D == 128);
+}
+
+cudaError_t launch_softmax_tc(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
+                              const void *kt, const void *vt, const float *scales, float sl2, void *o, float *lse,
+                              char *ws, const WsPlan &p, cudaStream_t st) {
+  (void)scales;
+  if (dt != VDN_BF16) return cudaErrorInvalidValue;
+  if (d.D == 128) return launch_t<128>(d, q, k, v, kt, vt, sl2, o, lse, ws, p, st);
+  if (d.D == 64) return launch_t<64>(d, q, k, v, kt, vt, sl2, o, lse, ws, p, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vdn

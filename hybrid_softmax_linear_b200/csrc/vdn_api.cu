@@ -140,6 +140,18 @@ vdn_status softmax_dispatch(const Dims &d, vdn_dtype dt, const void *q, const vo
   return VDN_OK;
 }
 
+vdn_status out_proj_dispatch(const Dims &d, vdn_dtype act, const void *a, const void *w_os, const void *w_ol, void *y,
+                             char *ws, const WsPlan &p, cudaStream_t st) {
+  if (act == VDN_BF16 && out_proj_tc_supported(d)) {
+    ProfScope ps(K_GEMM_TC, st);
+    VDN_CUDA(launch_out_proj_tc(d, a, w_os, w_ol, y, ws, p, st), "out-proj (tensor cores) launch");
+  } else {
+    ProfScope ps(K_GEMM_SIMT, st);
+    VDN_CUDA(launch_out_proj_simt(d, act, a, w_os, w_ol, y, st), "out-proj launch");
+  }
+  return VDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -280,13 +292,14 @@ vdn_status vdn_hybrid_fuse(const vdn_shape *shape, vdn_dtype dtype, const void *
 }
 
 vdn_status vdn_out_proj(const vdn_shape *shape, vdn_dtype dtype, const void *a, const void *w_os, const void *w_ol,
-                        void *y, vdn_stream stream) {
+                        void *y, void *ws, size_t ws_bytes, vdn_stream stream) {
   VDN_TRY(check_shape(shape));
   VDN_TRY(check_act_dtype(dtype));
   VDN_TRY(need(a, "a")); VDN_TRY(need(w_os, "w_os")); VDN_TRY(need(w_ol, "w_ol")); VDN_TRY(need(y, "y"));
+  const WsPlan p = plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16);
+  VDN_TRY(check_ws(ws, ws_bytes, p.step_end));
   VDN_TRY(check_device());
-  const Dims d = dims_of(*shape);
-  VDN_CUDA(launch_out_proj_simt(d, dtype, a, w_os, w_ol, y, (cudaStream_t)stream), "out-proj launch");
+  VDN_TRY(out_proj_dispatch(dims_of(*shape), dtype, a, w_os, w_ol, y, (char *)ws, p, (cudaStream_t)stream));
   return ok();
 }
 
@@ -342,10 +355,7 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
     ProfScope ps(K_FUSE, st);
     VDN_CUDA(launch_fuse(d, act, q, Os, Ol, w_gate_s, w_gate_l, G_l, gamma, eps, A, st), "fuse launch");
   }
-  {
-    ProfScope ps(K_GEMM_SIMT, st);
-    VDN_CUDA(launch_out_proj_simt(d, act, A, w_os, w_ol, y, st), "out-proj launch");
-  }
+  VDN_TRY(out_proj_dispatch(d, act, A, w_os, w_ol, y, w, p, st));
   return ok();
 }
 

@@ -182,9 +182,10 @@ VDN_API vdn_status vdn_hybrid_fuse(const vdn_shape *shape, vdn_dtype dtype, cons
 /* vdn_out_proj — separate output projections of the two branches, summed.  [ART]
  * 独立门控 para. 1.  y[N_v][HD] = A[:, :HD] W_os^T + A[:, HD:] W_ol^T, with W_os, W_ol
  * [HD (out)][HD (in)] row-major; no bias (the residual add is the caller's).  dtype
- * VDN_F32 or VDN_BF16 for a, w and y (fp32 accumulation). */
+ * VDN_F32 or VDN_BF16 for a, w and y (fp32 accumulation).  ws: vdn_step_workspace_size
+ * bytes (its status word receives bounded-wait timeouts of the tensor-core kernel). */
 VDN_API vdn_status vdn_out_proj(const vdn_shape *shape, vdn_dtype dtype, const void *a, const void *w_os,
-                        const void *w_ol, void *y, vdn_stream stream);
+                                const void *w_ol, void *y, void *ws, size_t ws_bytes, vdn_stream stream);
 
 /* ------------------------------------------------------------------ whole layer
  * vdn_hybrid_attn_fwd — the layer: both branches, fuse and projections, in one call.

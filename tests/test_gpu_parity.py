@@ -195,7 +195,7 @@ def test_step_entry_points_match_oracle():
     ref_a = vo.hybrid_fuse(o["q"], to_numpy(o_s), to_numpy(o_l), o["w_gate_s"], o["w_gate_l"], o["gamma"], 1e-6)
     assert_close("hybrid_fuse", to_numpy(a), ref_a, "bf16")
     y = empty((Nv, H * D), "bf16")
-    vdn.out_proj(s, vdn.BF16, a, d["w_os"], d["w_ol"], y)
+    vdn.out_proj(s, vdn.BF16, a, d["w_os"], d["w_ol"], y, ws)
     assert_close("out_proj", to_numpy(y), vo.out_proj(to_numpy(a), o["w_os"], o["w_ol"]), "bf16")
     vdn.check_device_status(ws)
 
