@@ -90,6 +90,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   Bars *bars = reinterpret_cast<Bars *>(base + STAGES * STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int *abort_flag = &bars->abort;
+  __shared__ int skip;  // an earlier block gave up: do no more work (block-uniform decision)
+  if (threadIdx.x == 0) skip = *(volatile uint32_t *)&st->code != 0u;
+  __syncthreads();
+  if (skip) return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(smem_u32(&bars->full[s]), 1); mbar_init(smem_u32(&bars->empty[s]), 1); }
@@ -169,7 +173,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       int m, n;
       tile_coords(t, num_m, num_n, m, n);
-      if (!mbar_wait(smem_u32(&bars->tfull[b]), tph, abort_flag, st, K_GEMM_TC, 5)) break;
+      // the warp proceeds (or gives up) as a whole: tensor-memory loads are warp-collective
+      const bool got = mbar_wait(smem_u32(&bars->tfull[b]), tph, abort_flag, st, K_GEMM_TC, 5);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const int row = m * BM + q * 32 + lane;
       __nv_bfloat16 *yr = y + (int64_t)row * N + n * BN;

@@ -40,9 +40,9 @@ struct Cfg {
   static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
   static constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);
-  // tensor memory columns
-  static constexpr uint32_t S_COL[2] = {0, 128};
-  static constexpr uint32_t O_COL[2] = {256, 384};
+  // tensor memory columns: S_0, S_1, O_0, O_1
+  __device__ static constexpr uint32_t s_col(int w) { return (uint32_t)w * 128u; }
+  __device__ static constexpr uint32_t o_col(int w) { return 256u + (uint32_t)w * 128u; }
 };
 
 struct alignas(8) Bars {
@@ -102,6 +102,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   Bars *bars = reinterpret_cast<Bars *>(base + C::BAR_OFF);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int *abort_flag = &bars->abort;
+  __shared__ int skip;  // an earlier block gave up: do no more work (block-uniform decision)
+  if (threadIdx.x == 0) skip = *(volatile uint32_t *)&st->code != 0u;
+  __syncthreads();
+  if (skip) return;
 
   const int h = blockIdx.x % d.H;
   const int32_t *tr = tiles + (int64_t)(blockIdx.x / d.H) * TILE_REC;
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          mma_ss(tmem + C::S_COL[w], sdesc(abase + off, 16, 1024), sdesc(kbase + off, 16, 1024), C::IDESC_S, kk > 0);
+          mma_ss(tmem + C::s_col(w), sdesc(abase + off, 16, 1024), sdesc(kbase + off, 16, 1024), C::IDESC_S, kk > 0);
         }
         mma_commit(smem_u32(&bars->s_full[w]));
       };
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           // O_w += P_w V_j: P_w (bf16, two per column) sits over the first 64 columns of S_w
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            mma_ts(tmem + C::O_COL[w], tmem + C::S_COL[w] + kk * 8, sdesc(vbase + kk * 2048, BM * 128, 1024),
+            mma_ts(tmem + C::o_col(w), tmem + C::s_col(w) + kk * 8, sdesc(vbase + kk * 2048, BM * 128, 1024),
                    C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
           if (more) issue_s(w, j + 1);
         }
@@ -221,8 +225,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quad = warp & 3;              // tensor-memory lane quadrant
     const int r = quad * 32 + lane;         // row within the Q tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + C::S_COL[w];
-    const uint32_t o_addr = tmem + lane_off + C::O_COL[w];
+    const uint32_t s_addr = tmem + lane_off + C::s_col(w);
+    const uint32_t o_addr = tmem + lane_off + C::o_col(w);
     float m = -INFINITY, l = 0.f;
     KvCursor cur;
     cur.init(parts);
@@ -230,7 +234,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int j = 0; j < nkv; ++j) {
       const int nvalid = min(BN, parts.hi[cur.part] - cur.row);
       cur.next(parts);
-      if (!mbar_wait(smem_u32(&bars->s_full[w]), j & 1, abort_flag, st, K_SOFTMAX_TC, 9)) { ok = false; break; }
+      // the warp proceeds (or gives up) as a whole: tensor-memory access is warp-collective
+      const bool got = mbar_wait(smem_u32(&bars->s_full[w]), j & 1, abort_flag, st, K_SOFTMAX_TC, 9);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
       float s[BN];
 #pragma unroll
@@ -289,7 +295,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[w]));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && mbar_wait(smem_u32(&bars->o_done), 0, abort_flag, st, K_SOFTMAX_TC, 13)) {
+    const bool done = ok && mbar_wait(smem_u32(&bars->o_done), 0, abort_flag, st, K_SOFTMAX_TC, 13);
+    if (__all_sync(0xffffffffu, done)) {
       tc_fence_after();
       const int row = row0 + w * BM + r;
       const bool valid = row < row_end;

@@ -57,6 +57,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0u) {
       if (*abort_flag) return false;
+      if (*(volatile uint32_t *)&st->code != 0u) {  // another block already gave up
+        *abort_flag = 1;
+        return false;
+      }
       if (globaltimer() - t0 > WAIT_LIMIT_NS) {
         *abort_flag = 1;
         report(st, VDN_ERR_TIMEOUT, where, detail);

@@ -134,9 +134,15 @@ float scale_log2_of(float sm_scale, int D) {
 vdn_status softmax_dispatch(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
                             const void *kt, const void *vt, const float *scales, float sl2, void *o, float *lse,
                             char *ws, const WsPlan &p, cudaStream_t st) {
-  (void)scales;
   if (dt == VDN_E4M3) return fail(VDN_ERR_UNSUPPORTED, "e4m3 softmax branch not available");
-  VDN_CUDA(launch_softmax_simt(d, dt, q, k, v, kt, vt, sl2, o, lse, ws, p, st), "softmax branch launch");
+  if (softmax_tc_supported(d, dt)) {
+    ProfScope ps(K_SOFTMAX_TC, st);
+    VDN_CUDA(launch_softmax_tc(d, dt, q, k, v, kt, vt, scales, sl2, o, lse, ws, p, st),
+             "softmax branch (tensor cores) launch");
+  } else {
+    ProfScope ps(K_SOFTMAX_SIMT, st);
+    VDN_CUDA(launch_softmax_simt(d, dt, q, k, v, kt, vt, sl2, o, lse, ws, p, st), "softmax branch launch");
+  }
   return VDN_OK;
 }
 
@@ -334,10 +340,7 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
     ProfScope ps(K_TABLES, st);
     VDN_CUDA(launch_tables(d, w, p, st), "tables launch");
   }
-  {
-    ProfScope ps(K_SOFTMAX_SIMT, st);
-    VDN_TRY(softmax_dispatch(d, dtype, q, k, v, kt, vt, nullptr, scale_log2_of(0.f, d.D), Os, nullptr, w, p, st));
-  }
+  VDN_TRY(softmax_dispatch(d, dtype, q, k, v, kt, vt, nullptr, scale_log2_of(0.f, d.D), Os, nullptr, w, p, st));
   {
     ProfScope ps(K_STATE, st);
     VDN_CUDA(launch_state_build(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, st),

@@ -115,7 +115,7 @@ VDN_HD int group_keys(const int32_t *grow) {
 // ---------------------------------------------------------------- query tiles
 // Query rows are cut into tiles of TILE_M rows that never straddle a group, so every
 // row of a tile shares one key set.  Tiles are listed longest key set first.
-constexpr int TILE_M = 128;
+constexpr int TILE_M = 256;
 constexpr int TILE_REC = 4;  // {group, row_lo, row_hi, n_keys}
 
 VDN_HD int64_t max_tiles(int F, int T, int C) {

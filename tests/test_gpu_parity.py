@@ -39,7 +39,7 @@ def _check_tables(run: Run):
     tiles = run.intermediate(7, (n, 4), torch.int32).cpu().numpy()
     covered = np.zeros(s.n_video, np.int32)
     for g, lo, hi, keys in tiles:
-        assert 0 < hi - lo <= 128
+        assert 0 < hi - lo <= 256
         flo, fhi = gtab[g][0] * s.tokens_per_frame, gtab[g][1] * s.tokens_per_frame
         assert flo <= lo < hi <= fhi
         assert keys == sum(gtab[g][5 + 2 * i] - gtab[g][4 + 2 * i] for i in range(gtab[g][2]))
