@@ -73,6 +73,8 @@ _SIGS = {
     "vdn_hybrid_attn_intermediate": (_vp, [_SP, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int]),
     "vdn_check_device_status": (ctypes.c_int, [_vp, _sz, _vp]),
     "vdn_debug_unset_flag_wait": (ctypes.c_int, [_vp, _sz, _u32, _vp]),
+    "vdn_softmax_branch_fwd_noalloc": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp,
+                                                      _vp]),
     "vdn_profile_begin": (ctypes.c_int, [_i32]),
     "vdn_profile_end": (ctypes.c_int, [_vp, _vp, _i32]),
 }
@@ -159,6 +161,13 @@ def softmax_branch_fwd(shape, dtype, q, k, v, kt, vt, o_s, ws, scales=None, sm_s
     _check(lib().vdn_softmax_branch_fwd(ctypes.byref(Shape.of(shape)), dtype, _p(q), _p(k), _p(v), _p(kt), _p(vt),
                                         _p(scales), sm_scale, _p(o_s), _p(lse), _p(ws), _nbytes(ws),
                                         _stream(stream)))
+
+
+def softmax_branch_fwd_noalloc(shape, dtype, q, k, v, kt, vt, o_s, sm_scale=0.0, lse=None, stream=None):
+    """Softmax branch without a workspace: the library's fixed device scratch array is
+    used instead (for callers that cannot allocate device memory)."""
+    _check(lib().vdn_softmax_branch_fwd_noalloc(ctypes.byref(Shape.of(shape)), dtype, _p(q), _p(k), _p(v), _p(kt),
+                                                _p(vt), sm_scale, _p(o_s), _p(lse), _stream(stream)))
 
 
 def linear_state_build(shape, kind, dtype, k, v, kt, vt, S, z, S_txt, z_txt, ws=None, stream=None):

@@ -160,6 +160,11 @@ vdn_status out_proj_dispatch(const Dims &d, vdn_dtype act, const void *a, const 
 
 }  // namespace
 
+namespace vdn {
+// lets entry points defined in other files report through vdn_last_error()
+void set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace vdn
+
 extern "C" {
 
 int vdn_version(void) { return 100; }

@@ -131,6 +131,29 @@ VDN_API vdn_status vdn_softmax_branch_fwd(const vdn_shape *shape, vdn_dtype dtyp
                                   float sm_scale, void *o_s, float *lse, void *ws, size_t ws_bytes,
                                   vdn_stream stream);
 
+/* vdn_softmax_branch_fwd_noalloc — the same softmax branch without a workspace.  The
+ * pages have no counterpart: this is a library convenience for callers that cannot
+ * allocate device memory, for example plug-ins that only receive tensors from a host
+ * framework that owns all device memory, or code that must not allocate once running.
+ * Such a caller cannot size and pass a workspace, so this call keeps its scratch
+ * (status word, layout tables, query-tile list) in a fixed 256 KiB array that the
+ * library holds in device memory on every GPU that loads it, until the process exits.
+ * Nothing is allocated or freed: no cudaMalloc, no cudaFree, no allocating library call.
+ *   - Arguments and results as vdn_softmax_branch_fwd, for dtype VDN_F32 or VDN_BF16.
+ *   - Shapes whose tables and tile list need more than the 256 KiB (about 16k query
+ *     tiles of 256 rows) are rejected with VDN_ERR_WORKSPACE.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents; each call
+ *     clears the status word and rewrites the tables before its kernels run.  Calls
+ *     that overlap on the GPU (other streams, other host threads) race on the array and
+ *     must be serialised by the caller.
+ *   - Device-side wait timeouts are recorded in the array's status word but not
+ *     reported: the call never synchronises.  Launch errors are returned. */
+VDN_API vdn_status vdn_softmax_branch_fwd_noalloc(const vdn_shape *shape, vdn_dtype dtype, const void *q,
+                                                  const void *k, const void *v, const void *kt, const void *vt,
+                                                  float sm_scale, void *o_s, float *lse, vdn_stream stream);
+
 /* ------------------------------------------------------------------ linear branch
  * vdn_linear_state_build — per-frame states.  [ART] 局部精确计算 para. 1 (frame-wise
  * linear branch) and para. 3 (text written into the memories).
