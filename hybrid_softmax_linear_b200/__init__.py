@@ -81,7 +81,8 @@ _SIGS = {
 
 PROF_KERNELS = 16
 KERNEL_NAMES = {1: "tables", 2: "softmax_simt", 3: "softmax_tc", 4: "state_build", 5: "scan", 6: "read", 7: "fuse",
-                8: "out_proj_simt", 9: "out_proj_tc", 10: "fp8_quant", 11: "delta_stats"}
+                8: "out_proj_simt", 9: "out_proj_tc", 10: "fp8_quant", 11: "delta_stats", 13: "state_build_tc",
+                14: "read_stage", 15: "read_tc"}
 
 
 def lib() -> ctypes.CDLL:
@@ -170,10 +171,9 @@ def softmax_branch_fwd_noalloc(shape, dtype, q, k, v, kt, vt, o_s, sm_scale=0.0,
                                                 _p(vt), sm_scale, _p(o_s), _p(lse), _stream(stream)))
 
 
-def linear_state_build(shape, kind, dtype, k, v, kt, vt, S, z, S_txt, z_txt, ws=None, stream=None):
+def linear_state_build(shape, kind, dtype, k, v, kt, vt, S, z, S_txt, z_txt, ws, stream=None):
     _check(lib().vdn_linear_state_build(ctypes.byref(Shape.of(shape)), kind, dtype, _p(k), _p(v), _p(kt), _p(vt),
-                                        _p(S), _p(z), _p(S_txt), _p(z_txt), _p(ws),
-                                        0 if ws is None else _nbytes(ws), _stream(stream)))
+                                        _p(S), _p(z), _p(S_txt), _p(z_txt), _p(ws), _nbytes(ws), _stream(stream)))
 
 
 def linear_state_scan(shape, kind, S, z, S_txt, z_txt, beta, S_fwd, S_bwd, z_fwd, z_bwd, ws, stream=None):

@@ -1,0 +1,514 @@
+// Linear branch on the 5th-generation tensor cores (bf16 inputs, head dim 128).
+// ("VDN-MiniMax-H3 开源" article, 技术解读 / 局部精确计算: a frame-wise linear branch
+// whose forward and backward memories are read at the query position; 独立门控: the
+// linear output is RMS-normalised and gated element-wise.)
+//
+// state_build_tc: S_f = phi(K_f)^T V_f and z_f = sum phi(K_f) for one (frame or text,
+//   head) per CTA.  TMA streams 64-token K/V tiles into a 3-stage ring; four warps apply
+//   phi = elu+1 in place in shared memory (masking tokens past the frame) and sum z;
+//   one thread issues tcgen05.mma with both operands MN-major (M = key feature, N =
+//   value dim, K = tokens) into a 128x128 fp32 accumulator in tensor memory.
+// read_stage: S_fwd + S_bwd of every group summed into bf16 (the MMA B operand), the
+//   normalisers summed, the linear-gate weights converted to bf16.
+// read_tc: 256 query rows of one group and head per CTA (two 128-row halves).  Four
+//   warps per half write phi(q) (or q/|q| for the delta rule) next to q in shared memory
+//   and the normaliser phi(q).z; one thread issues num = phi(Q) S_sum and, for the fused
+//   layer, the gate logits Q W_l; the same warps then form o = num / den and either
+//   store o or the gated, RMS-normalised A_l straight into the linear half of A.
+#include "tc_common.cuh"
+
+namespace vdn {
+namespace {
+
+using namespace tc;
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// 16-byte chunk `cl` (8 bf16 of columns 8cl..8cl+7) of row r in a tile stored as
+// 64-column boxes of `box_rows` rows with the 128-byte swizzle
+__device__ __forceinline__ uint32_t swz_off(int r, int cl, int box_rows) {
+  return (uint32_t)((cl >> 3) * box_rows * 128 + r * 128 + ((((cl & 7) ^ (r & 7))) << 4));
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(h[i]);
+    f[2 * i] = x.x; f[2 * i + 1] = x.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float *f) {
+  uint4 u;
+  u.x = pack_bf16(f[0], f[1]); u.y = pack_bf16(f[2], f[3]); u.z = pack_bf16(f[4], f[5]); u.w = pack_bf16(f[6], f[7]);
+  return u;
+}
+
+// ============================================================================ state build
+namespace sb {
+constexpr int D = 128, TK = 64, NS = 3, THREADS = 192;
+constexpr int BOX_BYTES = TK * 128;        // 64 tokens x 64 bf16
+constexpr int TILE_BYTES = 2 * BOX_BYTES;  // 64 tokens x 128 features
+constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+constexpr uint32_t IDESC = idesc_bf16(128, 128, true, true);
+struct alignas(8) Bars {
+  uint64_t full[NS], phi[NS], empty[NS], acc, drain;
+  uint32_t tmem;
+  int abort;
+  float zred[D];
+};
+constexpr size_t SMEM = 1024 + NS * STAGE_BYTES + sizeof(Bars);
+}  // namespace sb
+
+__global__ void __launch_bounds__(sb::THREADS, 2)
+    state_build_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                          const __grid_constant__ CUtensorMap tmKt, const __grid_constant__ CUtensorMap tmVt, Dims d,
+                          float *__restrict__ S, float *__restrict__ z, float *__restrict__ St,
+                          float *__restrict__ zt, DevStatus *st) {
+  using namespace sb;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  Bars *bars = reinterpret_cast<Bars *>(base + NS * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int *abort_flag = &bars->abort;
+  __shared__ int skip;
+  if (threadIdx.x == 0) skip = *(volatile uint32_t *)&st->code != 0u;
+  __syncthreads();
+  if (skip) return;
+
+  const int h = blockIdx.y;
+  const bool text = (int)blockIdx.x == d.F;
+  const int ntok = text ? d.L : d.T;
+  const int row_base = text ? 0 : (int)blockIdx.x * d.T;
+  const int nch = (ntok + TK - 1) / TK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_u32(&bars->full[s]), 1);
+      mbar_init(smem_u32(&bars->phi[s]), 4);
+      mbar_init(smem_u32(&bars->empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->acc), 1);
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < D) bars->zred[threadIdx.x] = 0.f;
+  if (warp == 1) { tmem_alloc(smem_u32(&bars->tmem), 128); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem;
+  const CUtensorMap *mk = text ? &tmKt : &tmK;
+  const CUtensorMap *mv = text ? &tmVt : &tmV;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t armed = 0, armed_ph = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NS;
+        if (!mbar_wait(smem_u32(&bars->empty[s]), ((c / NS) & 1) ^ 1, abort_flag, st, K_STATE, 1)) break;
+        const uint32_t fb = smem_u32(&bars->full[s]);
+        mbar_arrive_expect_tx(fb, STAGE_BYTES);
+        uint8_t *stg = base + s * STAGE_BYTES;
+        for (int b = 0; b < 2; ++b) {
+          tma_load_2d(smem_u32(stg + b * BOX_BYTES), mk, fb, h * D + b * 64, row_base + c * TK);
+          tma_load_2d(smem_u32(stg + TILE_BYTES + b * BOX_BYTES), mv, fb, h * D + b * 64, row_base + c * TK);
+        }
+        armed |= 1u << s;
+        armed_ph = (armed_ph & ~(1u << s)) | (((c / NS) & 1u) << s);
+      }
+      int no_abort = 0;
+      for (int s = 0; s < NS; ++s)
+        if (armed & (1u << s)) mbar_wait(smem_u32(&bars->full[s]), (armed_ph >> s) & 1u, &no_abort, st, K_STATE, 2);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NS;
+        if (!mbar_wait(smem_u32(&bars->phi[s]), (c / NS) & 1, abort_flag, st, K_STATE, 3)) break;
+        tc_fence_after();
+        const uint32_t kb = smem_u32(base + s * STAGE_BYTES), vb = kb + TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < TK / 16; ++kk)
+          mma_ss(tmem, sdesc(kb + kk * 2048, BOX_BYTES, 1024), sdesc(vb + kk * 2048, BOX_BYTES, 1024), IDESC,
+                 (c | kk) != 0);
+        mma_commit(smem_u32(&bars->empty[s]));
+      }
+      mma_commit(smem_u32(&bars->acc));
+      mma_commit(smem_u32(&bars->drain));
+      int no_abort = 0;
+      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_STATE, 4);
+    }
+  } else {
+    // ---------------- phi pass (in place, masked) and z; then the epilogue
+    const int tid = threadIdx.x - 64;
+    const int cl = tid & 15, rg = tid >> 4;  // column chunk 8cl..8cl+7; rows rg + 8i
+    float zacc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nch; ++c) {
+      const int s = c % NS;
+      const bool got = mbar_wait(smem_u32(&bars->full[s]), (c / NS) & 1, abort_flag, st, K_STATE, 5);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      uint8_t *kt = base + s * STAGE_BYTES;
+#pragma unroll
+      for (int i = 0; i < TK / 8; ++i) {
+        const int r = rg + 8 * i;
+        uint4 *p = reinterpret_cast<uint4 *>(kt + swz_off(r, cl, TK));
+        float f[8];
+        unpack8(*p, f);
+        const bool valid = c * TK + r < ntok;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float ph = valid ? (f[e] > 0.f ? f[e] + 1.f : expf(f[e])) : 0.f;
+          zacc[e] += ph;
+          f[e] = ph;
+        }
+        *p = pack8(f);
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->phi[s]));
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) atomicAdd(&bars->zred[cl * 8 + e], zacc[e]);
+    const int quad = warp & 3;
+    const int i = quad * 32 + lane;  // key feature = accumulator row = tensor-memory lane
+    float *So = text ? St + (int64_t)h * D * D : S + ((int64_t)blockIdx.x * d.H + h) * D * D;
+    if (nch > 0) {
+      const bool done = ok && mbar_wait(smem_u32(&bars->acc), 0, abort_flag, st, K_STATE, 6);
+      if (__all_sync(0xffffffffu, done)) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t u[32];
+          tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + cc, u);
+          tmem_wait_ld();
+          float4 *dst = reinterpret_cast<float4 *>(So + i * D + cc);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(u[4 * v]), __uint_as_float(u[4 * v + 1]),
+                                 __uint_as_float(u[4 * v + 2]), __uint_as_float(u[4 * v + 3]));
+        }
+      }
+    } else {
+      for (int cc = 0; cc < D; ++cc) So[i * D + cc] = 0.f;
+    }
+    named_bar_sync(1, 128);  // every phi thread has added its share of z
+    float *zo = text ? zt : z;
+    if (zo != nullptr) zo[(text ? (int64_t)h * D : ((int64_t)blockIdx.x * d.H + h) * D) + tid] = bars->zred[tid];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 128);
+}
+
+// ============================================================================ read staging
+__global__ void __launch_bounds__(256) read_stage_kernel(int64_t n_s8, int64_t n_z, int64_t n_w8,
+                                                         const float *__restrict__ Sf, const float *__restrict__ Sb,
+                                                         const float *__restrict__ zf, const float *__restrict__ zb,
+                                                         const float *__restrict__ wgl, __nv_bfloat16 *__restrict__ ssum,
+                                                         float *__restrict__ zsum, __nv_bfloat16 *__restrict__ wl) {
+  const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (i < n_s8) {
+    const float4 *a = reinterpret_cast<const float4 *>(Sf + 8 * i), *b = reinterpret_cast<const float4 *>(Sb + 8 * i);
+    const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
+    const float f[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
+                        a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
+    *reinterpret_cast<uint4 *>(ssum + 8 * i) = pack8(f);
+  } else if (i < n_s8 + n_z) {
+    const int64_t j = i - n_s8;
+    zsum[j] = zf[j] + zb[j];
+  } else if (i < n_s8 + n_z + n_w8) {
+    const int64_t j = i - n_s8 - n_z;
+    const float4 *a = reinterpret_cast<const float4 *>(wgl + 8 * j);
+    const float4 a0 = a[0], a1 = a[1];
+    const float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    *reinterpret_cast<uint4 *>(wl + 8 * j) = pack8(f);
+  }
+}
+
+// ============================================================================ read (+ gate, RMSNorm)
+namespace rd {
+constexpr int D = 128, BM = 128, NQ = 2, THREADS = 320;
+constexpr int TILE_BYTES = BM * D * 2;  // 32 KB: one 128-row bf16 tile (two 64-column boxes)
+constexpr int Q_OFF = 0, F_OFF = NQ * TILE_BYTES, S_OFF = 2 * NQ * TILE_BYTES, W_OFF = S_OFF + TILE_BYTES;
+constexpr int BAR_OFF = W_OFF + TILE_BYTES;
+constexpr uint32_t IDESC_NUM = idesc_bf16(BM, D, false, true);   // A K-major, B MN-major
+struct alignas(8) Bars {
+  uint64_t in_full, feat[NQ], acc[NQ], drain;
+  uint32_t tmem;
+  int abort;
+};
+constexpr size_t SMEM = 1024 + BAR_OFF + sizeof(Bars);
+}  // namespace rd
+
+__global__ void __launch_bounds__(rd::THREADS, 1)
+    read_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
+                   const __grid_constant__ CUtensorMap tmW, Dims d, int delta, int gate_mma,
+                   const float *__restrict__ zsum, const float *__restrict__ wgl, int G_l,
+                   const float *__restrict__ gamma, float eps, __nv_bfloat16 *__restrict__ out, int64_t out_stride,
+                   int fused, const int32_t *__restrict__ tiles, DevStatus *st) {
+  using namespace rd;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  Bars *bars = reinterpret_cast<Bars *>(base + BAR_OFF);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int *abort_flag = &bars->abort;
+  __shared__ int skip;
+  if (threadIdx.x == 0) skip = *(volatile uint32_t *)&st->code != 0u;
+  __syncthreads();
+  if (skip) return;
+
+  const int h = blockIdx.y;
+  const int32_t *tr = tiles + (int64_t)blockIdx.x * TILE_REC;
+  const int g = tr[0], row0 = tr[1], row_end = tr[2];
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->in_full), 1);
+    for (int w = 0; w < NQ; ++w) { mbar_init(smem_u32(&bars->feat[w]), 4); mbar_init(smem_u32(&bars->acc[w]), 1); }
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) { tmem_alloc(smem_u32(&bars->tmem), 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem;  // num_w at 128w, gate logits of half w at 256 + 128w
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t fb = smem_u32(&bars->in_full);
+      mbar_arrive_expect_tx(fb, (NQ + 1 + (gate_mma ? 1 : 0)) * TILE_BYTES);
+      for (int w = 0; w < NQ; ++w)
+        for (int b = 0; b < 2; ++b)
+          tma_load_2d(smem_u32(base + Q_OFF + w * TILE_BYTES + b * BM * 128), &tmQ, fb, h * D + b * 64, row0 + w * BM);
+      for (int b = 0; b < 2; ++b) {
+        tma_load_2d(smem_u32(base + S_OFF + b * BM * 128), &tmS, fb, b * 64, (g * d.H + h) * D);
+        if (gate_mma) tma_load_2d(smem_u32(base + W_OFF + b * BM * 128), &tmW, fb, b * 64, h * D);
+      }
+      int no_abort = 0;
+      mbar_wait(fb, 0, &no_abort, st, K_READ, 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(smem_u32(&bars->in_full), 0, abort_flag, st, K_READ, 2);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t sb_ = smem_u32(base + S_OFF), wb = smem_u32(base + W_OFF);
+        if (gate_mma) {
+          for (int w = 0; w < NQ; ++w) {
+            const uint32_t qa = smem_u32(base + Q_OFF + w * TILE_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + 256 + 128 * w, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
+                     sdesc(wb + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
+          }
+        }
+        for (int w = 0; w < NQ && ok; ++w) {
+          if (!mbar_wait(smem_u32(&bars->feat[w]), 0, abort_flag, st, K_READ, 3)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t fa = smem_u32(base + F_OFF + w * TILE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + 128 * w, sdesc(fa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc(sb_ + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
+          mma_commit(smem_u32(&bars->acc[w]));
+        }
+      }
+      mma_commit(smem_u32(&bars->drain));
+      int no_abort = 0;
+      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_READ, 4);
+    }
+  } else {
+    const int w = (warp - 2) >> 2, quad = warp & 3, r = quad * 32 + lane;
+    const int row = row0 + w * BM + r;
+    const bool valid = row < row_end;
+    const uint8_t *qt = base + Q_OFF + w * TILE_BYTES;
+    uint8_t *ft = base + F_OFF + w * TILE_BYTES;
+    const bool got = mbar_wait(smem_u32(&bars->in_full), 0, abort_flag, st, K_READ, 5);
+    bool ok = __all_sync(0xffffffffu, got);
+    float den = 0.f, scal_gate = 0.f, inv_norm = 1.f;
+    if (ok) {
+      // feature of this row: phi(q) (and the normaliser phi(q).z), or q/|q| (delta rule)
+      const float *zg = zsum + ((int64_t)g * d.H + h) * D;
+      const float *wg1 = wgl + (int64_t)h * D * G_l;
+      if (delta) {
+        float ss = 0.f;
+#pragma unroll 4
+        for (int cl = 0; cl < D / 8; ++cl) {
+          float f[8];
+          unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+        }
+        inv_norm = ss > 0.f ? rsqrtf(ss) : 0.f;
+      }
+#pragma unroll 2
+      for (int cl = 0; cl < D / 8; ++cl) {
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
+        if (fused && !gate_mma) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) scal_gate = fmaf(f[e], __ldg(wg1 + (cl * 8 + e) * G_l), scal_gate);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (delta) {
+            f[e] *= inv_norm;
+          } else {
+            f[e] = f[e] > 0.f ? f[e] + 1.f : expf(f[e]);
+            den = fmaf(f[e], __ldg(zg + cl * 8 + e), den);
+          }
+        }
+        *reinterpret_cast<uint4 *>(ft + swz_off(r, cl, BM)) = pack8(f);
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->feat[w]));
+      const bool done = mbar_wait(smem_u32(&bars->acc[w]), 0, abort_flag, st, K_READ, 6);
+      ok = __all_sync(0xffffffffu, done);
+    }
+    if (ok) {
+      tc_fence_after();
+      const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+      float o[D];
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_off + 128 * w + c, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[c + i] = __uint_as_float(u[i]);
+      }
+      const float scale = delta ? 1.f : (den > 0.f ? 1.f / den : 0.f);
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < D; ++j) { o[j] *= scale; ss = fmaf(o[j], o[j], ss); }
+      __nv_bfloat16 *orow = out + (int64_t)row * out_stride + (int64_t)h * D;
+      if (!fused) {
+        if (valid) {
+#pragma unroll
+          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4 *>(orow + c) = pack8(o + c);
+        }
+      } else {
+        const float rinv = rsqrtf(ss / (float)D + eps);
+        const float gs = 1.f / (1.f + expf(-scal_gate));
+        const float *gm = gamma + (int64_t)h * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float gl[32];
+          if (gate_mma) {
+            uint32_t u[32];
+            tmem_ld32(tmem + lane_off + 256 + 128 * w + c, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) gl[i] = 1.f / (1.f + expf(-__uint_as_float(u[i])));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) gl[i] = gs;
+          }
+          if (valid) {
+#pragma unroll
+            for (int v = 0; v < 32; v += 8) {
+              float a[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) a[e] = gl[v + e] * __ldg(gm + c + v + e) * o[c + v + e] * rinv;
+              *reinterpret_cast<uint4 *>(orow + c + v) = pack8(a);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+bool linear_tc_supported(const Dims &d, vdn_dtype dt) { return dt == VDN_BF16 && d.D == 128; }
+
+cudaError_t launch_state_build_tc(const Dims &d, const void *k, const void *v, const void *kt, const void *vt,
+                                  float *S, float *z, float *St, float *zt, char *ws, const WsPlan &p,
+                                  cudaStream_t st) {
+  using namespace sb;
+  const uint64_t HD = (uint64_t)d.H * D;
+  CUtensorMap mk, mv, mkt, mvt;
+  uint64_t strides[1] = {HD * 2};
+  uint32_t box[2] = {64, TK};
+  uint64_t dims_v[2] = {HD, (uint64_t)d.Nv()};
+  uint64_t dims_t[2] = {HD, (uint64_t)(d.L > 0 ? d.L : 1)};
+  const void *ktb = d.L > 0 ? kt : k, *vtb = d.L > 0 ? vt : v;
+  if (!encode_tmap(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mkt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ktb, dims_t, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mvt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vtb, dims_t, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(state_build_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+  if (e != cudaSuccess) return e;
+  state_build_tc_kernel<<<dim3(d.F + 1, d.H), THREADS, SMEM, st>>>(mk, mv, mkt, mvt, d, S, z, St, zt,
+                                                                   (DevStatus *)(ws + p.status));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf, const float *Sb, const float *zf,
+                              const float *zb, const float *wgl, int G_l, char *ws, const WsPlan &p,
+                              cudaStream_t st) {
+  const int64_t G = host_group_count(d), DD = (int64_t)d.D * d.D;
+  const int64_t n_s8 = G * d.H * DD / 8;
+  const int64_t n_z = kind == VDN_LIN_ELU1 ? G * d.H * d.D : 0;
+  const int64_t n_w8 = (wgl != nullptr && G_l == d.D) ? (int64_t)d.H * DD / 8 : 0;
+  const int64_t n = n_s8 + n_z + n_w8;
+  read_stage_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+      n_s8, n_z, n_w8, Sf, Sb, zf, zb, wgl, (__nv_bfloat16 *)(ws + p.ssum), (float *)(ws + p.zsum),
+      (__nv_bfloat16 *)(ws + p.wl));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void *out, const float *wgl, int G_l,
+                           const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st) {
+  using namespace rd;
+  const uint64_t HD = (uint64_t)d.H * D;
+  const int G = host_group_count(d);
+  const bool fused = wgl != nullptr;
+  const bool gate_mma = fused && G_l == D;
+  CUtensorMap mq, ms, mw;
+  {
+    uint64_t dims[2] = {HD, (uint64_t)d.Nv()}, strides[1] = {HD * 2};
+    uint32_t box[2] = {64, BM};
+    if (!encode_tmap(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t dims[2] = {(uint64_t)D, (uint64_t)G * d.H * D}, strides[1] = {(uint64_t)D * 2};
+    uint32_t box[2] = {64, (uint32_t)D};
+    if (!encode_tmap(&ms, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.ssum, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    uint64_t dimsw[2] = {(uint64_t)D, (uint64_t)d.H * D};
+    if (!encode_tmap(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.wl, dimsw, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(read_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+  if (e != cudaSuccess) return e;
+  const int64_t stride = fused ? 2 * (int64_t)HD : (int64_t)HD;
+  __nv_bfloat16 *o = (__nv_bfloat16 *)out + (fused ? HD : 0);  // fused: the linear half of A
+  read_tc_kernel<<<dim3(host_tile_count(d), d.H), THREADS, SMEM, st>>>(
+      mq, ms, mw, d, kind == VDN_LIN_DELTA, gate_mma ? 1 : 0, (const float *)(ws + p.zsum),
+      fused ? wgl : nullptr, G_l, gamma, eps, o, stride, fused ? 1 : 0, (const int32_t *)(ws + p.tiles),
+      (DevStatus *)(ws + p.status));
+  return cudaGetLastError();
+}
+
+}  // namespace vdn

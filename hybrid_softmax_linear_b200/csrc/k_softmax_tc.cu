@@ -94,8 +94,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     softmax_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
                       const __grid_constant__ CUtensorMap tmVt, Dims d, float sl2, __nv_bfloat16 *__restrict__ out,
-                      float *__restrict__ lse, const int32_t *__restrict__ gtab, const int32_t *__restrict__ tiles,
-                      DevStatus *st) {
+                      int64_t out_row_stride, const float *__restrict__ w_gate_s, float *__restrict__ lse,
+                      const int32_t *__restrict__ gtab, const int32_t *__restrict__ tiles, DevStatus *st) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -107,8 +107,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if (skip) return;
 
-  const int h = blockIdx.x % d.H;
-  const int32_t *tr = tiles + (int64_t)(blockIdx.x / d.H) * TILE_REC;
+  // Blocks [H*first, H*(first+count)) belong to the group whose tiles are first..first+count-1
+  // in the tile list; inside that range the head varies slowest, so the blocks that run
+  // together share one head's keys and values in L2.
+  const int32_t *t0 = tiles + (int64_t)(blockIdx.x / d.H) * TILE_REC;
+  const int first = t0[4], count = t0[5];
+  const int rel = (int)(blockIdx.x - (unsigned)first * d.H);
+  const int h = rel / count;
+  const int32_t *tr = tiles + (int64_t)(first + rel % count) * TILE_REC;
   const int g = tr[0], row0 = tr[1], row_end = tr[2];
   const int32_t *grow = gtab + g * 16;
   KvParts parts;
@@ -300,8 +306,29 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int row = row0 + w * BM + r;
       const bool valid = row < row_end;
-      const float inv = 1.f / l;
-      __nv_bfloat16 *orow = out + ((int64_t)row * d.H + h) * D;
+      float inv = 1.f / l;
+      if (w_gate_s != nullptr) {
+        // softmax gate of the layer, g_s = sigmoid(q . w_s[h]) from this row of Q in shared
+        // memory (128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7))
+        mbar_wait(smem_u32(&bars->q_full), 0, abort_flag, st, K_SOFTMAX_TC, 14);
+        const uint8_t *qt = base + C::Q_OFF + w * C::TILE_BYTES;
+        const float *ws_h = w_gate_s + h * D;
+        float dot = 0.f;
+#pragma unroll 1
+        for (int cl = 0; cl < D / 8; ++cl) {
+          const uint4 raw = *reinterpret_cast<const uint4 *>(qt + (cl >> 3) * (BM * 128) + r * 128 +
+                                                               (((cl & 7) ^ (r & 7)) << 4));
+          const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(hp[e]);
+            dot = fmaf(f.x, __ldg(ws_h + cl * 8 + 2 * e), dot);
+            dot = fmaf(f.y, __ldg(ws_h + cl * 8 + 2 * e + 1), dot);
+          }
+        }
+        inv *= 1.f / (1.f + expf(-dot));
+      }
+      __nv_bfloat16 *orow = out + (int64_t)row * out_row_stride + (int64_t)h * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t u[32];
@@ -331,7 +358,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 template <int D>
 cudaError_t launch_t(const Dims &d, const void *q, const void *k, const void *v, const void *kt, const void *vt,
-                     float sl2, void *o, float *lse, char *ws, const WsPlan &p, cudaStream_t st) {
+                     float sl2, void *o, int64_t o_row_stride, const float *w_gate_s, float *lse, char *ws,
+                     const WsPlan &p, cudaStream_t st) {
   using C = Cfg<D>;
   const uint64_t HD = (uint64_t)d.H * D;
   CUtensorMap mq, mk, mv, mkt, mvt;
@@ -352,7 +380,7 @@ cudaError_t launch_t(const Dims &d, const void *q, const void *k, const void *v,
   if (e != cudaSuccess) return e;
   const int ntiles = host_tile_count(d);
   softmax_tc_kernel<D><<<ntiles * d.H, THREADS, C::SMEM, st>>>(
-      mq, mk, mv, mkt, mvt, d, sl2, (__nv_bfloat16 *)o, lse, (const int32_t *)(ws + p.gtab),
+      mq, mk, mv, mkt, mvt, d, sl2, (__nv_bfloat16 *)o, o_row_stride, w_gate_s, lse, (const int32_t *)(ws + p.gtab),
       (const int32_t *)(ws + p.tiles), (DevStatus *)(ws + p.status));
   return cudaGetLastError();
 }
@@ -368,8 +396,18 @@ cudaError_t launch_softmax_tc(const Dims &d, vdn_dtype dt, const void *q, const 
                               char *ws, const WsPlan &p, cudaStream_t st) {
   (void)scales;
   if (dt != VDN_BF16) return cudaErrorInvalidValue;
-  if (d.D == 128) return launch_t<128>(d, q, k, v, kt, vt, sl2, o, lse, ws, p, st);
-  if (d.D == 64) return launch_t<64>(d, q, k, v, kt, vt, sl2, o, lse, ws, p, st);
+  const int64_t HD = (int64_t)d.H * d.D;
+  if (d.D == 128) return launch_t<128>(d, q, k, v, kt, vt, sl2, o, HD, nullptr, lse, ws, p, st);
+  if (d.D == 64) return launch_t<64>(d, q, k, v, kt, vt, sl2, o, HD, nullptr, lse, ws, p, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_softmax_tc_gated(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
+                                    const void *vt, const float *w_gate_s, float sl2, void *a, char *ws,
+                                    const WsPlan &p, cudaStream_t st) {
+  const int64_t stride = 2 * (int64_t)d.H * d.D;  // A = [A_s | A_l]: the softmax half of each row
+  if (d.D == 128) return launch_t<128>(d, q, k, v, kt, vt, sl2, a, stride, w_gate_s, nullptr, ws, p, st);
+  if (d.D == 64) return launch_t<64>(d, q, k, v, kt, vt, sl2, a, stride, w_gate_s, nullptr, ws, p, st);
   return cudaErrorInvalidValue;
 }
 

@@ -25,10 +25,12 @@ __global__ void tables_kernel(Dims d, int32_t *ftab, int32_t *gtab, int32_t *met
     last_keys = best_keys; last_g = best;
     const int32_t *r = gtab + best * 16;
     int64_t row_lo = (int64_t)r[0] * d.T, row_hi = (int64_t)r[1] * d.T;
+    const int64_t first = n, count = (row_hi - row_lo + TILE_M - 1) / TILE_M;
     for (int64_t a = row_lo; a < row_hi; a += TILE_M) {
       if (n >= tcap) { report(st, VDN_ERR_DEVICE, K_TABLES, 2); meta[0] = G; meta[1] = (int32_t)n; return; }
       int32_t *t = tiles + n * TILE_REC;
       t[0] = best; t[1] = (int32_t)a; t[2] = (int32_t)(a + TILE_M < row_hi ? a + TILE_M : row_hi); t[3] = best_keys;
+      t[4] = (int32_t)first; t[5] = (int32_t)count; t[6] = 0; t[7] = 0;
       ++n;
     }
   }

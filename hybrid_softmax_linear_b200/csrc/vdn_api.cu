@@ -146,6 +146,19 @@ vdn_status softmax_dispatch(const Dims &d, vdn_dtype dt, const void *q, const vo
   return VDN_OK;
 }
 
+vdn_status state_build_dispatch(const Dims &d, vdn_lin_kind kind, vdn_dtype act, const void *k, const void *v,
+                                const void *kt, const void *vt, float *S, float *z, float *St, float *zt, char *ws,
+                                const WsPlan &p, cudaStream_t st) {
+  if (kind == VDN_LIN_ELU1 && linear_tc_supported(d, act)) {
+    ProfScope ps(K_STATE_TC, st);
+    VDN_CUDA(launch_state_build_tc(d, k, v, kt, vt, S, z, St, zt, ws, p, st), "state build (tensor cores) launch");
+  } else {
+    ProfScope ps(K_STATE, st);
+    VDN_CUDA(launch_state_build(d, kind, act, k, v, kt, vt, S, z, St, zt, st), "state build launch");
+  }
+  return VDN_OK;
+}
+
 vdn_status out_proj_dispatch(const Dims &d, vdn_dtype act, const void *a, const void *w_os, const void *w_ol, void *y,
                              char *ws, const WsPlan &p, cudaStream_t st) {
   if (act == VDN_BF16 && out_proj_tc_supported(d)) {
@@ -196,7 +209,7 @@ size_t vdn_hybrid_attn_workspace_size(const vdn_shape *shape, vdn_lin_kind kind,
 
 size_t vdn_step_workspace_size(const vdn_shape *shape) {
   if (check_shape(shape) != VDN_OK) return 0;
-  return plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16).step_end;
+  return plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16).stage_end;
 }
 
 vdn_status vdn_workspace_init(void *ws, size_t ws_bytes, vdn_stream stream) {
@@ -230,7 +243,6 @@ vdn_status vdn_softmax_branch_fwd(const vdn_shape *shape, vdn_dtype dtype, const
 vdn_status vdn_linear_state_build(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *k,
                                   const void *v, const void *kt, const void *vt, float *S, float *z, float *S_txt,
                                   float *z_txt, void *ws, size_t ws_bytes, vdn_stream stream) {
-  (void)ws; (void)ws_bytes;
   VDN_TRY(check_shape(shape));
   VDN_TRY(check_kind(kind));
   VDN_TRY(check_act_dtype(dtype));
@@ -238,10 +250,11 @@ vdn_status vdn_linear_state_build(const vdn_shape *shape, vdn_lin_kind kind, vdn
   VDN_TRY(need(S_txt, "S_txt"));
   if (kind == VDN_LIN_ELU1) VDN_TRY(need(z_txt, "z_txt"));
   if (shape->text_tokens > 0) { VDN_TRY(need(kt, "kt")); VDN_TRY(need(vt, "vt")); }
+  const WsPlan p = plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16);
+  VDN_TRY(check_ws(ws, ws_bytes, p.step_end));
   VDN_TRY(check_device());
-  const Dims d = dims_of(*shape);
-  VDN_CUDA(launch_state_build(d, kind, dtype, k, v, kt, vt, S, z, S_txt, z_txt, (cudaStream_t)stream),
-           "state build launch");
+  VDN_TRY(state_build_dispatch(dims_of(*shape), kind, dtype, k, v, kt, vt, S, z, S_txt, z_txt, (char *)ws, p,
+                               (cudaStream_t)stream));
   return ok();
 }
 
@@ -277,12 +290,23 @@ vdn_status vdn_linear_read(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype 
   VDN_TRY(need(q, "q")); VDN_TRY(need(S_fwd, "S_fwd")); VDN_TRY(need(S_bwd, "S_bwd")); VDN_TRY(need(o_l, "o_l"));
   if (kind == VDN_LIN_ELU1) { VDN_TRY(need(z_fwd, "z_fwd")); VDN_TRY(need(z_bwd, "z_bwd")); }
   const WsPlan p = plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16);
-  VDN_TRY(check_ws(ws, ws_bytes, p.step_end));
+  VDN_TRY(check_ws(ws, ws_bytes, p.stage_end));
   VDN_TRY(check_device());
   const Dims d = dims_of(*shape);
   cudaStream_t st = (cudaStream_t)stream;
   VDN_CUDA(launch_tables(d, (char *)ws, p, st), "tables launch");
-  VDN_CUDA(launch_linear_read(d, kind, dtype, q, S_fwd, S_bwd, z_fwd, z_bwd, o_l, (char *)ws, p, st), "read launch");
+  if (linear_tc_supported(d, dtype)) {
+    {
+      ProfScope ps(K_READ_STAGE, st);
+      VDN_CUDA(launch_read_stage(d, kind, S_fwd, S_bwd, z_fwd, z_bwd, nullptr, 0, (char *)ws, p, st), "read staging");
+    }
+    ProfScope ps(K_READ_TC, st);
+    VDN_CUDA(launch_read_tc(d, kind, q, o_l, nullptr, 0, nullptr, 0.f, (char *)ws, p, st), "read launch");
+  } else {
+    ProfScope ps(K_READ, st);
+    VDN_CUDA(launch_linear_read(d, kind, dtype, q, S_fwd, S_bwd, z_fwd, z_bwd, o_l, (char *)ws, p, st),
+             "read launch");
+  }
   return ok();
 }
 
@@ -345,23 +369,44 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
     ProfScope ps(K_TABLES, st);
     VDN_CUDA(launch_tables(d, w, p, st), "tables launch");
   }
-  VDN_TRY(softmax_dispatch(d, dtype, q, k, v, kt, vt, nullptr, scale_log2_of(0.f, d.D), Os, nullptr, w, p, st));
-  {
-    ProfScope ps(K_STATE, st);
-    VDN_CUDA(launch_state_build(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, st),
-             "state build launch");
-  }
-  {
-    ProfScope ps(K_SCAN, st);
-    VDN_CUDA(launch_state_scan(d, kind, S, z, St, zt, beta, Sf, Sb, zf, zb, w, p, st), "scan launch");
-  }
-  {
-    ProfScope ps(K_READ, st);
-    VDN_CUDA(launch_linear_read(d, kind, act, q, Sf, Sb, zf, zb, Ol, w, p, st), "read launch");
-  }
-  {
-    ProfScope ps(K_FUSE, st);
-    VDN_CUDA(launch_fuse(d, act, q, Os, Ol, w_gate_s, w_gate_l, G_l, gamma, eps, A, st), "fuse launch");
+  if (layer_fused(*shape, dtype)) {
+    // tensor-core path: the softmax epilogue writes A_s = g_s * O_s and the linear read
+    // writes A_l = g_l * gamma * RMSNorm(O_l), both straight into A
+    {
+      ProfScope ps(K_SOFTMAX_TC, st);
+      VDN_CUDA(launch_softmax_tc_gated(d, q, k, v, kt, vt, w_gate_s, scale_log2_of(0.f, d.D), A, w, p, st),
+               "softmax branch (tensor cores) launch");
+    }
+    VDN_TRY(state_build_dispatch(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, w, p,
+                                 st));
+    {
+      ProfScope ps(K_SCAN, st);
+      VDN_CUDA(launch_state_scan(d, kind, S, z, St, zt, beta, Sf, Sb, zf, zb, w, p, st), "scan launch");
+    }
+    {
+      ProfScope ps(K_READ_STAGE, st);
+      VDN_CUDA(launch_read_stage(d, kind, Sf, Sb, zf, zb, w_gate_l, G_l, w, p, st), "read staging");
+    }
+    {
+      ProfScope ps(K_READ_TC, st);
+      VDN_CUDA(launch_read_tc(d, kind, q, A, w_gate_l, G_l, gamma, eps, w, p, st), "read launch");
+    }
+  } else {
+    VDN_TRY(softmax_dispatch(d, dtype, q, k, v, kt, vt, nullptr, scale_log2_of(0.f, d.D), Os, nullptr, w, p, st));
+    VDN_TRY(state_build_dispatch(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, w, p,
+                                 st));
+    {
+      ProfScope ps(K_SCAN, st);
+      VDN_CUDA(launch_state_scan(d, kind, S, z, St, zt, beta, Sf, Sb, zf, zb, w, p, st), "scan launch");
+    }
+    {
+      ProfScope ps(K_READ, st);
+      VDN_CUDA(launch_linear_read(d, kind, act, q, Sf, Sb, zf, zb, Ol, w, p, st), "read launch");
+    }
+    {
+      ProfScope ps(K_FUSE, st);
+      VDN_CUDA(launch_fuse(d, act, q, Os, Ol, w_gate_s, w_gate_l, G_l, gamma, eps, A, st), "fuse launch");
+    }
   }
   VDN_TRY(out_proj_dispatch(d, act, A, w_os, w_ol, y, w, p, st));
   return ok();
@@ -371,9 +416,10 @@ void *vdn_hybrid_attn_intermediate(const vdn_shape *shape, vdn_lin_kind kind, vd
   if (check_shape(shape) != VDN_OK || ws == nullptr) return nullptr;
   const WsPlan p = plan_workspace(*shape, kind, dtype);
   char *w = (char *)ws;
+  const bool fused = layer_fused(*shape, dtype);
   switch (which) {
-    case 0: return w + p.Os;
-    case 1: return w + p.Ol;
+    case 0: return fused ? nullptr : w + p.Os;
+    case 1: return fused ? nullptr : w + p.Ol;
     case 2: return w + p.A;
     case 3: return w + p.Sf;
     case 4: return w + p.Sb;

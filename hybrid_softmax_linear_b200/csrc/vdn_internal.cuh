@@ -116,7 +116,7 @@ VDN_HD int group_keys(const int32_t *grow) {
 // Query rows are cut into tiles of TILE_M rows that never straddle a group, so every
 // row of a tile shares one key set.  Tiles are listed longest key set first.
 constexpr int TILE_M = 256;
-constexpr int TILE_REC = 4;  // {group, row_lo, row_hi, n_keys}
+constexpr int TILE_REC = 8;  // {group, row_lo, row_hi, n_keys, first tile of the group, tiles of the group, 0, 0}
 
 VDN_HD int64_t max_tiles(int F, int T, int C) {
   return (int64_t)F * T / TILE_M + max_groups(F, C) + 1;
@@ -129,9 +129,18 @@ VDN_HD size_t align_up(size_t x) { return (x + WS_ALIGN - 1) / WS_ALIGN * WS_ALI
 struct WsPlan {
   // step part (tables, tile list, status)
   size_t status, ftab, gtab, meta, tiles, step_end;
+  // read staging: per-group summed memory in bf16 (tensor-core B operand), summed
+  // normaliser, linear-gate weights in bf16
+  size_t ssum, zsum, wl, stage_end;
   // layer part
   size_t S, z, St, zt, Sf, Sb, zf, zb, Os, Ol, A, q8, k8, v8, kt8, vt8, scales, amax, total;
 };
+
+// The whole layer runs on the tensor-core path (softmax and linear read write A
+// directly; O_s and O_l are never stored) for bf16 activations with D = 128.
+inline bool layer_fused(const vdn_shape &s, vdn_dtype dtype) {
+  return (dtype == VDN_BF16 || dtype == VDN_E4M3) && s.head_dim == 128;
+}
 
 // meta: int32[8] = {G, n_tiles, ...}
 inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dtype) {
@@ -147,6 +156,10 @@ inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dt
   p.meta = take(64);
   p.tiles = take((size_t)max_tiles(s.frames, s.tokens_per_frame, s.chunk_frames) * TILE_REC * 4);
   p.step_end = off;
+  p.ssum = take(G * H * D * D * 2);
+  p.zsum = take(G * H * D * 4);
+  p.wl = take(H * D * D * 2);
+  p.stage_end = off;
   size_t act = (dtype == VDN_F32) ? 4 : 2;
   // per-frame states: ELU1 S [F][H][D][D]; DELTA kbar [F][H][D] in S, vbar in z
   p.S = take(kind == VDN_LIN_ELU1 ? F * H * D * D * 4 : F * H * D * 4);
@@ -157,8 +170,9 @@ inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dt
   p.Sb = take(G * H * D * D * 4);
   p.zf = take(G * H * D * 4);
   p.zb = take(G * H * D * 4);
-  p.Os = take(Nv * H * D * act);
-  p.Ol = take(Nv * H * D * act);
+  const bool fused = layer_fused(s, dtype);
+  p.Os = take(fused ? 0 : Nv * H * D * act);
+  p.Ol = take(fused ? 0 : Nv * H * D * act);
   p.A = take(Nv * 2 * H * D * act);
   if (dtype == VDN_E4M3) {
     p.q8 = take(Nv * H * D);
@@ -184,6 +198,7 @@ struct DevStatus {
 enum KernelId : uint32_t {
   K_TABLES = 1, K_SOFTMAX_SIMT = 2, K_SOFTMAX_TC = 3, K_STATE = 4, K_SCAN = 5, K_READ = 6,
   K_FUSE = 7, K_GEMM_SIMT = 8, K_GEMM_TC = 9, K_QUANT = 10, K_DELTA = 11, K_DEBUG_WAIT = 12,
+  K_STATE_TC = 13, K_READ_STAGE = 14, K_READ_TC = 15,
 };
 
 __device__ __forceinline__ void report(DevStatus *st, uint32_t code, uint32_t where, uint32_t detail) {
@@ -265,6 +280,22 @@ cudaError_t launch_state_scan(const Dims &d, vdn_lin_kind kind, const float *S, 
 cudaError_t launch_linear_read(const Dims &d, vdn_lin_kind kind, vdn_dtype dt, const void *q, const float *Sf,
                                const float *Sb, const float *zf, const float *zb, void *o, char *ws,
                                const WsPlan &p, cudaStream_t st);
+// tensor-core linear branch (bf16, D = 128)
+bool linear_tc_supported(const Dims &d, vdn_dtype dt);
+cudaError_t launch_state_build_tc(const Dims &d, const void *k, const void *v, const void *kt, const void *vt,
+                                  float *S, float *z, float *St, float *zt, char *ws, const WsPlan &p,
+                                  cudaStream_t st);
+// sums the two memories of every group into the bf16 staging buffers (and the gate weights to bf16)
+cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf, const float *Sb, const float *zf,
+                              const float *zb, const float *wgl, int G_l, char *ws, const WsPlan &p,
+                              cudaStream_t st);
+// o_l (plain) or, with gate weights, A_l = g_l * gamma * RMSNorm(o_l) into the linear half of A
+cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void *out, const float *wgl, int G_l,
+                           const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st);
+cudaError_t launch_softmax_tc_gated(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
+                                    const void *vt, const float *w_gate_s, float sl2, void *a, char *ws,
+                                    const WsPlan &p, cudaStream_t st);
+
 cudaError_t launch_fuse(const Dims &d, vdn_dtype dt, const void *q, const void *os, const void *ol,
                         const float *wgs, const float *wgl, int G_l, const float *gamma, float eps, void *a,
                         cudaStream_t st);

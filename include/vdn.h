@@ -228,8 +228,9 @@ VDN_API vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind
 /* Device pointers (inside ws) of the layer's intermediates after vdn_hybrid_attn_fwd:
  * which = 0: O_s [N_v][H][D] (bf16, or float for VDN_F32); 1: O_l (same type);
  * 2: A [N_v][2HD]; 3: per-group S_fwd; 4: S_bwd; 5: frame table int32[F][8];
- * 6: group table int32[G][16]; 7: query-tile list int32[n][4] (group, row_lo, row_hi,
- * keys), longest key set first; 8: meta int32[2] (G, n).  Entries 5-8 are also
+ * 6: group table int32[G][16]; 7: query-tile list int32[n][8] (group, row_lo, row_hi,
+ * keys, first tile of the group, tiles of the group, 0, 0) of 256-row tiles, groups with
+ * the longest key set first; 8: meta int32[2] (G, n).  Entries 5-8 are also
  * written by the step entry points that take a workspace.  NULL if not materialised.
  * Valid until the next call that uses ws. */
 VDN_API void *vdn_hybrid_attn_intermediate(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, void *ws,

@@ -69,6 +69,10 @@ class Run:
         vdn.check_device_status(self.ws)
         return y
 
+    def materialises_branches(self) -> bool:
+        """False on the fused tensor-core path, where O_s and O_l never reach memory."""
+        return vdn.hybrid_attn_intermediate(self.shape, self.kind, self.cdt, self.ws, 0) != 0
+
     def intermediate(self, which, shape, tdtype):
         ptr = vdn.hybrid_attn_intermediate(self.shape, self.kind, self.cdt, self.ws, which)
         n = int(np.prod(shape))

@@ -36,9 +36,10 @@ def _check_tables(run: Run):
     assert G == len(gtab)
     np.testing.assert_array_equal(run.intermediate(5, (s.frames, 8), torch.int32).cpu().numpy(), ftab)
     np.testing.assert_array_equal(run.intermediate(6, (G, 16), torch.int32).cpu().numpy(), gtab)
-    tiles = run.intermediate(7, (n, 4), torch.int32).cpu().numpy()
+    tiles = run.intermediate(7, (n, 8), torch.int32).cpu().numpy()
     covered = np.zeros(s.n_video, np.int32)
-    for g, lo, hi, keys in tiles:
+    for i, (g, lo, hi, keys, first, count, _, _) in enumerate(tiles):
+        assert first <= i < first + count and all(tiles[first:first + count, 0] == g)
         assert 0 < hi - lo <= 256
         flo, fhi = gtab[g][0] * s.tokens_per_frame, gtab[g][1] * s.tokens_per_frame
         assert flo <= lo < hi <= fhi
@@ -56,21 +57,29 @@ def _layer_parity(run: Run, rows, kind_tol, check_states=True):
     y = run.layer()
     Nv, H, D = run.Nv, run.H, run.D
     rows_t = torch.from_numpy(rows).cuda()
-    Os = to_numpy(run.intermediate(0, (Nv, H, D), tdt)[rows_t])
-    Ol = to_numpy(run.intermediate(1, (Nv, H, D), tdt)[rows_t])
     A = to_numpy(run.intermediate(2, (Nv, 2 * H * D), tdt)[rows_t])
     yr = to_numpy(y[rows_t])
     _check_tables(run)
     # each step against the oracle of that step
     ref_os = vo.softmax_branch(o["q"], o["k"], o["v"], o["kt"], o["vt"], F, T, C, rows=rows)
-    assert_close("O_s", Os, ref_os, kind_tol)
     if run.kind == vdn.DELTA:
         ref_ol = vo.delta_branch(o["q"], o["k"], o["v"], o["kt"], o["vt"], o["beta"], F, T, C, rows=rows)
     else:
         ref_ol = vo.linear_branch(o["q"], o["k"], o["v"], o["kt"], o["vt"], F, T, C, rows=rows)
-    assert_close("O_l", Ol, ref_ol, kind_tol)
-    ref_a_dev = vo.hybrid_fuse(o["q"][rows], Os, Ol, o["w_gate_s"], o["w_gate_l"], o["gamma"], 1e-6)
-    assert_close("A (fuse of device O_s, O_l)", A, ref_a_dev, kind_tol)
+    if run.materialises_branches():
+        Os = to_numpy(run.intermediate(0, (Nv, H, D), tdt)[rows_t])
+        Ol = to_numpy(run.intermediate(1, (Nv, H, D), tdt)[rows_t])
+        assert_close("O_s", Os, ref_os, kind_tol)
+        assert_close("O_l", Ol, ref_ol, kind_tol)
+        ref_a_dev = vo.hybrid_fuse(o["q"][rows], Os, Ol, o["w_gate_s"], o["w_gate_l"], o["gamma"], 1e-6)
+        assert_close("A (fuse of device O_s, O_l)", A, ref_a_dev, kind_tol)
+    else:
+        # fused path: O_s and O_l never leave the kernels; each half of A is checked
+        # against the oracle of its branch followed by the gate (and RMSNorm)
+        ref_a = vo.hybrid_fuse(o["q"][rows], ref_os, ref_ol, o["w_gate_s"], o["w_gate_l"], o["gamma"], 1e-6)
+        HD = H * D
+        assert_close("A_s (softmax branch + gate)", A[:, :HD], ref_a[:, :HD], kind_tol)
+        assert_close("A_l (linear branch + RMSNorm + gate)", A[:, HD:], ref_a[:, HD:], kind_tol)
     assert_close("y (projection of device A)", yr, vo.out_proj(A, o["w_os"], o["w_ol"]), kind_tol)
     # the whole layer, float64 from the inputs
     ref_a = vo.hybrid_fuse(o["q"][rows], ref_os, ref_ol, o["w_gate_s"], o["w_gate_l"], o["gamma"], 1e-6)
@@ -83,8 +92,10 @@ def _layer_parity(run: Run, rows, kind_tol, check_states=True):
         first = [int(r[0]) for r in gtab]
         Sf = run.intermediate(3, (G, H, D, D), torch.float32).cpu().numpy()
         Sb = run.intermediate(4, (G, H, D, D), torch.float32).cpu().numpy()
-        assert rel_l2(Sf, num_f[first]) <= 1e-5
-        assert rel_l2(Sb, num_b[first]) <= 1e-5
+        # fp32 sums; on the tensor-core path phi(k) enters the MMA in bf16
+        state_tol = 1e-5 if run.dtype == "f32" else 5e-3
+        assert rel_l2(Sf, num_f[first]) <= state_tol
+        assert rel_l2(Sb, num_b[first]) <= state_tol
 
 
 # ----------------------------------------------------------------------------- configurations
@@ -143,10 +154,16 @@ def test_scalar_linear_gate():
 
 
 # ----------------------------------------------------------------------------- step entry points
-def test_step_entry_points_match_oracle():
-    w = synth.CONFIGS[2]
-    s, inp = w.shape, cfg_inputs(2)
+@pytest.mark.parametrize("shape", [None, (12, 300, 5, 40, 2, 128)])
+def test_step_entry_points_match_oracle(shape):
+    if shape is None:
+        s, inp = synth.CONFIGS[2].shape, cfg_inputs(2)
+    else:
+        s = synth.Shape(*shape)
+        inp = synth.make_inputs(s, "bf16", seed=4242)
     F, T, C, L, H, D = s.frames, s.tokens_per_frame, s.chunk_frames, s.text_tokens, s.heads, s.head_dim
+    # states: fp32 sums; the tensor-core state build (D = 128) feeds phi(k) to the MMA in bf16
+    st_tol = 5e-3 if D == 128 else 1e-5
     Nv = s.n_video
     o = oracle_inputs(inp)
     d = {n: to_device(a) for n, a in inp.items()}
@@ -171,11 +188,11 @@ def test_step_entry_points_match_oracle():
     z = torch.empty((F, H, D), dtype=torch.float32, device="cuda")
     St = torch.empty((H, D, D), dtype=torch.float32, device="cuda")
     zt = torch.empty((H, D), dtype=torch.float32, device="cuda")
-    vdn.linear_state_build(s, vdn.ELU1, vdn.BF16, d["k"], d["v"], d["kt"], d["vt"], S, z, St, zt)
+    vdn.linear_state_build(s, vdn.ELU1, vdn.BF16, d["k"], d["v"], d["kt"], d["vt"], S, z, St, zt, ws)
     rS, rz = vo.frame_states(o["k"], o["v"], F, T)
     rSt, rzt = vo.text_state(o["kt"], o["vt"])
-    assert rel_l2(S.cpu().numpy(), rS) < 1e-5 and rel_l2(z.cpu().numpy(), rz) < 1e-5
-    assert rel_l2(St.cpu().numpy(), rSt) < 1e-5 and rel_l2(zt.cpu().numpy(), rzt) < 1e-5
+    assert rel_l2(S.cpu().numpy(), rS) < st_tol and rel_l2(z.cpu().numpy(), rz) < 1e-5
+    assert rel_l2(St.cpu().numpy(), rSt) < st_tol and rel_l2(zt.cpu().numpy(), rzt) < 1e-5
     G = vdn.max_groups(s)
     Sf, Sb = (torch.empty((G, H, D, D), dtype=torch.float32, device="cuda") for _ in range(2))
     zf, zb = (torch.empty((G, H, D), dtype=torch.float32, device="cuda") for _ in range(2))
@@ -184,7 +201,7 @@ def test_step_entry_points_match_oracle():
     first = [int(r[0]) for r in gtab]
     nf, nb, df, db = vo.linear_memory(o["k"], o["v"], o["kt"], o["vt"], F, T, C)
     ng = len(gtab)
-    assert rel_l2(Sf[:ng].cpu().numpy(), nf[first]) < 1e-5 and rel_l2(Sb[:ng].cpu().numpy(), nb[first]) < 1e-5
+    assert rel_l2(Sf[:ng].cpu().numpy(), nf[first]) < st_tol and rel_l2(Sb[:ng].cpu().numpy(), nb[first]) < st_tol
     assert rel_l2(zf[:ng].cpu().numpy(), df[first]) < 1e-5 and rel_l2(zb[:ng].cpu().numpy(), db[first]) < 1e-5
     o_l = empty((Nv, H, D), "bf16")
     vdn.linear_read(s, vdn.ELU1, vdn.BF16, d["q"], Sf, Sb, zf, zb, o_l, ws)
