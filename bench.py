@@ -167,6 +167,22 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, n_video: int, ms_per_step: float) -> float:
+    """Video tokens per second over all replicas: every rank runs its own batch."""
+    return world * n_video / (ms_per_step / 1e3)
+
+
 def workload_config(cfg: int) -> dict:
     w = synth.CONFIGS[cfg]
     s = w.shape
@@ -211,11 +227,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     for _ in range(args.warmup):
         step(d)
@@ -263,7 +275,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return
     per_step_ms = ms / max(args.steps, 1)
-    value = world * s.n_video / (per_step_ms / 1e3)
+    value = whole_job_value(world, s.n_video, per_step_ms)
     peaks, peak_src = load_peaks()
     fl = layer_flops(s)
     sm_key = "softmax_tc" if "softmax_tc" in prof else "softmax_simt"
@@ -283,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
         "layer_tflops": sum(v for k, v in fl.items()) / (per_step_ms / 1e3) / 1e12,
         "per_kernel_ms_per_step": {k: round(v[0] / max(args.steps, 1), 4) for k, v in prof.items()},
         "gpu_launches": launches,
-        "e2e": {"value": world * s.n_video / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_value(world, s.n_video, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "clocks": clk,
     }
@@ -300,7 +312,7 @@ def main():
     ap.add_argument("--config", type=int, default=4, choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-rows", type=int, default=48, help="query rows of the CPU oracle sample")
-    ap.add_argument("--ref-rows", type=int, default=32, help="query rows per step of --impl reference")
+    ap.add_argument("--ref-rows", type=int, default=16, help="query rows per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))

@@ -1,0 +1,61 @@
+"""Host logic of the benchmark on CPU: the replica (data-parallel) layout with two ranks
+over gloo.  Each rank draws its own batch, the timing reduction takes the max over
+ranks, and the whole-job value counts every rank's tokens."""
+import os
+import socket
+
+import numpy as np
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from hybrid_softmax_linear_b200 import synth
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = 10.0 + 5.0 * rank          # rank 1 is the slow one
+        out[rank] = bench.reduce_max(local_ms, world, torch.device("cpu"))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_with_gloo_world_size_2():
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+    assert out[0] == out[1] == 15.0
+
+
+def test_whole_job_value_counts_every_replica():
+    assert bench.whole_job_value(1, 90720, 50.0) == 90720 / 0.05
+    assert bench.whole_job_value(4, 90720, 50.0) == 4 * 90720 / 0.05
+
+
+def test_replicas_draw_distinct_batches():
+    a = synth.workload_inputs(1, rank=0)
+    b = synth.workload_inputs(1, rank=1)
+    c = synth.workload_inputs(1, rank=0)
+    assert not np.array_equal(a["q"], b["q"])
+    for n in a:
+        np.testing.assert_array_equal(a[n], c[n])      # deterministic per rank
+
+
+def test_softmax_flop_count_matches_brute_force():
+    s = synth.Shape(12, 7, 2, 3, 2, 32)
+    from oracle import vdn_oracle as vo
+    M = vo.frame_mask(s.frames, s.chunk_frames)
+    keys = sum(s.tokens_per_frame * (s.text_tokens + s.tokens_per_frame * int((M[f] == vo.SOFT).sum()))
+               for f in range(s.frames))
+    assert bench.softmax_flops(s) == 4.0 * s.head_dim * s.heads * keys
