@@ -19,7 +19,7 @@ __all__ = [
     "mask_layout_build", "max_groups", "hybrid_attn_workspace_size", "step_workspace_size", "workspace_init",
     "softmax_branch_fwd", "linear_state_build", "linear_state_scan", "linear_read", "hybrid_fuse", "out_proj",
     "hybrid_attn_fwd", "hybrid_attn_intermediate", "check_device_status", "debug_unset_flag_wait", "version",
-    "profile_begin", "profile_end",
+    "profile_begin", "profile_end", "fp8_quant_per_head", "softmax_branch_fwd_noalloc",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdn.so")
@@ -75,6 +75,8 @@ _SIGS = {
     "vdn_debug_unset_flag_wait": (ctypes.c_int, [_vp, _sz, _u32, _vp]),
     "vdn_softmax_branch_fwd_noalloc": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp,
                                                       _vp]),
+    "vdn_fp8_quant_per_head": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                              _vp]),
     "vdn_profile_begin": (ctypes.c_int, [_i32]),
     "vdn_profile_end": (ctypes.c_int, [_vp, _vp, _i32]),
 }
@@ -169,6 +171,13 @@ def softmax_branch_fwd_noalloc(shape, dtype, q, k, v, kt, vt, o_s, sm_scale=0.0,
     used instead (for callers that cannot allocate device memory)."""
     _check(lib().vdn_softmax_branch_fwd_noalloc(ctypes.byref(Shape.of(shape)), dtype, _p(q), _p(k), _p(v), _p(kt),
                                                 _p(vt), sm_scale, _p(o_s), _p(lse), _stream(stream)))
+
+
+def fp8_quant_per_head(shape, q, k, v, kt, vt, q8, k8, v8, kt8, vt8, scales, ws, stream=None):
+    """Per-head e4m3 copies of q, k (+ kt), v (+ vt) and their float[3][H] scales."""
+    _check(lib().vdn_fp8_quant_per_head(ctypes.byref(Shape.of(shape)), _p(q), _p(k), _p(v), _p(kt), _p(vt), _p(q8),
+                                        _p(k8), _p(v8), _p(kt8), _p(vt8), _p(scales), _p(ws), _nbytes(ws),
+                                        _stream(stream)))
 
 
 def linear_state_build(shape, kind, dtype, k, v, kt, vt, S, z, S_txt, z_txt, ws, stream=None):

@@ -29,17 +29,24 @@ constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
-template <int D>
+// FP8 = false: bf16 Q/K/V and P (kind::f16, K = 16 per MMA).  FP8 = true: e4m3 Q/K/V
+// with per-head scales and e4m3 P at unit scale (kind::f8f6f4, K = 32 per MMA).  A
+// 128-byte swizzle row holds 64 bf16 or 128 e4m3 values; one MMA K-step is 32 bytes of a
+// row either way, and one P column of tensor memory packs 2 bf16 or 4 e4m3 values.
+template <int D, bool FP8>
 struct Cfg {
-  static constexpr int BOXES = D / 64;                 // 64-column (128-byte) boxes per row
-  static constexpr int TILE_BYTES = BM * D * 2;        // one 128 x D bf16 tile
+  static constexpr int EB = FP8 ? 1 : 2;               // bytes per element
+  static constexpr int BOX_ELEMS = 128 / EB;           // elements in a 128-byte box row
+  static constexpr int BOXES = D * EB / 128;           // 128-byte boxes per row
+  static constexpr int TILE_BYTES = BM * D * EB;       // one 128 x D tile
+  static constexpr int KSTEP = 32 / EB;                // elements per MMA K-step
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + NQ * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + KST * TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + VST * TILE_BYTES;
   static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
-  static constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);
-  static constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);
+  static constexpr uint32_t IDESC_S = FP8 ? idesc_e4m3(BM, BN, false, false) : idesc_bf16(BM, BN, false, false);
+  static constexpr uint32_t IDESC_O = FP8 ? idesc_e4m3(BM, D, false, true) : idesc_bf16(BM, D, false, true);
   // tensor memory columns: S_0, S_1, O_0, O_1
   __device__ static constexpr uint32_t s_col(int w) { return (uint32_t)w * 128u; }
   __device__ static constexpr uint32_t o_col(int w) { return 256u + (uint32_t)w * 128u; }
@@ -89,14 +96,15 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-template <int D>
+template <int D, bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
     softmax_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
-                      const __grid_constant__ CUtensorMap tmVt, Dims d, float sl2, __nv_bfloat16 *__restrict__ out,
-                      int64_t out_row_stride, const float *__restrict__ w_gate_s, float *__restrict__ lse,
-                      const int32_t *__restrict__ gtab, const int32_t *__restrict__ tiles, DevStatus *st) {
-  using C = Cfg<D>;
+                      const __grid_constant__ CUtensorMap tmVt, Dims d, float sl2, const float *__restrict__ scales,
+                      __nv_bfloat16 *__restrict__ out, int64_t out_row_stride, const float *__restrict__ w_gate_s,
+                      float *__restrict__ lse, const int32_t *__restrict__ gtab, const int32_t *__restrict__ tiles,
+                      DevStatus *st) {
+  using C = Cfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   Bars *bars = reinterpret_cast<Bars *>(base + C::BAR_OFF);
@@ -117,6 +125,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int32_t *tr = tiles + (int64_t)(first + rel % count) * TILE_REC;
   const int g = tr[0], row0 = tr[1], row_end = tr[2];
   const int32_t *grow = gtab + g * 16;
+  // e4m3: scores carry s_q * s_k, the output s_v (per-head dequantisation scales)
+  if (FP8) sl2 *= scales[h] * scales[d.H + h];
+  const float out_scale = FP8 ? scales[2 * d.H + h] : 1.f;
   KvParts parts;
   kv_parts(grow, d.L, parts);
   const int nkv = kv_tiles(parts);
@@ -146,8 +157,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive_expect_tx(qb, NQ * C::TILE_BYTES);
       for (int w = 0; w < NQ; ++w)
         for (int c = 0; c < C::BOXES; ++c)
-          tma_load_2d(smem_u32(base + C::Q_OFF + w * C::TILE_BYTES + c * BM * 128), &tmQ, qb, h * D + c * 64,
-                      row0 + w * BM);
+          tma_load_2d(smem_u32(base + C::Q_OFF + w * C::TILE_BYTES + c * BM * 128), &tmQ, qb,
+                      h * D + c * C::BOX_ELEMS, row0 + w * BM);
       KvCursor cur;
       cur.init(parts);
       for (int j = 0; j < nkv; ++j) {
@@ -158,14 +169,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t kb = smem_u32(&bars->k_full[ks]);
         mbar_arrive_expect_tx(kb, C::TILE_BYTES);
         for (int c = 0; c < C::BOXES; ++c)
-          tma_load_2d(smem_u32(base + C::K_OFF + ks * C::TILE_BYTES + c * BN * 128), mk, kb, h * D + c * 64, cur.row);
+          tma_load_2d(smem_u32(base + C::K_OFF + ks * C::TILE_BYTES + c * BN * 128), mk, kb, h * D + c * C::BOX_ELEMS,
+                      cur.row);
         armed_k |= 1u << ks;
         ph_k = (ph_k & ~(1u << ks)) | (((j / KST) & 1u) << ks);
         if (!mbar_wait(smem_u32(&bars->v_empty[vs]), ((j / VST) & 1) ^ 1, abort_flag, st, K_SOFTMAX_TC, 2)) break;
         const uint32_t vb = smem_u32(&bars->v_full[vs]);
         mbar_arrive_expect_tx(vb, C::TILE_BYTES);
         for (int c = 0; c < C::BOXES; ++c)
-          tma_load_2d(smem_u32(base + C::V_OFF + vs * C::TILE_BYTES + c * BN * 128), mv, vb, h * D + c * 64, cur.row);
+          tma_load_2d(smem_u32(base + C::V_OFF + vs * C::TILE_BYTES + c * BN * 128), mv, vb, h * D + c * C::BOX_ELEMS,
+                      cur.row);
         armed_v |= 1u << vs;
         ph_v = (ph_v & ~(1u << vs)) | (((j / VST) & 1u) << vs);
         cur.next(parts);
@@ -186,9 +199,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t kbase = smem_u32(base + C::K_OFF + (j % KST) * C::TILE_BYTES);
         const uint32_t abase = qa + w * C::TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          mma_ss(tmem + C::s_col(w), sdesc(abase + off, 16, 1024), sdesc(kbase + off, 16, 1024), C::IDESC_S, kk > 0);
+        for (int kk = 0; kk < D / C::KSTEP; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;  // 32-byte K-steps, 4 per box row
+          if (FP8)
+            mma_ss_f8(tmem + C::s_col(w), sdesc(abase + off, 16, 1024), sdesc(kbase + off, 16, 1024), C::IDESC_S,
+                      kk > 0);
+          else
+            mma_ss(tmem + C::s_col(w), sdesc(abase + off, 16, 1024), sdesc(kbase + off, 16, 1024), C::IDESC_S,
+                   kk > 0);
         }
         mma_commit(smem_u32(&bars->s_full[w]));
       };
@@ -210,11 +228,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int w = 0; w < NQ && ok; ++w) {
           if (!mbar_wait(smem_u32(&bars->p_full[w]), j & 1, abort_flag, st, K_SOFTMAX_TC, 7)) { ok = false; break; }
           tc_fence_after();
-          // O_w += P_w V_j: P_w (bf16, two per column) sits over the first 64 columns of S_w
+          // O_w += P_w V_j: P_w (two bf16 or four e4m3 per column) sits over the first columns
+          // of S_w; each K-step takes 8 of those columns and KSTEP rows of V (128 bytes each)
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_ts(tmem + C::o_col(w), tmem + C::s_col(w) + kk * 8, sdesc(vbase + kk * 2048, BM * 128, 1024),
-                   C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / C::KSTEP; ++kk) {
+            const uint64_t bdesc = sdesc(vbase + kk * (C::KSTEP * 128), BM * 128, 1024);
+            if (FP8)
+              mma_ts_f8(tmem + C::o_col(w), tmem + C::s_col(w) + kk * 8, bdesc, C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+            else
+              mma_ts(tmem + C::o_col(w), tmem + C::s_col(w) + kk * 8, bdesc, C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          }
           if (more) issue_s(w, j + 1);
         }
         mma_commit(smem_u32(&bars->v_empty[vs]));
@@ -270,17 +293,38 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       float rs = 0.f;
       const float neg_m = -m;
+      if (FP8) {
+        // e4m3 P at unit scale, four per tensor-memory column (p <= 2^8 < 448)
 #pragma unroll
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t pk[16];
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(s[c + 2 * i], sl2, neg_m));
-          const float p1 = ex2(fmaf(s[c + 2 * i + 1], sl2, neg_m));
-          rs += p0 + p1;
-          pk[i] = pack_bf16(p0, p1);
+          for (int i = 0; i < 8; ++i) {
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              p[e] = ex2(fmaf(s[c + 4 * i + e], sl2, neg_m));
+              rs += p[e];
+            }
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p[0], p[1]), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p[2], p[3]), __NV_SATFINITE, __NV_E4M3);
+            pk[i] = (lo & 0xffffu) | (hi << 16);
+          }
+          tmem_st8(s_addr + (c >> 2), pk);
         }
-        tmem_st16(s_addr + (c >> 1), pk);
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(fmaf(s[c + 2 * i], sl2, neg_m));
+            const float p1 = ex2(fmaf(s[c + 2 * i + 1], sl2, neg_m));
+            rs += p0 + p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st16(s_addr + (c >> 1), pk);
+        }
       }
       if (need && j > 0) {
         // O_w was last written by P V of tile j-1, which completed before S_w of tile j
@@ -306,7 +350,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int row = row0 + w * BM + r;
       const bool valid = row < row_end;
-      float inv = 1.f / l;
+      float inv = out_scale / l;
       if (w_gate_s != nullptr) {
         // softmax gate of the layer, g_s = sigmoid(q . w_s[h]) from this row of Q in shared
         // memory (128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7))
@@ -314,18 +358,32 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint8_t *qt = base + C::Q_OFF + w * C::TILE_BYTES;
         const float *ws_h = w_gate_s + h * D;
         float dot = 0.f;
+        constexpr int PER_CHUNK = 16 / C::EB;  // elements per 16-byte chunk
 #pragma unroll 1
-        for (int cl = 0; cl < D / 8; ++cl) {
+        for (int cl = 0; cl < D / PER_CHUNK; ++cl) {
           const uint4 raw = *reinterpret_cast<const uint4 *>(qt + (cl >> 3) * (BM * 128) + r * 128 +
                                                                (((cl & 7) ^ (r & 7)) << 4));
-          const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+          if (FP8) {
+            // dequantised e4m3 q (the per-head scale is applied once below)
+            const __nv_fp8x2_storage_t *pp = reinterpret_cast<const __nv_fp8x2_storage_t *>(&raw);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(hp[e]);
-            dot = fmaf(f.x, __ldg(ws_h + cl * 8 + 2 * e), dot);
-            dot = fmaf(f.y, __ldg(ws_h + cl * 8 + 2 * e + 1), dot);
+            for (int e = 0; e < 8; ++e) {
+              const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pp[e], __NV_E4M3);
+              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+              dot = fmaf(f.x, __ldg(ws_h + cl * 16 + 2 * e), dot);
+              dot = fmaf(f.y, __ldg(ws_h + cl * 16 + 2 * e + 1), dot);
+            }
+          } else {
+            const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(hp[e]);
+              dot = fmaf(f.x, __ldg(ws_h + cl * 8 + 2 * e), dot);
+              dot = fmaf(f.y, __ldg(ws_h + cl * 8 + 2 * e + 1), dot);
+            }
           }
         }
+        if (FP8) dot *= scales[h];  // s_q
         inv *= 1.f / (1.f + expf(-dot));
       }
       __nv_bfloat16 *orow = out + (int64_t)row * out_row_stride + (int64_t)h * D;
@@ -356,58 +414,62 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-template <int D>
+template <int D, bool FP8>
 cudaError_t launch_t(const Dims &d, const void *q, const void *k, const void *v, const void *kt, const void *vt,
-                     float sl2, void *o, int64_t o_row_stride, const float *w_gate_s, float *lse, char *ws,
-                     const WsPlan &p, cudaStream_t st) {
-  using C = Cfg<D>;
+                     const float *scales, float sl2, void *o, int64_t o_row_stride, const float *w_gate_s,
+                     float *lse, char *ws, const WsPlan &p, cudaStream_t st) {
+  using C = Cfg<D, FP8>;
   const uint64_t HD = (uint64_t)d.H * D;
+  const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap mq, mk, mv, mkt, mvt;
-  uint64_t strides[1] = {HD * 2};
-  uint32_t box[2] = {64, BM};
+  uint64_t strides[1] = {HD * C::EB};
+  uint32_t box[2] = {(uint32_t)C::BOX_ELEMS, BM};
   uint64_t dims_v[2] = {HD, (uint64_t)d.Nv()};
   uint64_t dims_t[2] = {HD, (uint64_t)(d.L > 0 ? d.L : 1)};
   const void *kt_base = d.L > 0 ? kt : k, *vt_base = d.L > 0 ? vt : v;  // unused when there is no text
-  if (!encode_tmap(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&mkt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kt_base, dims_t, strides, box,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&mvt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vt_base, dims_t, strides, box,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!encode_tmap(&mq, dt, 2, q, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mk, dt, 2, k, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mv, dt, 2, v, dims_v, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mkt, dt, 2, kt_base, dims_t, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&mvt, dt, 2, vt_base, dims_t, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(softmax_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  cudaError_t e = cudaFuncSetAttribute(softmax_tc_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int ntiles = host_tile_count(d);
-  softmax_tc_kernel<D><<<ntiles * d.H, THREADS, C::SMEM, st>>>(
-      mq, mk, mv, mkt, mvt, d, sl2, (__nv_bfloat16 *)o, o_row_stride, w_gate_s, lse, (const int32_t *)(ws + p.gtab),
-      (const int32_t *)(ws + p.tiles), (DevStatus *)(ws + p.status));
+  softmax_tc_kernel<D, FP8><<<ntiles * d.H, THREADS, C::SMEM, st>>>(
+      mq, mk, mv, mkt, mvt, d, sl2, scales, (__nv_bfloat16 *)o, o_row_stride, w_gate_s, lse,
+      (const int32_t *)(ws + p.gtab), (const int32_t *)(ws + p.tiles), (DevStatus *)(ws + p.status));
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool softmax_tc_supported(const Dims &d, vdn_dtype dt) {
-  return dt == VDN_BF16 && (d.D == 64 || d.D == 128);
+  return (dt == VDN_BF16 && (d.D == 64 || d.D == 128)) || (dt == VDN_E4M3 && d.D == 128);
 }
 
 cudaError_t launch_softmax_tc(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
                               const void *kt, const void *vt, const float *scales, float sl2, void *o, float *lse,
                               char *ws, const WsPlan &p, cudaStream_t st) {
-  (void)scales;
-  if (dt != VDN_BF16) return cudaErrorInvalidValue;
   const int64_t HD = (int64_t)d.H * d.D;
-  if (d.D == 128) return launch_t<128>(d, q, k, v, kt, vt, sl2, o, HD, nullptr, lse, ws, p, st);
-  if (d.D == 64) return launch_t<64>(d, q, k, v, kt, vt, sl2, o, HD, nullptr, lse, ws, p, st);
+  if (dt == VDN_E4M3 && d.D == 128)
+    return launch_t<128, true>(d, q, k, v, kt, vt, scales, sl2, o, HD, nullptr, lse, ws, p, st);
+  if (dt != VDN_BF16) return cudaErrorInvalidValue;
+  if (d.D == 128) return launch_t<128, false>(d, q, k, v, kt, vt, nullptr, sl2, o, HD, nullptr, lse, ws, p, st);
+  if (d.D == 64) return launch_t<64, false>(d, q, k, v, kt, vt, nullptr, sl2, o, HD, nullptr, lse, ws, p, st);
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_softmax_tc_gated(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
-                                    const void *vt, const float *w_gate_s, float sl2, void *a, char *ws,
-                                    const WsPlan &p, cudaStream_t st) {
+cudaError_t launch_softmax_tc_gated(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
+                                    const void *kt, const void *vt, const float *scales, const float *w_gate_s,
+                                    float sl2, void *a, char *ws, const WsPlan &p, cudaStream_t st) {
   const int64_t stride = 2 * (int64_t)d.H * d.D;  // A = [A_s | A_l]: the softmax half of each row
-  if (d.D == 128) return launch_t<128>(d, q, k, v, kt, vt, sl2, a, stride, w_gate_s, nullptr, ws, p, st);
-  if (d.D == 64) return launch_t<64>(d, q, k, v, kt, vt, sl2, a, stride, w_gate_s, nullptr, ws, p, st);
+  if (dt == VDN_E4M3 && d.D == 128)
+    return launch_t<128, true>(d, q, k, v, kt, vt, scales, sl2, a, stride, w_gate_s, nullptr, ws, p, st);
+  if (dt != VDN_BF16) return cudaErrorInvalidValue;
+  if (d.D == 128) return launch_t<128, false>(d, q, k, v, kt, vt, nullptr, sl2, a, stride, w_gate_s, nullptr, ws, p, st);
+  if (d.D == 64) return launch_t<64, false>(d, q, k, v, kt, vt, nullptr, sl2, a, stride, w_gate_s, nullptr, ws, p, st);
   return cudaErrorInvalidValue;
 }
 

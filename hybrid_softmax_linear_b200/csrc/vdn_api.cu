@@ -134,7 +134,8 @@ float scale_log2_of(float sm_scale, int D) {
 vdn_status softmax_dispatch(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
                             const void *kt, const void *vt, const float *scales, float sl2, void *o, float *lse,
                             char *ws, const WsPlan &p, cudaStream_t st) {
-  if (dt == VDN_E4M3) return fail(VDN_ERR_UNSUPPORTED, "e4m3 softmax branch not available");
+  if (dt == VDN_E4M3 && !softmax_tc_supported(d, dt))
+    return fail(VDN_ERR_UNSUPPORTED, "the e4m3 softmax branch needs head_dim 128");
   if (softmax_tc_supported(d, dt)) {
     ProfScope ps(K_SOFTMAX_TC, st);
     VDN_CUDA(launch_softmax_tc(d, dt, q, k, v, kt, vt, scales, sl2, o, lse, ws, p, st),
@@ -237,6 +238,28 @@ vdn_status vdn_softmax_branch_fwd(const vdn_shape *shape, vdn_dtype dtype, const
   VDN_CUDA(launch_tables(d, (char *)ws, p, st), "tables launch");
   VDN_TRY(softmax_dispatch(d, dtype, q, k, v, kt, vt, scales, scale_log2_of(sm_scale, d.D), o_s, lse, (char *)ws, p,
                            st));
+  return ok();
+}
+
+vdn_status vdn_fp8_quant_per_head(const vdn_shape *shape, const void *q, const void *k, const void *v, const void *kt,
+                                  const void *vt, void *q8, void *k8, void *v8, void *kt8, void *vt8, float *scales,
+                                  void *ws, size_t ws_bytes, vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  if ((int64_t)shape->heads * shape->head_dim > FP8_MAX_HD)
+    return fail(VDN_ERR_UNSUPPORTED, "H*D above %d", FP8_MAX_HD);
+  VDN_TRY(need(q, "q")); VDN_TRY(need(k, "k")); VDN_TRY(need(v, "v"));
+  VDN_TRY(need(q8, "q8")); VDN_TRY(need(k8, "k8")); VDN_TRY(need(v8, "v8")); VDN_TRY(need(scales, "scales"));
+  if (shape->text_tokens > 0) {
+    VDN_TRY(need(kt, "kt")); VDN_TRY(need(vt, "vt")); VDN_TRY(need(kt8, "kt8")); VDN_TRY(need(vt8, "vt8"));
+  }
+  const WsPlan p = plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16);
+  VDN_TRY(check_ws(ws, ws_bytes, p.step_end));
+  VDN_TRY(check_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  ProfScope ps(K_QUANT, st);
+  VDN_CUDA(launch_fp8_quant(dims_of(*shape), q, k, v, kt, vt, q8, k8, v8, kt8, vt8, scales,
+                            (uint32_t *)((char *)ws + p.qamax), st),
+           "fp8 quantisation launch");
   return ok();
 }
 
@@ -355,6 +378,8 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
   else if (beta != nullptr) return fail(VDN_ERR_INVALID_ARG, "beta must be NULL for VDN_LIN_ELU1");
   if (G_l != 1 && G_l != shape->head_dim) return fail(VDN_ERR_INVALID_ARG, "G_l must be 1 or D");
   if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(VDN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (dtype == VDN_E4M3 && (shape->head_dim != 128 || (int64_t)shape->heads * shape->head_dim > FP8_MAX_HD))
+    return fail(VDN_ERR_UNSUPPORTED, "the e4m3 layer needs head_dim 128 and H*D <= %d", FP8_MAX_HD);
   const WsPlan p = plan_workspace(*shape, kind, dtype);
   VDN_TRY(check_ws(ws, ws_bytes, p.total));
   VDN_TRY(check_device());
@@ -372,9 +397,22 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
   if (layer_fused(*shape, dtype)) {
     // tensor-core path: the softmax epilogue writes A_s = g_s * O_s and the linear read
     // writes A_l = g_l * gamma * RMSNorm(O_l), both straight into A
-    {
+    if (dtype == VDN_E4M3) {
+      // per-head e4m3 Q/K/V for the softmax branch; the linear branch keeps the bf16 inputs
+      {
+        ProfScope ps(K_QUANT, st);
+        VDN_CUDA(launch_fp8_quant(d, q, k, v, kt, vt, w + p.q8, w + p.k8, w + p.v8, w + p.kt8, w + p.vt8,
+                                  (float *)(w + p.scales), (uint32_t *)(w + p.amax), st),
+                 "fp8 quantisation launch");
+      }
       ProfScope ps(K_SOFTMAX_TC, st);
-      VDN_CUDA(launch_softmax_tc_gated(d, q, k, v, kt, vt, w_gate_s, scale_log2_of(0.f, d.D), A, w, p, st),
+      VDN_CUDA(launch_softmax_tc_gated(d, VDN_E4M3, w + p.q8, w + p.k8, w + p.v8, w + p.kt8, w + p.vt8,
+                                       (const float *)(w + p.scales), w_gate_s, scale_log2_of(0.f, d.D), A, w, p, st),
+               "softmax branch (tensor cores, e4m3) launch");
+    } else {
+      ProfScope ps(K_SOFTMAX_TC, st);
+      VDN_CUDA(launch_softmax_tc_gated(d, VDN_BF16, q, k, v, kt, vt, nullptr, w_gate_s, scale_log2_of(0.f, d.D), A, w,
+                                       p, st),
                "softmax branch (tensor cores) launch");
     }
     VDN_TRY(state_build_dispatch(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, w, p,

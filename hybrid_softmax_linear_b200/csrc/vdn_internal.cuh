@@ -128,7 +128,7 @@ VDN_HD size_t align_up(size_t x) { return (x + WS_ALIGN - 1) / WS_ALIGN * WS_ALI
 
 struct WsPlan {
   // step part (tables, tile list, status)
-  size_t status, ftab, gtab, meta, tiles, step_end;
+  size_t status, ftab, gtab, meta, qamax, tiles, step_end;
   // read staging: per-group summed memory in bf16 (tensor-core B operand), summed
   // normaliser, linear-gate weights in bf16
   size_t ssum, zsum, wl, stage_end;
@@ -154,6 +154,7 @@ inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dt
   p.ftab = take(F * 8 * 4);
   p.gtab = take(G * 16 * 4);
   p.meta = take(64);
+  p.qamax = take(3 * H * 4);
   p.tiles = take((size_t)max_tiles(s.frames, s.tokens_per_frame, s.chunk_frames) * TILE_REC * 4);
   p.step_end = off;
   p.ssum = take(G * H * D * D * 2);
@@ -292,9 +293,14 @@ cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf,
 // o_l (plain) or, with gate weights, A_l = g_l * gamma * RMSNorm(o_l) into the linear half of A
 cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void *out, const float *wgl, int G_l,
                            const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st);
-cudaError_t launch_softmax_tc_gated(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
-                                    const void *vt, const float *w_gate_s, float sl2, void *a, char *ws,
-                                    const WsPlan &p, cudaStream_t st);
+cudaError_t launch_softmax_tc_gated(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
+                                    const void *kt, const void *vt, const float *scales, const float *w_gate_s,
+                                    float sl2, void *a, char *ws, const WsPlan &p, cudaStream_t st);
+// per-head e4m3 quantisation of q, k (+ text), v (+ text); scales float[3][H]
+cudaError_t launch_fp8_quant(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
+                             const void *vt, void *q8, void *k8, void *v8, void *kt8, void *vt8, float *scales,
+                             uint32_t *amax_bits, cudaStream_t st);
+constexpr int FP8_MAX_HD = 256 * 8 * 8;  // column chunks the amax pass keeps in registers
 
 cudaError_t launch_fuse(const Dims &d, vdn_dtype dt, const void *q, const void *os, const void *ol,
                         const float *wgs, const float *wgl, int G_l, const float *gamma, float eps, void *a,

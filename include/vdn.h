@@ -123,7 +123,9 @@ VDN_API vdn_status vdn_workspace_init(void *ws, size_t ws_bytes, vdn_stream stre
  *   dtype VDN_F32:  q,k,v,kt,vt float; o_s float.
  *   dtype VDN_BF16: q,k,v,kt,vt bf16;  o_s bf16 (fp32 accumulation, fp32 softmax).
  *   dtype VDN_E4M3: q,k,v,kt,vt e4m3 with scales = float[3][H] (q, k, v dequantisation
- *                   scales per head; text shares the video k/v scales); o_s bf16.
+ *                   scales per head; text shares the video k/v scales), as written by
+ *                   vdn_fp8_quant_per_head; P is rounded to e4m3 at unit scale for P.V;
+ *                   o_s bf16; head_dim 128 only.
  *   lse: optional float[N_v][H], natural-log sum of exp of the scaled scores.
  * scales must be NULL unless dtype is VDN_E4M3. */
 VDN_API vdn_status vdn_softmax_branch_fwd(const vdn_shape *shape, vdn_dtype dtype, const void *q, const void *k,
@@ -153,6 +155,18 @@ VDN_API vdn_status vdn_softmax_branch_fwd(const vdn_shape *shape, vdn_dtype dtyp
 VDN_API vdn_status vdn_softmax_branch_fwd_noalloc(const vdn_shape *shape, vdn_dtype dtype, const void *q,
                                                   const void *k, const void *v, const void *kt, const void *vt,
                                                   float sm_scale, void *o_s, float *lse, vdn_stream stream);
+
+/* vdn_fp8_quant_per_head — per-head e4m3 quantisation of the softmax branch's inputs
+ * ([CARD] "Inference with Diffusers": fp8 e4m3).  For each head h and tensor X in
+ * (q; k with kt; v with vt): s_X[h] = amax / 448 over the video rows and, for k and v,
+ * the text rows too (text shares the video scale); X8 = e4m3(X / s_X[h]), round to
+ * nearest even, saturating.  Inputs bf16 [N_v][H][D] and [L][H][D]; outputs e4m3 bytes
+ * in the same layouts; scales float[3][H] (q, k, v), the dequantisation factors that
+ * vdn_softmax_branch_fwd takes with VDN_E4M3.  An all-zero head gets scale 1.
+ * Requires H*D <= 16384.  ws: vdn_step_workspace_size bytes. */
+VDN_API vdn_status vdn_fp8_quant_per_head(const vdn_shape *shape, const void *q, const void *k, const void *v,
+                                          const void *kt, const void *vt, void *q8, void *k8, void *v8, void *kt8,
+                                          void *vt8, float *scales, void *ws, size_t ws_bytes, vdn_stream stream);
 
 /* ------------------------------------------------------------------ linear branch
  * vdn_linear_state_build — per-frame states.  [ART] 局部精确计算 para. 1 (frame-wise

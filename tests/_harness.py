@@ -50,9 +50,11 @@ def f32view(x):
 class Run:
     """Device copies of one input set plus a workspace for the layer."""
 
-    def __init__(self, shape: synth.Shape, inp: dict, dtype: str, kind: int = vdn.ELU1, G_l: int | None = None):
+    def __init__(self, shape: synth.Shape, inp: dict, dtype: str, kind: int = vdn.ELU1, G_l: int | None = None,
+                 layer_dtype: int | None = None):
         self.shape, self.inp, self.dtype, self.kind = shape, inp, dtype, kind
-        self.cdt = vdn.F32 if dtype == "f32" else vdn.BF16
+        # dtype of the layer call (VDN_E4M3 runs the softmax branch in e4m3 on bf16 inputs)
+        self.cdt = layer_dtype if layer_dtype is not None else (vdn.F32 if dtype == "f32" else vdn.BF16)
         self.dev = {n: to_device(a) for n, a in inp.items()}
         self.G_l = inp["w_gate_l"].shape[2] if G_l is None else G_l
         s = shape
@@ -60,12 +62,12 @@ class Run:
         vdn.workspace_init(self.ws)
         self.Nv, self.H, self.D = s.n_video, s.heads, s.head_dim
 
-    def layer(self, ltype=None):
+    def layer(self):
         d = self.dev
         y = empty((self.Nv, self.H * self.D), self.dtype)
-        vdn.hybrid_attn_fwd(self.shape, self.kind, self.cdt if ltype is None else ltype, d["q"], d["k"], d["v"],
-                            d["kt"], d["vt"], d.get("beta") if self.kind == vdn.DELTA else None, d["w_gate_s"],
-                            d["w_gate_l"], self.G_l, d["gamma"], 1e-6, d["w_os"], d["w_ol"], y, self.ws)
+        vdn.hybrid_attn_fwd(self.shape, self.kind, self.cdt, d["q"], d["k"], d["v"], d["kt"], d["vt"],
+                            d.get("beta") if self.kind == vdn.DELTA else None, d["w_gate_s"], d["w_gate_l"],
+                            self.G_l, d["gamma"], 1e-6, d["w_os"], d["w_ol"], y, self.ws)
         vdn.check_device_status(self.ws)
         return y
 

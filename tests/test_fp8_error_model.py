@@ -1,0 +1,38 @@
+"""CPU pin of the e4m3 error bound used for the softmax branch on the GPU.
+
+Per-head e4m3 rounding (3 mantissa bits, about 2.6% RMS relative error per value) of Q,
+K, V and P cannot reproduce a float64 softmax to 3e-2 on unit-Gaussian data: the
+rounded scores shift the weights by about 3.7%, and the rounded V and P add about 2.6%
+each.  This test measures that model error with torch's own CPU e4m3 conversion on a
+query block with the key count and head size of the full-size workload (17,648 keys,
+D = 128), and checks that the GPU bound of 7e-2 sits above it with margin.  The kernel
+itself is held to 3e-2 against the oracle evaluated on its own e4m3 inputs."""
+import numpy as np
+import torch
+
+GPU_BOUND = 7e-2
+
+
+def _e4m3(x, amax):
+    s = amax / 448.0
+    return (x / s).float().to(torch.float8_e4m3fn).double() * s
+
+
+def test_e4m3_attention_model_error():
+    g = torch.Generator().manual_seed(0)
+    n, nk, d = 128, 17648, 128
+    q = torch.randn(n, d, generator=g, dtype=torch.float64)
+    k = torch.randn(nk, d, generator=g, dtype=torch.float64)
+    v = torch.randn(nk, d, generator=g, dtype=torch.float64)
+    ref = torch.softmax(q @ k.T / d ** 0.5, -1) @ v
+    q8, k8, v8 = (_e4m3(x, x.abs().max()) for x in (q, k, v))
+    s = q8 @ k8.T / d ** 0.5
+    p = torch.exp(s - s.max(-1, keepdim=True).values)
+    p8 = p.float().to(torch.float8_e4m3fn).double()           # unit scale
+    out = (p8 @ v8) / p.sum(-1, keepdim=True)
+    err = ((out - ref).norm() / ref.norm()).item()
+    assert 0.03 < err < 0.8 * GPU_BOUND, err                  # above the 3e-2 bar, below the bound
+    # with only P rounded (the kernel's own arithmetic on e4m3 inputs) the error is inside 3e-2
+    ref8 = torch.softmax(s, -1) @ v8
+    err_p = (((p8 @ v8) / p.sum(-1, keepdim=True) - ref8).norm() / ref8.norm()).item()
+    assert err_p < 0.03, err_p
