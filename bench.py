@@ -283,6 +283,11 @@ def run_ours(args, rank, world, local_rank):
     sm_avg = sm_ms / max(sm_n, 1)
     achieved = fl["softmax"] / (sm_avg / 1e3) / 1e12 if sm_avg > 0 else None
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_note = f"{peak_src} bf16_tflops_sustained (kernel runs inside a long step)"
+    if w.softmax_fp8:
+        # e4m3 contraction: the measured bf16 peak times the nominal fp8/bf16 ratio (4.5 / 2.25)
+        peak *= 2.0
+        peak_note = f"{peak_src} bf16_tflops_sustained x 2 (nominal fp8/bf16 ratio; kernel runs inside a long step)"
     launches = sum(n for _, n in prof.values())
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -290,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic", "config": workload_config(cfg),
         "roofline": {"kernel": sm_key, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": None,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel runs inside a long step)",
+                     "peak_source": peak_note,
                      "algorithmic_tflop_per_launch": fl["softmax"] / 1e12, "avg_launch_ms": sm_avg},
         "layer_tflops": sum(v for k, v in fl.items()) / (per_step_ms / 1e3) / 1e12,
         "per_kernel_ms_per_step": {k: round(v[0] / max(args.steps, 1), 4) for k, v in prof.items()},

@@ -235,21 +235,32 @@ __global__ void __launch_bounds__(256) read_stage_kernel(int64_t n_s8, int64_t n
 }
 
 // ============================================================================ read (+ gate, RMSNorm)
+// One CTA per 128 query rows (half of a 256-row tile) and head; two CTAs fit on an SM.
+// Warp 0 loads Q, S_sum and W_l with TMA and one of its threads issues the MMAs: the gate
+// logits Q W_l as soon as Q lands, then num = feature * S_sum once the feature rows are
+// in place.  Warps 1-4 (one query row per thread) compute the feature row phi(q) (or
+// q/|q|), the normaliser phi(q).z and, with G_l = 1, the scalar gate, keep it in
+// registers until the gate MMA has consumed Q, and write it over Q; then they form
+// o = num / den and store o (plain) or A_l = g_l * gamma * o / rms(o) (layer).
 namespace rd {
-constexpr int D = 128, BM = 128, NQ = 2, THREADS = 320;
+constexpr int D = 128, BM = 128, THREADS = 160;
 constexpr int TILE_BYTES = BM * D * 2;  // 32 KB: one 128-row bf16 tile (two 64-column boxes)
-constexpr int Q_OFF = 0, F_OFF = NQ * TILE_BYTES, S_OFF = 2 * NQ * TILE_BYTES, W_OFF = S_OFF + TILE_BYTES;
-constexpr int BAR_OFF = W_OFF + TILE_BYTES;
+constexpr int Q_OFF = 0, S_OFF = TILE_BYTES, W_OFF = 2 * TILE_BYTES;
+constexpr int BAR_OFF = 3 * TILE_BYTES;
 constexpr uint32_t IDESC_NUM = idesc_bf16(BM, D, false, true);   // A K-major, B MN-major
+constexpr uint32_t TMEM_COLS = 256;                               // num at 0, gate logits at 128
 struct alignas(8) Bars {
-  uint64_t in_full, feat[NQ], acc[NQ], drain;
+  uint64_t in_full, gate_done, feat, acc, drain;
   uint32_t tmem;
   int abort;
+  float z[D], gamma[D], wg1[D];
 };
 constexpr size_t SMEM = 1024 + BAR_OFF + sizeof(Bars);
 }  // namespace rd
 
-__global__ void __launch_bounds__(rd::THREADS, 1)
+__device__ __forceinline__ float fast_sigmoid(float x) { return __frcp_rn(1.f + __expf(-x)); }
+
+__global__ void __launch_bounds__(rd::THREADS, 2)
     read_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                    const __grid_constant__ CUtensorMap tmW, Dims d, int delta, int gate_mma,
                    const float *__restrict__ zsum, const float *__restrict__ wgl, int G_l,
@@ -267,82 +278,80 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
   if (skip) return;
 
   const int h = blockIdx.y;
-  const int32_t *tr = tiles + (int64_t)blockIdx.x * TILE_REC;
-  const int g = tr[0], row0 = tr[1], row_end = tr[2];
+  const int32_t *tr = tiles + (int64_t)(blockIdx.x >> 1) * TILE_REC;
+  const int g = tr[0];
+  const int row0 = tr[1] + (blockIdx.x & 1) * BM, row_end = tr[2];
+  if (row0 >= row_end) return;  // the second half of a short tile (block-uniform)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->in_full), 1);
-    for (int w = 0; w < NQ; ++w) { mbar_init(smem_u32(&bars->feat[w]), 4); mbar_init(smem_u32(&bars->acc[w]), 1); }
+    mbar_init(smem_u32(&bars->gate_done), 1);
+    mbar_init(smem_u32(&bars->feat), 4);
+    mbar_init(smem_u32(&bars->acc), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) { tmem_alloc(smem_u32(&bars->tmem), 512); tmem_relinquish(); }
+  if (threadIdx.x < D) {
+    bars->z[threadIdx.x] = delta ? 0.f : zsum[((int64_t)g * d.H + h) * D + threadIdx.x];
+    bars->gamma[threadIdx.x] = fused ? gamma[(int64_t)h * D + threadIdx.x] : 0.f;
+    bars->wg1[threadIdx.x] = (fused && !gate_mma) ? wgl[((int64_t)h * D + threadIdx.x) * G_l] : 0.f;
+  }
+  if (warp == 0) { tmem_alloc(smem_u32(&bars->tmem), TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem;  // num_w at 128w, gate logits of half w at 256 + 128w
+  const uint32_t tmem = bars->tmem;
 
   if (warp == 0) {
     if (lane == 0) {
       const uint32_t fb = smem_u32(&bars->in_full);
-      mbar_arrive_expect_tx(fb, (NQ + 1 + (gate_mma ? 1 : 0)) * TILE_BYTES);
-      for (int w = 0; w < NQ; ++w)
-        for (int b = 0; b < 2; ++b)
-          tma_load_2d(smem_u32(base + Q_OFF + w * TILE_BYTES + b * BM * 128), &tmQ, fb, h * D + b * 64, row0 + w * BM);
+      mbar_arrive_expect_tx(fb, (2 + (gate_mma ? 1 : 0)) * TILE_BYTES);
       for (int b = 0; b < 2; ++b) {
+        tma_load_2d(smem_u32(base + Q_OFF + b * BM * 128), &tmQ, fb, h * D + b * 64, row0);
         tma_load_2d(smem_u32(base + S_OFF + b * BM * 128), &tmS, fb, b * 64, (g * d.H + h) * D);
         if (gate_mma) tma_load_2d(smem_u32(base + W_OFF + b * BM * 128), &tmW, fb, b * 64, h * D);
       }
-      int no_abort = 0;
-      mbar_wait(fb, 0, &no_abort, st, K_READ, 1);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      bool ok = mbar_wait(smem_u32(&bars->in_full), 0, abort_flag, st, K_READ, 2);
+      bool ok = mbar_wait(fb, 0, abort_flag, st, K_READ, 1);
       if (ok) {
         tc_fence_after();
-        const uint32_t sb_ = smem_u32(base + S_OFF), wb = smem_u32(base + W_OFF);
+        const uint32_t qa = smem_u32(base + Q_OFF), sb_ = smem_u32(base + S_OFF), wb = smem_u32(base + W_OFF);
         if (gate_mma) {
-          for (int w = 0; w < NQ; ++w) {
-            const uint32_t qa = smem_u32(base + Q_OFF + w * TILE_BYTES);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tmem + 256 + 128 * w, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
-                     sdesc(wb + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
-          }
-        }
-        for (int w = 0; w < NQ && ok; ++w) {
-          if (!mbar_wait(smem_u32(&bars->feat[w]), 0, abort_flag, st, K_READ, 3)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t fa = smem_u32(base + F_OFF + w * TILE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + 128 * w, sdesc(fa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
+            mma_ss(tmem + 128, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc(wb + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
+        }
+        mma_commit(smem_u32(&bars->gate_done));  // Q may be overwritten once this arrives
+        if (mbar_wait(smem_u32(&bars->feat), 0, abort_flag, st, K_READ, 3)) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
                    sdesc(sb_ + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
-          mma_commit(smem_u32(&bars->acc[w]));
+          mma_commit(smem_u32(&bars->acc));
         }
       }
       mma_commit(smem_u32(&bars->drain));
       int no_abort = 0;
+      mbar_wait(fb, 0, &no_abort, st, K_READ, 2);
       mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_READ, 4);
     }
   } else {
-    const int w = (warp - 2) >> 2, quad = warp & 3, r = quad * 32 + lane;
-    const int row = row0 + w * BM + r;
+    const int quad = warp & 3, r = quad * 32 + lane;
+    const int row = row0 + r;
     const bool valid = row < row_end;
-    const uint8_t *qt = base + Q_OFF + w * TILE_BYTES;
-    uint8_t *ft = base + F_OFF + w * TILE_BYTES;
+    uint8_t *qt = base + Q_OFF;
     const bool got = mbar_wait(smem_u32(&bars->in_full), 0, abort_flag, st, K_READ, 5);
     bool ok = __all_sync(0xffffffffu, got);
-    float den = 0.f, scal_gate = 0.f, inv_norm = 1.f;
+    float den = 0.f, gate1 = 0.f;
     if (ok) {
-      // feature of this row: phi(q) (and the normaliser phi(q).z), or q/|q| (delta rule)
-      const float *zg = zsum + ((int64_t)g * d.H + h) * D;
-      const float *wg1 = wgl + (int64_t)h * D * G_l;
+      // feature row in registers (bf16 pairs): phi(q), or q/|q| for the delta rule
+      uint32_t fr[D / 2];
+      float inv_norm = 1.f;
       if (delta) {
         float ss = 0.f;
-#pragma unroll 4
+#pragma unroll
         for (int cl = 0; cl < D / 8; ++cl) {
           float f[8];
           unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
@@ -351,78 +360,86 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
         }
         inv_norm = ss > 0.f ? rsqrtf(ss) : 0.f;
       }
-#pragma unroll 2
+#pragma unroll
       for (int cl = 0; cl < D / 8; ++cl) {
         float f[8];
         unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
-        if (fused && !gate_mma) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) scal_gate = fmaf(f[e], __ldg(wg1 + (cl * 8 + e) * G_l), scal_gate);
-        }
+        for (int e = 0; e < 8; ++e) gate1 = fmaf(f[e], bars->wg1[cl * 8 + e], gate1);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           if (delta) {
             f[e] *= inv_norm;
           } else {
-            f[e] = f[e] > 0.f ? f[e] + 1.f : expf(f[e]);
-            den = fmaf(f[e], __ldg(zg + cl * 8 + e), den);
+            f[e] = f[e] > 0.f ? f[e] + 1.f : __expf(f[e]);
+            den = fmaf(f[e], bars->z[cl * 8 + e], den);
           }
         }
-        *reinterpret_cast<uint4 *>(ft + swz_off(r, cl, BM)) = pack8(f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) fr[cl * 4 + e] = pack_bf16(f[2 * e], f[2 * e + 1]);
       }
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->feat[w]));
-      const bool done = mbar_wait(smem_u32(&bars->acc[w]), 0, abort_flag, st, K_READ, 6);
-      ok = __all_sync(0xffffffffu, done);
+      // Q is the A operand of the gate MMA: write the features over it only afterwards
+      const bool gd = mbar_wait(smem_u32(&bars->gate_done), 0, abort_flag, st, K_READ, 7);
+      ok = __all_sync(0xffffffffu, gd);
+      if (ok) {
+#pragma unroll
+        for (int cl = 0; cl < D / 8; ++cl)
+          *reinterpret_cast<uint4 *>(qt + swz_off(r, cl, BM)) =
+              make_uint4(fr[cl * 4], fr[cl * 4 + 1], fr[cl * 4 + 2], fr[cl * 4 + 3]);
+        fence_proxy_async();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->feat));
+        const bool done = mbar_wait(smem_u32(&bars->acc), 0, abort_flag, st, K_READ, 6);
+        ok = __all_sync(0xffffffffu, done);
+      }
     }
     if (ok) {
       tc_fence_after();
       const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-      float o[D];
+      const float scale = delta ? 1.f : (den > 0.f ? 1.f / den : 0.f);
+      __nv_bfloat16 *orow = out + (int64_t)row * out_stride + (int64_t)h * D;
+      // the accumulator is read twice (sum of squares, then the output) to keep registers low
+      float rinv = 1.f;
+      if (fused) {
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < D; c += 64) {
+          uint32_t u0[32], u1[32];
+          tmem_ld32(tmem + lane_off + c, u0);
+          tmem_ld32(tmem + lane_off + c + 32, u1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float a = __uint_as_float(u0[i]) * scale, b = __uint_as_float(u1[i]) * scale;
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+          }
+        }
+        rinv = rsqrtf(ss / (float)D + eps);
+      }
+      const float gs = fast_sigmoid(gate1);
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_off + 128 * w + c, u);
+        uint32_t u[32], ug[32];
+        tmem_ld32(tmem + lane_off + c, u);
+        if (fused && gate_mma) tmem_ld32(tmem + lane_off + 128 + c, ug);
         tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[c + i] = __uint_as_float(u[i]);
-      }
-      const float scale = delta ? 1.f : (den > 0.f ? 1.f / den : 0.f);
-      float ss = 0.f;
-#pragma unroll
-      for (int j = 0; j < D; ++j) { o[j] *= scale; ss = fmaf(o[j], o[j], ss); }
-      __nv_bfloat16 *orow = out + (int64_t)row * out_stride + (int64_t)h * D;
-      if (!fused) {
         if (valid) {
 #pragma unroll
-          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4 *>(orow + c) = pack8(o + c);
-        }
-      } else {
-        const float rinv = rsqrtf(ss / (float)D + eps);
-        const float gs = 1.f / (1.f + expf(-scal_gate));
-        const float *gm = gamma + (int64_t)h * D;
+          for (int v = 0; v < 32; v += 8) {
+            float a[8];
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          float gl[32];
-          if (gate_mma) {
-            uint32_t u[32];
-            tmem_ld32(tmem + lane_off + 256 + 128 * w + c, u);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) gl[i] = 1.f / (1.f + expf(-__uint_as_float(u[i])));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) gl[i] = gs;
-          }
-          if (valid) {
-#pragma unroll
-            for (int v = 0; v < 32; v += 8) {
-              float a[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) a[e] = gl[v + e] * __ldg(gm + c + v + e) * o[c + v + e] * rinv;
-              *reinterpret_cast<uint4 *>(orow + c + v) = pack8(a);
+            for (int e = 0; e < 8; ++e) {
+              const float o = __uint_as_float(u[v + e]) * scale;
+              if (!fused) {
+                a[e] = o;
+              } else {
+                const float gl = gate_mma ? fast_sigmoid(__uint_as_float(ug[v + e])) : gs;
+                a[e] = gl * bars->gamma[c + v + e] * o * rinv;
+              }
             }
+            *reinterpret_cast<uint4 *>(orow + c + v) = pack8(a);
           }
         }
       }
@@ -431,7 +448,7 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 }  // namespace
@@ -504,7 +521,7 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
   if (e != cudaSuccess) return e;
   const int64_t stride = fused ? 2 * (int64_t)HD : (int64_t)HD;
   __nv_bfloat16 *o = (__nv_bfloat16 *)out + (fused ? HD : 0);  // fused: the linear half of A
-  read_tc_kernel<<<dim3(host_tile_count(d), d.H), THREADS, SMEM, st>>>(
+  read_tc_kernel<<<dim3(2 * host_tile_count(d), d.H), THREADS, SMEM, st>>>(
       mq, ms, mw, d, kind == VDN_LIN_DELTA, gate_mma ? 1 : 0, (const float *)(ws + p.zsum),
       fused ? wgl : nullptr, G_l, gamma, eps, o, stride, fused ? 1 : 0, (const int32_t *)(ws + p.tiles),
       (DevStatus *)(ws + p.status));

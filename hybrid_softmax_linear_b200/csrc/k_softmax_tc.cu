@@ -16,6 +16,10 @@
 // Keys past the end of a segment are masked in the last tile of that segment.
 #include "tc_common.cuh"
 
+#ifndef VDN_SOFTMAX_POLY_EIGHTHS
+#define VDN_SOFTMAX_POLY_EIGHTHS 0
+#endif
+
 namespace vdn {
 namespace {
 
@@ -94,6 +98,36 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA and integer pipes, for a share of the exponentials, so that the
+// hardware exponential unit (shared by both softmax warpgroups) is not the only path.
+// Range reduction: x = n + f with n = round(x) (read from the low mantissa bits after
+// adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial, fitted here for
+// minimal relative error on [-1/2, 1/2] (iteratively reweighted least squares, Lawson's
+// method; max relative error 7.5e-5, below bf16's 2^-9); 2^n is added to the exponent
+// field.  x is clamped to -125 so that the result stays a normal float (~1e-38 there).
+constexpr int POLY_EIGHTHS = VDN_SOFTMAX_POLY_EIGHTHS;  // eighths of the exponentials computed this way
+
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float j = x + 12582912.f;
+  const float n = j - 12582912.f;
+  const float f = x - n;
+  const float p = fmaf(fmaf(fmaf(0.05517132f, f, 0.24261054f), f, 0.69326097f), f, 0.99992812f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(j) << 23));
+}
+
+// element idx of a row (a compile-time constant once the loops are unrolled)
+__device__ __forceinline__ float exp2_mixed(float x, int idx) {
+  return (idx & 7) < POLY_EIGHTHS ? exp2_poly(x) : ex2(x);
+}
+
+// three-input max of sm_100 (half the instructions of a pairwise max tree)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 template <int D, bool FP8>
@@ -212,10 +246,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       };
       bool ok = mbar_wait(smem_u32(&bars->q_full), 0, abort_flag, st, K_SOFTMAX_TC, 3);
       if (ok) ok = mbar_wait(smem_u32(&bars->k_full[0]), 0, abort_flag, st, K_SOFTMAX_TC, 4);
+      // Q tile 1 starts half a step behind Q tile 0: its first S is issued only once P_0 of
+      // tile 0 is ready.  In steady state each warpgroup then exponentiates while the tensor
+      // cores run the other one's P.V and next S, instead of both competing for the
+      // exponential units at the same time.
       if (ok) {
         tc_fence_after();
-        for (int w = 0; w < NQ; ++w) issue_s(w, 0);
-        mma_commit(smem_u32(&bars->k_empty[0]));
+        issue_s(0, 0);
       }
       for (int j = 0; ok && j < nkv; ++j) {
         const int vs = j % VST;
@@ -237,6 +274,10 @@ __global__ void __launch_bounds__(THREADS, 1)
               mma_ts_f8(tmem + C::o_col(w), tmem + C::s_col(w) + kk * 8, bdesc, C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
             else
               mma_ts(tmem + C::o_col(w), tmem + C::s_col(w) + kk * 8, bdesc, C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (j == 0 && w == 0) {
+            issue_s(1, 0);                               // staggered start of Q tile 1
+            mma_commit(smem_u32(&bars->k_empty[0]));     // K tile 0 is free once both S of it complete
           }
           if (more) issue_s(w, j + 1);
         }
@@ -267,23 +308,38 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool got = mbar_wait(smem_u32(&bars->s_full[w]), j & 1, abort_flag, st, K_SOFTMAX_TC, 9);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
+      // the whole row of S in one round trip: four loads in flight, one wait
       float s[BN];
-#pragma unroll
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(s_addr + c, u);
+      {
+        uint32_t u0[32], u1[32], u2[32], u3[32];
+        tmem_ld32(s_addr + 0, u0);
+        tmem_ld32(s_addr + 32, u1);
+        tmem_ld32(s_addr + 64, u2);
+        tmem_ld32(s_addr + 96, u3);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(u[i]);
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(u0[i]);
+          s[32 + i] = __uint_as_float(u1[i]);
+          s[64 + i] = __uint_as_float(u2[i]);
+          s[96 + i] = __uint_as_float(u3[i]);
+        }
       }
       if (nvalid < BN) {
 #pragma unroll
         for (int i = 0; i < BN; ++i)
           if (i >= nvalid) s[i] = -INFINITY;
       }
-      float mx = s[0];
+      // row max as a tree of three-input maxima (eight independent chains)
+      float mx8[8];
 #pragma unroll
-      for (int i = 1; i < BN; ++i) mx = fmaxf(mx, s[i]);
+      for (int k = 0; k < 8; ++k) {
+        mx8[k] = s[k];
+#pragma unroll
+        for (int t = 0; t < 7; ++t) mx8[k] = max3(mx8[k], s[8 + 16 * t + k], s[16 + 16 * t + k]);
+        mx8[k] = fmaxf(mx8[k], s[120 + k]);
+      }
+      const float mx = fmaxf(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], max3(mx8[5], mx8[6], mx8[7])));
       const float m_new = fmaxf(m, mx * sl2);
       const bool need = __any_sync(0xffffffffu, m_new > m + RESCALE_THRESHOLD);
       float alpha = 1.f;
@@ -291,7 +347,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         alpha = ex2(m - m_new);   // 0 on the first tile (m = -inf)
         m = m_new;
       }
-      float rs = 0.f;
+      float rs8[8];               // row sum in eight independent chains
+#pragma unroll
+      for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
       const float neg_m = -m;
       if (FP8) {
         // e4m3 P at unit scale, four per tensor-memory column (p <= 2^8 < 448)
@@ -303,8 +361,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             float p[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              p[e] = ex2(fmaf(s[c + 4 * i + e], sl2, neg_m));
-              rs += p[e];
+              p[e] = exp2_mixed(fmaf(s[c + 4 * i + e], sl2, neg_m), 4 * i + e);
+              rs8[(4 * i + e) & 7] += p[e];
             }
             const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p[0], p[1]), __NV_SATFINITE, __NV_E4M3);
             const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p[2], p[3]), __NV_SATFINITE, __NV_E4M3);
@@ -318,9 +376,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(s[c + 2 * i], sl2, neg_m));
-            const float p1 = ex2(fmaf(s[c + 2 * i + 1], sl2, neg_m));
-            rs += p0 + p1;
+            const float p0 = exp2_mixed(fmaf(s[c + 2 * i], sl2, neg_m), 2 * i);
+            const float p1 = exp2_mixed(fmaf(s[c + 2 * i + 1], sl2, neg_m), 2 * i + 1);
+            rs8[(2 * i) & 7] += p0;
+            rs8[(2 * i + 1) & 7] += p1;
             pk[i] = pack_bf16(p0, p1);
           }
           tmem_st16(s_addr + (c >> 1), pk);
@@ -338,6 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_st16(o_addr + c, u);
         }
       }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l = l * alpha + rs;
       tmem_wait_st();
       tc_fence_before();

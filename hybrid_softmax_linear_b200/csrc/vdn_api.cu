@@ -397,6 +397,16 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
   if (layer_fused(*shape, dtype)) {
     // tensor-core path: the softmax epilogue writes A_s = g_s * O_s and the linear read
     // writes A_l = g_l * gamma * RMSNorm(O_l), both straight into A
+    VDN_TRY(state_build_dispatch(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, w, p,
+                                 st));
+    {
+      ProfScope ps(K_SCAN, st);
+      VDN_CUDA(launch_state_scan(d, kind, S, z, St, zt, beta, Sf, Sb, zf, zb, w, p, st), "scan launch");
+    }
+    {
+      ProfScope ps(K_READ_STAGE, st);
+      VDN_CUDA(launch_read_stage(d, kind, Sf, Sb, zf, zb, w_gate_l, G_l, w, p, st), "read staging");
+    }
     if (dtype == VDN_E4M3) {
       // per-head e4m3 Q/K/V for the softmax branch; the linear branch keeps the bf16 inputs
       {
@@ -414,16 +424,6 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
       VDN_CUDA(launch_softmax_tc_gated(d, VDN_BF16, q, k, v, kt, vt, nullptr, w_gate_s, scale_log2_of(0.f, d.D), A, w,
                                        p, st),
                "softmax branch (tensor cores) launch");
-    }
-    VDN_TRY(state_build_dispatch(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, w, p,
-                                 st));
-    {
-      ProfScope ps(K_SCAN, st);
-      VDN_CUDA(launch_state_scan(d, kind, S, z, St, zt, beta, Sf, Sb, zf, zb, w, p, st), "scan launch");
-    }
-    {
-      ProfScope ps(K_READ_STAGE, st);
-      VDN_CUDA(launch_read_stage(d, kind, Sf, Sb, zf, zb, w_gate_l, G_l, w, p, st), "read staging");
     }
     {
       ProfScope ps(K_READ_TC, st);
