@@ -482,10 +482,11 @@ cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf,
                               const float *zb, const float *wgl, int G_l, char *ws, const WsPlan &p,
                               cudaStream_t st) {
   const int64_t G = host_group_count(d), DD = (int64_t)d.D * d.D;
-  const int64_t n_s8 = G * d.H * DD / 8;
-  const int64_t n_z = kind == VDN_LIN_ELU1 ? G * d.H * d.D : 0;
+  const int64_t n_s8 = Sf != nullptr ? G * d.H * DD / 8 : 0;
+  const int64_t n_z = (Sf != nullptr && kind == VDN_LIN_ELU1) ? G * d.H * d.D : 0;
   const int64_t n_w8 = (wgl != nullptr && G_l == d.D) ? (int64_t)d.H * DD / 8 : 0;
   const int64_t n = n_s8 + n_z + n_w8;
+  if (n == 0) return cudaSuccess;
   read_stage_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
       n_s8, n_z, n_w8, Sf, Sb, zf, zb, wgl, (__nv_bfloat16 *)(ws + p.ssum), (float *)(ws + p.zsum),
       (__nv_bfloat16 *)(ws + p.wl));

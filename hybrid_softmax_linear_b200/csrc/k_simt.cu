@@ -361,12 +361,132 @@ __global__ void __launch_bounds__(256) scan_delta_kernel(Dims d, const float *__
   }
 }
 
+// Segmented scan of the ELU1 memories.  A block owns 128 consecutive entries (32 lanes x
+// float4) of the flattened [D*D | D] state of one head.  Its warps first sum the frames
+// of each segment (the frames between two consecutive memory boundaries; four loads in
+// flight per lane), then warp 0 forms the exclusive prefix sums and warp 1 the suffix
+// sums over the segments, and every group's memories are read off those:
+// S_fwd = S_txt/2 + prefix[ie_g], S_bwd = S_txt/2 + suffix[ib_g].  With SUM the block
+// stores S_fwd + S_bwd in bf16 and z_fwd + z_bwd in float, the operands of the
+// tensor-core read, instead of the four float memories.
+constexpr int SCAN_THREADS = 256;
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float4 f4add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+template <bool SUM>
+__global__ void __launch_bounds__(SCAN_THREADS) scan_seg_kernel(Dims d, const float *__restrict__ S,
+                                                                const float *__restrict__ z,
+                                                                const float *__restrict__ St,
+                                                                const float *__restrict__ zt, float *__restrict__ Sf,
+                                                                float *__restrict__ Sb, float *__restrict__ zf,
+                                                                float *__restrict__ zb,
+                                                                __nv_bfloat16 *__restrict__ ssum,
+                                                                float *__restrict__ zsum,
+                                                                const int32_t *__restrict__ splan, int gcap) {
+  extern __shared__ float4 sm4[];
+  const int nseg = splan[0], G = splan[1];
+  float4 *seg = sm4, *pre = sm4 + nseg * 32, *suf = pre + (nseg + 1) * 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int D = d.D, h = blockIdx.y;
+  const int64_t DD = (int64_t)D * D;
+  const int64_t c0 = (int64_t)blockIdx.x * 128;
+  const bool isz = c0 >= DD;  // D*D is a multiple of 128: a block never straddles S and z
+  const int64_t per = isz ? D : DD;
+  const int64_t off = (isz ? c0 - DD : c0) + lane * 4;
+  const bool valid = off < per;
+  const float *src = (isz ? z : S) + h * per + off;
+  const int64_t fstride = (int64_t)d.H * per;
+  const int32_t *bnd = splan + 4;
+  for (int j = warp; j < nseg; j += SCAN_THREADS / 32) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (valid) {
+      const int hi = bnd[j + 1];
+      int f = bnd[j];
+      for (; f + 4 <= hi; f += 4) {
+        const float4 x0 = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)f * fstride));
+        const float4 x1 = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(f + 1) * fstride));
+        const float4 x2 = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(f + 2) * fstride));
+        const float4 x3 = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(f + 3) * fstride));
+        a = f4add(a, f4add(x0, x1));
+        b = f4add(b, f4add(x2, x3));
+      }
+      for (; f < hi; ++f) a = f4add(a, __ldg(reinterpret_cast<const float4 *>(src + (int64_t)f * fstride)));
+    }
+    seg[j * 32 + lane] = f4add(a, b);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < nseg; ++j) { pre[j * 32 + lane] = acc; acc = f4add(acc, seg[j * 32 + lane]); }
+    pre[nseg * 32 + lane] = acc;
+  } else if (warp == 1) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    suf[nseg * 32 + lane] = acc;
+    for (int j = nseg - 1; j >= 0; --j) { acc = f4add(acc, seg[j * 32 + lane]); suf[j * 32 + lane] = acc; }
+  }
+  __syncthreads();
+  if (!valid) return;
+  const float4 t = *reinterpret_cast<const float4 *>((isz ? zt : St) + h * per + off);
+  const int32_t *ie = splan + splan_ie(d.F), *ib = splan + splan_ib(d.F, gcap);
+  for (int g = warp; g < G; g += SCAN_THREADS / 32) {
+    const float4 pf = pre[ie[g] * 32 + lane], sb = suf[ib[g] * 32 + lane];
+    const int64_t o = ((int64_t)g * d.H + h) * per + off;
+    if (SUM) {
+      const float4 v = f4add(t, f4add(pf, sb));
+      if (isz) {
+        *reinterpret_cast<float4 *>(zsum + o) = v;
+      } else {
+        uint2 u;
+        u.x = pack_bf16x2(v.x, v.y);
+        u.y = pack_bf16x2(v.z, v.w);
+        *reinterpret_cast<uint2 *>(ssum + o) = u;
+      }
+    } else {
+      const float4 ht = make_float4(0.5f * t.x, 0.5f * t.y, 0.5f * t.z, 0.5f * t.w);
+      *reinterpret_cast<float4 *>((isz ? zf : Sf) + o) = f4add(ht, pf);
+      *reinterpret_cast<float4 *>((isz ? zb : Sb) + o) = f4add(ht, sb);
+    }
+  }
+}
+
+template <bool SUM>
+cudaError_t launch_scan_seg(const Dims &d, const float *S, const float *z, const float *St, const float *zt,
+                            float *Sf, float *Sb, float *zf, float *zb, __nv_bfloat16 *ssum, float *zsum,
+                            char *ws, const WsPlan &p, int nseg, cudaStream_t st) {
+  const size_t smem = (size_t)(3 * nseg + 2) * 32 * sizeof(float4);
+  cudaError_t e = cudaFuncSetAttribute(scan_seg_kernel<SUM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t DD = (int64_t)d.D * d.D;
+  dim3 grid((unsigned)(DD / 128 + (d.D + 127) / 128), d.H);
+  scan_seg_kernel<SUM><<<grid, SCAN_THREADS, smem, st>>>(d, S, z, St, zt, Sf, Sb, zf, zb, ssum, zsum,
+                                                          (const int32_t *)(ws + p.splan), max_groups(d.F, d.C));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_scan_sum(const Dims &d, const float *S, const float *z, const float *St, const float *zt,
+                                  char *ws, const WsPlan &p, cudaStream_t st) {
+  const int nseg = host_scan_segments(d.F, d.T, d.C, d.L);
+  if (nseg > SCAN_SEG_MAX) return cudaErrorInvalidValue;
+  return launch_scan_seg<true>(d, S, z, St, zt, nullptr, nullptr, nullptr, nullptr,
+                               (__nv_bfloat16 *)(ws + p.ssum), (float *)(ws + p.zsum), ws, p, nseg, st);
+}
+
 cudaError_t launch_state_scan(const Dims &d, vdn_lin_kind kind, const float *S, const float *z, const float *St,
                               const float *zt, const float *beta, float *Sf, float *Sb, float *zf, float *zb,
                               char *ws, const WsPlan &p, cudaStream_t st) {
   const int32_t *gtab = (const int32_t *)(ws + p.gtab);
   const int G = host_group_count(d);
   if (kind == VDN_LIN_ELU1) {
+    const int nseg = host_scan_segments(d.F, d.T, d.C, d.L);
+    if (nseg <= SCAN_SEG_MAX)
+      return launch_scan_seg<false>(d, S, z, St, zt, Sf, Sb, zf, zb, nullptr, nullptr, ws, p, nseg, st);
     const int64_t n4 = ((int64_t)d.D * d.D + d.D) / 4;
     dim3 grid((unsigned)((n4 + 255) / 256), d.H, 2);
     scan_elu1_kernel<<<grid, 256, 0, st>>>(d, S, z, St, zt, Sf, Sb, zf, zb, gtab, G);

@@ -399,13 +399,17 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
     // writes A_l = g_l * gamma * RMSNorm(O_l), both straight into A
     VDN_TRY(state_build_dispatch(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, w, p,
                                  st));
+    const bool seg = layer_seg_scan(*shape, kind);
     {
       ProfScope ps(K_SCAN, st);
-      VDN_CUDA(launch_state_scan(d, kind, S, z, St, zt, beta, Sf, Sb, zf, zb, w, p, st), "scan launch");
+      if (seg)
+        VDN_CUDA(launch_state_scan_sum(d, S, z, St, zt, w, p, st), "scan launch");
+      else
+        VDN_CUDA(launch_state_scan(d, kind, S, z, St, zt, beta, Sf, Sb, zf, zb, w, p, st), "scan launch");
     }
-    {
+    if (!seg || (w_gate_l != nullptr && G_l == d.D)) {
       ProfScope ps(K_READ_STAGE, st);
-      VDN_CUDA(launch_read_stage(d, kind, Sf, Sb, zf, zb, w_gate_l, G_l, w, p, st), "read staging");
+      VDN_CUDA(launch_read_stage(d, kind, seg ? nullptr : Sf, Sb, zf, zb, w_gate_l, G_l, w, p, st), "read staging");
     }
     if (dtype == VDN_E4M3) {
       // per-head e4m3 Q/K/V for the softmax branch; the linear branch keeps the bf16 inputs
@@ -459,12 +463,13 @@ void *vdn_hybrid_attn_intermediate(const vdn_shape *shape, vdn_lin_kind kind, vd
     case 0: return fused ? nullptr : w + p.Os;
     case 1: return fused ? nullptr : w + p.Ol;
     case 2: return w + p.A;
-    case 3: return w + p.Sf;
-    case 4: return w + p.Sb;
+    case 3: return (fused && layer_seg_scan(*shape, kind)) ? nullptr : w + p.Sf;
+    case 4: return (fused && layer_seg_scan(*shape, kind)) ? nullptr : w + p.Sb;
     case 5: return w + p.ftab;
     case 6: return w + p.gtab;
     case 7: return w + p.tiles;
     case 8: return w + p.meta;
+    case 9: return w + p.splan;
     default: return nullptr;
   }
 }

@@ -126,9 +126,28 @@ VDN_HD int64_t max_tiles(int F, int T, int C) {
 constexpr size_t WS_ALIGN = 256;
 VDN_HD size_t align_up(size_t x) { return (x + WS_ALIGN - 1) / WS_ALIGN * WS_ALIGN; }
 
+// Scan plan (written by the tables kernel): the frames [1, F-1) that the two memories
+// can hold are cut at every memory boundary (the end e_g of a forward memory and the
+// start b_g of a backward one) into nseg segments; the forward memory of group g is the
+// sum of segments [0, ie[g]) and its backward memory that of segments [ib[g], nseg).
+// int32 layout: {nseg, G, 0, 0, bnd[F + 1], ie[gcap], ib[gcap]} with bnd[j] the first
+// frame of segment j and bnd[nseg] = F - 1.
+VDN_HD int64_t splan_ints(int F, int gcap) { return 4 + (int64_t)F + 1 + 2 * (int64_t)gcap; }
+VDN_HD int splan_ie(int F) { return 4 + F + 1; }
+VDN_HD int splan_ib(int F, int gcap) { return 4 + F + 1 + gcap; }
+// Segments one block of the segmented scan keeps in shared memory (three float4 rows of
+// 32 lanes per segment); layouts with more fall back to the per-frame walk.
+constexpr int SCAN_SEG_MAX = 96;
+
+// Memory boundaries of a group: forward memory [1, e), backward memory [b, F-1).
+VDN_HD void memory_bounds(const FrameSets &s, int F, int *e, int *b) {
+  *e = s.fwd[1] > s.fwd[0] ? s.fwd[1] : 1;
+  *b = s.bwd[1] > s.bwd[0] ? s.bwd[0] : F - 1;
+}
+
 struct WsPlan {
-  // step part (tables, tile list, status)
-  size_t status, ftab, gtab, meta, qamax, tiles, step_end;
+  // step part (tables, tile list, scan plan, tables scratch, status)
+  size_t status, ftab, gtab, meta, qamax, tiles, splan, tscr, step_end;
   // read staging: per-group summed memory in bf16 (tensor-core B operand), summed
   // normaliser, linear-gate weights in bf16
   size_t ssum, zsum, wl, stage_end;
@@ -140,6 +159,30 @@ struct WsPlan {
 // directly; O_s and O_l are never stored) for bf16 activations with D = 128.
 inline bool layer_fused(const vdn_shape &s, vdn_dtype dtype) {
   return (dtype == VDN_BF16 || dtype == VDN_E4M3) && s.head_dim == 128;
+}
+
+// Number of scan segments of a layout (the same rule the tables kernel applies).
+inline int host_scan_segments(int F, int T, int C, int L) {
+  if (F < 3) return 0;
+  int n = 0;
+  bool *mark = new bool[F + 1]();
+  mark[1] = mark[F - 1] = true;
+  FrameSets cur;
+  for (int f = 0; f < F; ++f) {
+    frame_sets(f, F, T, C, L, &cur);
+    int e, b;
+    memory_bounds(cur, F, &e, &b);
+    mark[e] = mark[b] = true;
+  }
+  for (int f = 1; f <= F - 1; ++f) n += mark[f] ? 1 : 0;
+  delete[] mark;
+  return n - 1;
+}
+
+// The ELU1 memories go through the segmented scan when the segments fit one block.
+inline bool layer_seg_scan(const vdn_shape &s, vdn_lin_kind kind) {
+  return kind == VDN_LIN_ELU1 &&
+         host_scan_segments(s.frames, s.tokens_per_frame, s.chunk_frames, s.text_tokens) <= SCAN_SEG_MAX;
 }
 
 // meta: int32[8] = {G, n_tiles, ...}
@@ -156,6 +199,8 @@ inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dt
   p.meta = take(64);
   p.qamax = take(3 * H * 4);
   p.tiles = take((size_t)max_tiles(s.frames, s.tokens_per_frame, s.chunk_frames) * TILE_REC * 4);
+  p.splan = take((size_t)splan_ints(s.frames, (int)G) * 4);
+  p.tscr = take((4 * G + 2 * (F + 1)) * 4);  // keys, order, count, first; mark, idx
   p.step_end = off;
   p.ssum = take(G * H * D * D * 2);
   p.zsum = take(G * H * D * 4);
@@ -167,11 +212,13 @@ inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dt
   p.z = take(F * H * D * 4);
   p.St = take(H * D * D * 4);
   p.zt = take(H * D * 4);
-  p.Sf = take(G * H * D * D * 4);
-  p.Sb = take(G * H * D * D * 4);
-  p.zf = take(G * H * D * 4);
-  p.zb = take(G * H * D * 4);
+  // the segmented scan of the fused layer writes the bf16 sum S_fwd + S_bwd directly
   const bool fused = layer_fused(s, dtype);
+  const size_t Gm = (fused && layer_seg_scan(s, kind)) ? 0 : G;
+  p.Sf = take(Gm * H * D * D * 4);
+  p.Sb = take(Gm * H * D * D * 4);
+  p.zf = take(Gm * H * D * 4);
+  p.zb = take(Gm * H * D * 4);
   p.Os = take(fused ? 0 : Nv * H * D * act);
   p.Ol = take(fused ? 0 : Nv * H * D * act);
   p.A = take(Nv * 2 * H * D * act);
@@ -278,6 +325,10 @@ cudaError_t launch_state_build(const Dims &d, vdn_lin_kind kind, vdn_dtype dt, c
 cudaError_t launch_state_scan(const Dims &d, vdn_lin_kind kind, const float *S, const float *z, const float *St,
                               const float *zt, const float *beta, float *Sf, float *Sb, float *zf, float *zb,
                               char *ws, const WsPlan &p, cudaStream_t st);
+// ELU1 memories of the fused layer: S_fwd + S_bwd in bf16 and z_fwd + z_bwd straight
+// into the read staging buffers (segmented scan; needs at most SCAN_SEG_MAX segments)
+cudaError_t launch_state_scan_sum(const Dims &d, const float *S, const float *z, const float *St, const float *zt,
+                                  char *ws, const WsPlan &p, cudaStream_t st);
 cudaError_t launch_linear_read(const Dims &d, vdn_lin_kind kind, vdn_dtype dt, const void *q, const float *Sf,
                                const float *Sb, const float *zf, const float *zb, void *o, char *ws,
                                const WsPlan &p, cudaStream_t st);
@@ -286,7 +337,8 @@ bool linear_tc_supported(const Dims &d, vdn_dtype dt);
 cudaError_t launch_state_build_tc(const Dims &d, const void *k, const void *v, const void *kt, const void *vt,
                                   float *S, float *z, float *St, float *zt, char *ws, const WsPlan &p,
                                   cudaStream_t st);
-// sums the two memories of every group into the bf16 staging buffers (and the gate weights to bf16)
+// sums the two memories of every group into the bf16 staging buffers (skipped when Sf is
+// NULL: the segmented scan wrote them) and converts the gate weights to bf16
 cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf, const float *Sb, const float *zf,
                               const float *zb, const float *wgl, int G_l, char *ws, const WsPlan &p,
                               cudaStream_t st);

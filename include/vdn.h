@@ -241,10 +241,15 @@ VDN_API vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind
 
 /* Device pointers (inside ws) of the layer's intermediates after vdn_hybrid_attn_fwd:
  * which = 0: O_s [N_v][H][D] (bf16, or float for VDN_F32); 1: O_l (same type);
- * 2: A [N_v][2HD]; 3: per-group S_fwd; 4: S_bwd; 5: frame table int32[F][8];
+ * 2: A [N_v][2HD]; 3: per-group S_fwd; 4: S_bwd (both NULL on the fused ELU1 path,
+ * whose scan stores only the bf16 sum S_fwd + S_bwd); 5: frame table int32[F][8];
  * 6: group table int32[G][16]; 7: query-tile list int32[n][8] (group, row_lo, row_hi,
  * keys, first tile of the group, tiles of the group, 0, 0) of 256-row tiles, groups with
- * the longest key set first; 8: meta int32[2] (G, n).  Entries 5-8 are also
+ * the longest key set first; 8: meta int32[2] (G, n); 9: scan plan int32
+ * {nseg, G, 0, 0, bnd[F + 1], ie[max_groups], ib[max_groups]}: the frames [1, F-1) cut
+ * at every memory boundary into nseg segments starting at bnd[j] (bnd[nseg] = F - 1);
+ * group g's forward memory sums segments [0, ie[g]), its backward memory segments
+ * [ib[g], nseg).  Entries 5-9 are also
  * written by the step entry points that take a workspace.  NULL if not materialised.
  * Valid until the next call that uses ws. */
 VDN_API void *vdn_hybrid_attn_intermediate(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, void *ws,

@@ -47,6 +47,29 @@ def _check_tables(run: Run):
         covered[lo:hi] += 1
     assert (covered == 1).all()
     assert all(tiles[i][3] >= tiles[i + 1][3] for i in range(n - 1)), "tiles not longest-first"
+    _check_scan_plan(run, gtab)
+
+
+def _check_scan_plan(run: Run, gtab):
+    """Segments of the frames [1, F-1) cut at every memory boundary; each group's
+    forward memory [1, e) and backward memory [b, F-1) are unions of whole segments."""
+    s = run.shape
+    F, G = s.frames, len(gtab)
+    gcap = vdn.max_groups(s)
+    plan = run.intermediate(9, (4 + F + 1 + 2 * gcap,), torch.int32).cpu().numpy()
+    nseg = int(plan[0])
+    assert int(plan[1]) == G
+    ends = [int(r[13]) if r[13] > r[12] else 1 for r in gtab]
+    starts = [int(r[14]) if r[15] > r[14] else F - 1 for r in gtab]
+    if F < 3:
+        assert nseg == 0
+        return
+    bnd = sorted(set([1, F - 1] + ends + starts))
+    assert nseg == len(bnd) - 1
+    np.testing.assert_array_equal(plan[4:4 + nseg + 1], bnd)
+    ie, ib = plan[4 + F + 1:4 + F + 1 + G], plan[4 + F + 1 + gcap:4 + F + 1 + gcap + G]
+    for g in range(G):
+        assert bnd[ie[g]] == ends[g] and bnd[ib[g]] == starts[g]
 
 
 def _layer_parity(run: Run, rows, kind_tol, check_states=True):
@@ -85,7 +108,9 @@ def _layer_parity(run: Run, rows, kind_tol, check_states=True):
     ref_a = vo.hybrid_fuse(o["q"][rows], ref_os, ref_ol, o["w_gate_s"], o["w_gate_l"], o["gamma"], 1e-6)
     assert_close("A (layer)", A, ref_a, kind_tol)
     assert_close("y (layer)", yr, vo.out_proj(ref_a, o["w_os"], o["w_ol"]), kind_tol)
-    if check_states and run.kind == vdn.ELU1:
+    # the fused ELU1 layer keeps only S_fwd + S_bwd (bf16); A_l above checks it
+    stored = vdn.hybrid_attn_intermediate(s, run.kind, run.cdt, run.ws, 3) != 0
+    if check_states and run.kind == vdn.ELU1 and stored:
         _, gtab = vdn.mask_layout_build(s)
         G = len(gtab)
         num_f, num_b, den_f, den_b = vo.linear_memory(o["k"], o["v"], o["kt"], o["vt"], F, T, C)
@@ -215,6 +240,36 @@ def test_step_entry_points_match_oracle(shape):
     vdn.out_proj(s, vdn.BF16, a, d["w_os"], d["w_ol"], y, ws)
     assert_close("out_proj", to_numpy(y), vo.out_proj(to_numpy(a), o["w_os"], o["w_ol"]), "bf16")
     vdn.check_device_status(ws)
+
+
+@pytest.mark.parametrize("shape", [(130, 4, 1, 3, 1, 32),    # 127 segments: the per-frame walk
+                                   (87, 6, 5, 2, 2, 64),     # ragged last chunk
+                                   (3, 5, 1, 0, 1, 32),      # a single segment, no text
+                                   (2, 5, 5, 4, 1, 32)])     # no frame outside the anchors
+def test_state_scan_layouts(shape):
+    s = synth.Shape(*shape)
+    F, T, C, L, H, D = shape
+    inp = synth.make_inputs(s, "f32", seed=77 + F)
+    o = oracle_inputs(inp)
+    d = {n: to_device(a) for n, a in inp.items()}
+    ws = workspace(vdn.step_workspace_size(s))
+    vdn.workspace_init(ws)
+    S = torch.empty((F, H, D, D), dtype=torch.float32, device="cuda")
+    z = torch.empty((F, H, D), dtype=torch.float32, device="cuda")
+    St = torch.empty((H, D, D), dtype=torch.float32, device="cuda")
+    zt = torch.empty((H, D), dtype=torch.float32, device="cuda")
+    vdn.linear_state_build(s, vdn.ELU1, vdn.F32, d["k"], d["v"], d["kt"], d["vt"], S, z, St, zt, ws)
+    G = vdn.max_groups(s)
+    Sf, Sb = (torch.full((G, H, D, D), float("nan"), device="cuda") for _ in range(2))
+    zf, zb = (torch.full((G, H, D), float("nan"), device="cuda") for _ in range(2))
+    vdn.linear_state_scan(s, vdn.ELU1, S, z, St, zt, None, Sf, Sb, zf, zb, ws)
+    vdn.check_device_status(ws)
+    _, gtab = vdn.mask_layout_build(s)
+    first = [int(r[0]) for r in gtab]
+    nf, nb, df, db = vo.linear_memory(o["k"], o["v"], o["kt"], o["vt"], F, T, C)
+    ng = len(gtab)
+    for got, ref in ((Sf, nf), (Sb, nb), (zf, df), (zb, db)):
+        assert rel_l2(got[:ng].cpu().numpy(), ref[first]) < 1e-5
 
 
 # ----------------------------------------------------------------------------- bounded device wait
