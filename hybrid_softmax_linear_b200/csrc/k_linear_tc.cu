@@ -4,7 +4,7 @@
 // linear output is RMS-normalised and gated element-wise.)
 //
 // state_build_tc: S_f = phi(K_f)^T V_f and z_f = sum phi(K_f) for one (frame or text,
-//   head) per CTA.  TMA streams 64-token K/V tiles into a 3-stage ring; four warps apply
+//   head) per CTA.  TMA streams 64-token K/V tiles into a 3-stage ring; eight warps apply
 //   phi = elu+1 in place in shared memory (masking tokens past the frame) and sum z;
 //   one thread issues tcgen05.mma with both operands MN-major (M = key feature, N =
 //   value dim, K = tokens) into a 128x128 fp32 accumulator in tensor memory.
@@ -49,7 +49,7 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
 
 // ============================================================================ state build
 namespace sb {
-constexpr int D = 128, TK = 64, NS = 3, THREADS = 192;
+constexpr int D = 128, TK = 64, NS = 3, THREADS = 320, PHI_WARPS = 8;
 constexpr int BOX_BYTES = TK * 128;        // 64 tokens x 64 bf16
 constexpr int TILE_BYTES = 2 * BOX_BYTES;  // 64 tokens x 128 features
 constexpr int STAGE_BYTES = 2 * TILE_BYTES;
@@ -79,16 +79,18 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
   __syncthreads();
   if (skip) return;
 
-  const int h = blockIdx.y;
-  const bool text = (int)blockIdx.x == d.F;
+  // heads vary fastest across the grid, so the CTAs in flight read whole token rows of K and V
+  const int h = (int)(blockIdx.x % (unsigned)d.H);
+  const int fr = (int)(blockIdx.x / (unsigned)d.H);
+  const bool text = fr == d.F;
   const int ntok = text ? d.L : d.T;
-  const int row_base = text ? 0 : (int)blockIdx.x * d.T;
+  const int row_base = text ? 0 : fr * d.T;
   const int nch = (ntok + TK - 1) / TK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(smem_u32(&bars->full[s]), 1);
-      mbar_init(smem_u32(&bars->phi[s]), 4);
+      mbar_init(smem_u32(&bars->phi[s]), PHI_WARPS);
       mbar_init(smem_u32(&bars->empty[s]), 1);
     }
     mbar_init(smem_u32(&bars->acc), 1);
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
   } else {
     // ---------------- phi pass (in place, masked) and z; then the epilogue
     const int tid = threadIdx.x - 64;
-    const int cl = tid & 15, rg = tid >> 4;  // column chunk 8cl..8cl+7; rows rg + 8i
+    const int cl = tid & 15, rg = tid >> 4;  // column chunk 8cl..8cl+7; rows rg + 16i
     float zacc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
@@ -157,15 +159,16 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       uint8_t *kt = base + s * STAGE_BYTES;
 #pragma unroll
-      for (int i = 0; i < TK / 8; ++i) {
-        const int r = rg + 8 * i;
+      for (int i = 0; i < TK / 16; ++i) {
+        const int r = rg + 16 * i;
         uint4 *p = reinterpret_cast<uint4 *>(kt + swz_off(r, cl, TK));
         float f[8];
         unpack8(*p, f);
         const bool valid = c * TK + r < ntok;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float ph = valid ? (f[e] > 0.f ? f[e] + 1.f : expf(f[e])) : 0.f;
+          // phi enters the MMA in bf16, so the fast exponential is accurate enough
+          const float ph = valid ? (f[e] > 0.f ? f[e] + 1.f : __expf(f[e])) : 0.f;
           zacc[e] += ph;
           f[e] = ph;
         }
@@ -177,31 +180,34 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) atomicAdd(&bars->zred[cl * 8 + e], zacc[e]);
-    const int quad = warp & 3;
+    const int quad = warp & 3, c_lo = ((warp - 2) >> 2) * (D / 2);  // lane quarter; column half
     const int i = quad * 32 + lane;  // key feature = accumulator row = tensor-memory lane
-    float *So = text ? St + (int64_t)h * D * D : S + ((int64_t)blockIdx.x * d.H + h) * D * D;
+    float *So = text ? St + (int64_t)h * D * D : S + ((int64_t)fr * d.H + h) * D * D;
     if (nch > 0) {
       const bool done = ok && mbar_wait(smem_u32(&bars->acc), 0, abort_flag, st, K_STATE, 6);
       if (__all_sync(0xffffffffu, done)) {
         tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < D; cc += 32) {
-          uint32_t u[32];
-          tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + cc, u);
-          tmem_wait_ld();
-          float4 *dst = reinterpret_cast<float4 *>(So + i * D + cc);
+        uint32_t u0[32], u1[32];
+        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c_lo, u0);
+        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c_lo + 32, u1);
+        tmem_wait_ld();
+        float4 *dst = reinterpret_cast<float4 *>(So + i * D + c_lo);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(__uint_as_float(u[4 * v]), __uint_as_float(u[4 * v + 1]),
-                                 __uint_as_float(u[4 * v + 2]), __uint_as_float(u[4 * v + 3]));
-        }
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_float4(__uint_as_float(u0[4 * v]), __uint_as_float(u0[4 * v + 1]),
+                               __uint_as_float(u0[4 * v + 2]), __uint_as_float(u0[4 * v + 3]));
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[8 + v] = make_float4(__uint_as_float(u1[4 * v]), __uint_as_float(u1[4 * v + 1]),
+                                   __uint_as_float(u1[4 * v + 2]), __uint_as_float(u1[4 * v + 3]));
       }
     } else {
-      for (int cc = 0; cc < D; ++cc) So[i * D + cc] = 0.f;
+      for (int cc = 0; cc < D / 2; ++cc) So[i * D + c_lo + cc] = 0.f;
     }
-    named_bar_sync(1, 128);  // every phi thread has added its share of z
+    named_bar_sync(1, 32 * PHI_WARPS);  // every phi thread has added its share of z
     float *zo = text ? zt : z;
-    if (zo != nullptr) zo[(text ? (int64_t)h * D : ((int64_t)blockIdx.x * d.H + h) * D) + tid] = bars->zred[tid];
+    if (zo != nullptr && tid < D)
+      zo[(text ? (int64_t)h * D : ((int64_t)fr * d.H + h) * D) + tid] = bars->zred[tid];
   }
   tc_fence_before();
   __syncthreads();
@@ -277,10 +283,12 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
   __syncthreads();
   if (skip) return;
 
-  const int h = blockIdx.y;
-  const int32_t *tr = tiles + (int64_t)(blockIdx.x >> 1) * TILE_REC;
+  // heads vary fastest across the grid: the CTAs in flight read and write whole rows
+  const int h = (int)(blockIdx.x % (unsigned)d.H);
+  const unsigned half_tile = blockIdx.x / (unsigned)d.H;
+  const int32_t *tr = tiles + (int64_t)(half_tile >> 1) * TILE_REC;
   const int g = tr[0];
-  const int row0 = tr[1] + (blockIdx.x & 1) * BM, row_end = tr[2];
+  const int row0 = tr[1] + (int)(half_tile & 1) * BM, row_end = tr[2];
   if (row0 >= row_end) return;  // the second half of a short tile (block-uniform)
 
   if (threadIdx.x == 0) {
@@ -473,7 +481,7 @@ cudaError_t launch_state_build_tc(const Dims &d, const void *k, const void *v, c
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(state_build_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
   if (e != cudaSuccess) return e;
-  state_build_tc_kernel<<<dim3(d.F + 1, d.H), THREADS, SMEM, st>>>(mk, mv, mkt, mvt, d, S, z, St, zt,
+  state_build_tc_kernel<<<(unsigned)((d.F + 1) * d.H), THREADS, SMEM, st>>>(mk, mv, mkt, mvt, d, S, z, St, zt,
                                                                    (DevStatus *)(ws + p.status));
   return cudaGetLastError();
 }
@@ -522,7 +530,7 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
   if (e != cudaSuccess) return e;
   const int64_t stride = fused ? 2 * (int64_t)HD : (int64_t)HD;
   __nv_bfloat16 *o = (__nv_bfloat16 *)out + (fused ? HD : 0);  // fused: the linear half of A
-  read_tc_kernel<<<dim3(2 * host_tile_count(d), d.H), THREADS, SMEM, st>>>(
+  read_tc_kernel<<<(unsigned)(2 * host_tile_count(d) * d.H), THREADS, SMEM, st>>>(
       mq, ms, mw, d, kind == VDN_LIN_DELTA, gate_mma ? 1 : 0, (const float *)(ws + p.zsum),
       fused ? wgl : nullptr, G_l, gamma, eps, o, stride, fused ? 1 : 0, (const int32_t *)(ws + p.tiles),
       (DevStatus *)(ws + p.status));
