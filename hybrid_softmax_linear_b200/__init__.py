@@ -18,7 +18,7 @@ __all__ = [
     "VdnError", "Shape", "lib", "F32", "BF16", "E4M3", "ELU1", "DELTA",
     "mask_layout_build", "max_groups", "hybrid_attn_workspace_size", "step_workspace_size", "workspace_init",
     "softmax_branch_fwd", "linear_state_build", "linear_state_scan", "linear_read", "hybrid_fuse", "out_proj",
-    "hybrid_attn_fwd", "hybrid_attn_intermediate", "check_device_status", "debug_unset_flag_wait", "version",
+    "hybrid_attn_fwd", "hybrid_attn_host_workspace_size", "hybrid_attn_fwd_host", "hybrid_attn_intermediate", "check_device_status", "debug_unset_flag_wait", "version",
     "profile_begin", "profile_end", "fp8_quant_per_head", "softmax_branch_fwd_noalloc",
 ]
 
@@ -70,6 +70,9 @@ _SIGS = {
     "vdn_out_proj": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "vdn_hybrid_attn_fwd": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                            _i32, _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "vdn_hybrid_attn_host_workspace_size": (_sz, [_SP, ctypes.c_int, ctypes.c_int]),
+    "vdn_hybrid_attn_fwd_host": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                _vp, _i32, _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "vdn_hybrid_attn_intermediate": (_vp, [_SP, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int]),
     "vdn_check_device_status": (ctypes.c_int, [_vp, _sz, _vp]),
     "vdn_debug_unset_flag_wait": (ctypes.c_int, [_vp, _sz, _u32, _vp]),
@@ -211,6 +214,19 @@ def hybrid_attn_fwd(shape, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_
     _check(lib().vdn_hybrid_attn_fwd(ctypes.byref(Shape.of(shape)), kind, dtype, _p(q), _p(k), _p(v), _p(kt),
                                      _p(vt), _p(beta), _p(w_gate_s), _p(w_gate_l), G_l, _p(gamma), eps, _p(w_os),
                                      _p(w_ol), _p(y), _p(ws), _nbytes(ws), _stream(stream)))
+
+
+def hybrid_attn_host_workspace_size(shape, kind: int, dtype: int) -> int:
+    return lib().vdn_hybrid_attn_host_workspace_size(ctypes.byref(Shape.of(shape)), kind, dtype)
+
+
+def hybrid_attn_fwd_host(shape, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma, eps, w_os,
+                         w_ol, y, ws, stream=None):
+    """The layer with q, k, v, kt, vt, beta and y in (page-locked) host memory; weights on
+    the device.  Asynchronous on `stream`: y is complete when the stream is."""
+    _check(lib().vdn_hybrid_attn_fwd_host(ctypes.byref(Shape.of(shape)), kind, dtype, _p(q), _p(k), _p(v), _p(kt),
+                                          _p(vt), _p(beta), _p(w_gate_s), _p(w_gate_l), G_l, _p(gamma), eps,
+                                          _p(w_os), _p(w_ol), _p(y), _p(ws), _nbytes(ws), _stream(stream)))
 
 
 def hybrid_attn_intermediate(shape, kind, dtype, ws, which: int) -> int:

@@ -264,7 +264,9 @@ struct alignas(8) Bars {
 constexpr size_t SMEM = 1024 + BAR_OFF + sizeof(Bars);
 }  // namespace rd
 
-__device__ __forceinline__ float fast_sigmoid(float x) { return __frcp_rn(1.f + __expf(-x)); }
+// 1 / (1 + 2^(-x log2 e)) with the hardware exp2 and reciprocal approximations (relative
+// error near 2^-21); the result goes to bf16
+__device__ __forceinline__ float fast_sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
 __global__ void __launch_bounds__(rd::THREADS, 2)
     read_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
@@ -357,6 +359,7 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
       // feature row in registers (bf16 pairs): phi(q), or q/|q| for the delta rule
       uint32_t fr[D / 2];
       float inv_norm = 1.f;
+      const bool scalar_gate = fused && !gate_mma;
       if (delta) {
         float ss = 0.f;
 #pragma unroll
@@ -373,7 +376,8 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
         float f[8];
         unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) gate1 = fmaf(f[e], bars->wg1[cl * 8 + e], gate1);
+        for (int e = 0; e < 8; ++e)
+          if (scalar_gate) gate1 = fmaf(f[e], bars->wg1[cl * 8 + e], gate1);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           if (delta) {

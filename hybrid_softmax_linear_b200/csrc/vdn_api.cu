@@ -454,6 +454,75 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
   return ok();
 }
 
+namespace {
+// Staging area of the host entry point, after the layer's workspace.
+struct HostStage {
+  size_t q, k, v, kt, vt, beta, y, total;
+};
+HostStage plan_host_stage(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dtype) {
+  HostStage h{};
+  const size_t act = dtype == VDN_F32 ? 4 : 2;
+  const size_t nv = (size_t)s.frames * s.tokens_per_frame, hd = (size_t)s.heads * s.head_dim;
+  size_t off = plan_workspace(s, kind, dtype).total;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+  h.q = take(nv * hd * act);
+  h.k = take(nv * hd * act);
+  h.v = take(nv * hd * act);
+  h.kt = take((size_t)s.text_tokens * hd * act);
+  h.vt = take((size_t)s.text_tokens * hd * act);
+  h.beta = take(kind == VDN_LIN_DELTA ? (size_t)s.frames * s.heads * 4 : 0);
+  h.y = take(nv * hd * act);
+  h.total = off;
+  return h;
+}
+}  // namespace
+
+size_t vdn_hybrid_attn_host_workspace_size(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype) {
+  if (check_shape(shape) != VDN_OK || check_kind(kind) != VDN_OK) return 0;
+  return plan_host_stage(*shape, kind, dtype).total;
+}
+
+vdn_status vdn_hybrid_attn_fwd_host(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *q_host,
+                                    const void *k_host, const void *v_host, const void *kt_host,
+                                    const void *vt_host, const float *beta_host, const float *w_gate_s,
+                                    const float *w_gate_l, int32_t G_l, const float *gamma, float eps,
+                                    const void *w_os, const void *w_ol, void *y_host, void *ws, size_t ws_bytes,
+                                    vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  VDN_TRY(check_kind(kind));
+  if (dtype != VDN_F32 && dtype != VDN_BF16 && dtype != VDN_E4M3)
+    return fail(VDN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  const bool text = shape->text_tokens > 0;
+  if (q_host == nullptr || k_host == nullptr || v_host == nullptr || y_host == nullptr ||
+      (text && (kt_host == nullptr || vt_host == nullptr)))
+    return fail(VDN_ERR_INVALID_ARG, "a host tensor pointer is NULL");
+  if (kind == VDN_LIN_DELTA && beta_host == nullptr) return fail(VDN_ERR_INVALID_ARG, "beta is NULL");
+  const HostStage h = plan_host_stage(*shape, kind, dtype);
+  VDN_TRY(check_ws(ws, ws_bytes, h.total));
+  VDN_TRY(check_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  char *w = (char *)ws;
+  const size_t act = dtype == VDN_F32 ? 4 : 2;
+  const size_t nv = (size_t)shape->frames * shape->tokens_per_frame, hd = (size_t)shape->heads * shape->head_dim;
+  const size_t big = nv * hd * act, small = (size_t)shape->text_tokens * hd * act;
+  VDN_CUDA(cudaMemcpyAsync(w + h.q, q_host, big, cudaMemcpyHostToDevice, st), "copy of q to the device");
+  VDN_CUDA(cudaMemcpyAsync(w + h.k, k_host, big, cudaMemcpyHostToDevice, st), "copy of k to the device");
+  VDN_CUDA(cudaMemcpyAsync(w + h.v, v_host, big, cudaMemcpyHostToDevice, st), "copy of v to the device");
+  if (text) {
+    VDN_CUDA(cudaMemcpyAsync(w + h.kt, kt_host, small, cudaMemcpyHostToDevice, st), "copy of kt to the device");
+    VDN_CUDA(cudaMemcpyAsync(w + h.vt, vt_host, small, cudaMemcpyHostToDevice, st), "copy of vt to the device");
+  }
+  if (kind == VDN_LIN_DELTA)
+    VDN_CUDA(cudaMemcpyAsync(w + h.beta, beta_host, (size_t)shape->frames * shape->heads * 4,
+                             cudaMemcpyHostToDevice, st),
+             "copy of beta to the device");
+  VDN_TRY(vdn_hybrid_attn_fwd(shape, kind, dtype, w + h.q, w + h.k, w + h.v, text ? w + h.kt : nullptr,
+                              text ? w + h.vt : nullptr, kind == VDN_LIN_DELTA ? (const float *)(w + h.beta) : nullptr,
+                              w_gate_s, w_gate_l, G_l, gamma, eps, w_os, w_ol, w + h.y, ws, ws_bytes, stream));
+  VDN_CUDA(cudaMemcpyAsync(y_host, w + h.y, big, cudaMemcpyDeviceToHost, st), "copy of y to the host");
+  return ok();
+}
+
 void *vdn_hybrid_attn_intermediate(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, void *ws, int which) {
   if (check_shape(shape) != VDN_OK || ws == nullptr) return nullptr;
   const WsPlan p = plan_workspace(*shape, kind, dtype);

@@ -239,6 +239,24 @@ VDN_API vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind
                                float eps, const void *w_os, const void *w_ol, void *y, void *ws,
                                size_t ws_bytes, vdn_stream stream);
 
+/* vdn_hybrid_attn_fwd_host — the layer with its per-call tensors in HOST memory.  No
+ * counterpart in the pages: it is the streaming form of vdn_hybrid_attn_fwd.
+ *   q, k, v, kt, vt (and beta for DELTA) are read from host memory and y is written to
+ *   host memory; weights (w_gate_s, w_gate_l, gamma, w_os, w_ol) stay device pointers.
+ *   Everything is enqueued on `stream`: one cudaMemcpyAsync per input into the staging
+ *   area at the end of ws, the layer, and one copy of y back.  y_host is complete when
+ *   the stream is.  Host buffers should be page-locked, or the copies do not overlap
+ *   other work.  Calls on two streams with two workspaces overlap the copies of one
+ *   call with the kernels of the other.
+ * ws: vdn_hybrid_attn_host_workspace_size(shape, kind, dtype) bytes. */
+VDN_API size_t vdn_hybrid_attn_host_workspace_size(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype);
+VDN_API vdn_status vdn_hybrid_attn_fwd_host(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype,
+                                            const void *q_host, const void *k_host, const void *v_host,
+                                            const void *kt_host, const void *vt_host, const float *beta_host,
+                                            const float *w_gate_s, const float *w_gate_l, int32_t G_l,
+                                            const float *gamma, float eps, const void *w_os, const void *w_ol,
+                                            void *y_host, void *ws, size_t ws_bytes, vdn_stream stream);
+
 /* Device pointers (inside ws) of the layer's intermediates after vdn_hybrid_attn_fwd:
  * which = 0: O_s [N_v][H][D] (bf16, or float for VDN_F32); 1: O_l (same type);
  * 2: A [N_v][2HD]; 3: per-group S_fwd; 4: S_bwd (both NULL on the fused ELU1 path,

@@ -286,3 +286,32 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     run = Run(w.shape, cfg_inputs(1), w.dtype)
     y = run.layer()
     assert torch.isfinite(y).all()
+
+
+# ----------------------------------------------------------------------------- host-buffer entry point
+@pytest.mark.parametrize("kind_dtype", [(vdn.ELU1, vdn.BF16), (vdn.DELTA, vdn.E4M3)])
+def test_host_entry_point_matches_device_entry_point(kind_dtype):
+    kind, cdt = kind_dtype
+    s = synth.Shape(12, 300, 5, 40, 2, 128)
+    inp = synth.make_inputs(s, "bf16", seed=99, with_beta=kind == vdn.DELTA)
+    run = Run(s, inp, "bf16", kind=kind, layer_dtype=cdt)
+    y_dev = to_numpy(run.layer())
+    names = ["q", "k", "v", "kt", "vt"] + (["beta"] if kind == vdn.DELTA else [])
+    host = {n: torch.from_numpy(inp[n].view(np.int16) if inp[n].dtype == np.uint16 else inp[n]).pin_memory()
+            for n in names}
+    y_host = torch.empty((s.n_video, s.hidden), dtype=torch.int16).pin_memory()
+    ws = workspace(vdn.hybrid_attn_host_workspace_size(s, kind, cdt))
+    assert ws.numel() > vdn.hybrid_attn_workspace_size(s, kind, cdt)
+    vdn.workspace_init(ws)
+    stream = torch.cuda.Stream()
+    d = run.dev
+    vdn.hybrid_attn_fwd_host(s, kind, cdt, host["q"], host["k"], host["v"], host["kt"], host["vt"], host.get("beta"),
+                             d["w_gate_s"], d["w_gate_l"], run.G_l, d["gamma"], 1e-6, d["w_os"], d["w_ol"], y_host, ws,
+                             stream)
+    stream.synchronize()
+    vdn.check_device_status(ws)
+    got = synth.bf16_bits_to_f32(y_host.numpy().view(np.uint16))
+    assert rel_l2(got, y_dev) < 1e-3
+    ref = vo.layer(oracle_inputs(inp), s.frames, s.tokens_per_frame, s.chunk_frames, rows=np.arange(s.n_video),
+                   linear="delta" if kind == vdn.DELTA else "elu1")
+    assert rel_l2(got, ref["y"]) <= (3e-2 if cdt == vdn.E4M3 else 5e-3)
