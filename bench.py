@@ -184,11 +184,102 @@ def oracle_sample(cfg: int, inp: dict, n_rows: int, seed: int = 11) -> dict:
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:  # pragma: no cover
         cores = len(os.sched_getaffinity(0))
-    return {"value": s.n_video / t_full, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+    cpu_model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            cpu_model = next((ln.split(":", 1)[1].strip() for ln in f if ln.startswith("model name")), None)
+    except OSError:
+        pass
+    return {"value": s.n_video / t_full, "unit": UNIT, "cores": int(cores), "kind": "oracle", "cpu_model": cpu_model,
             "sample": f"all per-frame linear states + {n_rows} random query rows x {s.heads} heads "
                       f"(softmax, linear read, fuse, projections); extrapolated as "
                       f"t_states + t_rows*N_v/{n_rows}",
             "t_states_s": round(t1 - t0, 3), "t_rows_s": round(t2 - t1, 3)}
+
+
+def dense_reference(s, dev, iters: int = 2) -> dict:
+    """The dense full-attention layer on the same shapes, through library kernels: torch SDPA
+    with the cuDNN backend (Q [1,H,N_v,D], K/V [1,H,N_v+L,D], no mask, bf16), plus one bf16
+    matmul for the two output projections (K = 2HD).  A comparator, not part of the product."""
+    import torch
+    import torch.nn.functional as Fn
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    H, D, Nv, L = s.heads, s.head_dim, s.n_video, s.text_tokens
+    g = torch.Generator(device=dev).manual_seed(7)
+    q = torch.randn((1, H, Nv, D), device=dev, dtype=torch.bfloat16, generator=g)
+    k = torch.randn((1, H, Nv + L, D), device=dev, dtype=torch.bfloat16, generator=g)
+    v = torch.randn((1, H, Nv + L, D), device=dev, dtype=torch.bfloat16, generator=g)
+    a = torch.randn((Nv, 2 * H * D), device=dev, dtype=torch.bfloat16, generator=g)
+    w = torch.randn((H * D, 2 * H * D), device=dev, dtype=torch.bfloat16, generator=g) * 0.02
+    out = {}
+    backend = None
+    for name, be in (("cudnn", SDPBackend.CUDNN_ATTENTION), ("flash", SDPBackend.FLASH_ATTENTION),
+                     ("efficient", SDPBackend.EFFICIENT_ATTENTION)):
+        try:
+            with sdpa_kernel(be):
+                Fn.scaled_dot_product_attention(q, k, v)
+            torch.cuda.synchronize(dev)
+            backend = (name, be)
+            break
+        except RuntimeError:
+            continue
+    if backend is None:
+        return {"unavailable": "no SDPA backend ran on these shapes"}
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / iters
+
+    with sdpa_kernel(backend[1]):
+        sdpa_ms = timed(lambda: Fn.scaled_dot_product_attention(q, k, v))
+    proj_ms = timed(lambda: torch.matmul(a, w.t()))
+    attn_flop = 4.0 * D * H * Nv * (Nv + L)
+    proj_flop = 2.0 * Nv * (2 * H * D) * (H * D)
+    out.update({"backend": backend[0], "sdpa_ms": sdpa_ms, "proj_ms": proj_ms, "layer_ms": sdpa_ms + proj_ms,
+                "sdpa_tflops": attn_flop / (sdpa_ms / 1e3) / 1e12, "iters": iters,
+                "shapes": f"Q [1,{H},{Nv},{D}], K/V [1,{H},{Nv + L},{D}] bf16, no mask; projections "
+                          f"[{Nv},{2 * H * D}] x [{2 * H * D},{H * D}]"})
+    del q, k, v, a, w
+    torch.cuda.empty_cache()
+    return out
+
+
+def fp8_peak(dev) -> float | None:
+    """Dense e4m3 GEMM throughput (torch._scaled_mm, 8192^3, best of 10), TFLOP/s."""
+    import torch
+    try:
+        n = 8192
+        a = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev)
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize(dev)
+        best = None
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        return 2.0 * n ** 3 / (best / 1e3) / 1e12
+    except Exception:
+        return None
+
+
+# The pages' whole-model figures (single B200, 50 steps): dense MiniMax-H3 with cuDNN attention
+# 16.74 s per function evaluation, VDN-H3 with fp8 6.41 s ("VDN-MiniMax-H3 开源" article,
+# performance table).  Context only: a different workload from one layer.
+PAGES_CONTEXT = {"dense_minimax_h3_cudnn_s_per_nfe": 16.74, "vdn_h3_fp8_s_per_nfe": 6.41,
+                 "note": "whole model, 50 steps, single B200, as printed by the pages; context only"}
 
 
 def run_reference(args, rank, world):
@@ -349,10 +440,15 @@ def run_ours(args, rank, world, local_rank):
     achieved = fl["softmax"] / (sm_avg / 1e3) / 1e12 if sm_avg > 0 else None
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_note = f"{peak_src} bf16_tflops_sustained (kernel runs inside a long step)"
+    fp8_burst = fp8_peak(dev) if w.softmax_fp8 else None
     if w.softmax_fp8:
-        # e4m3 contraction: the measured bf16 peak times the nominal fp8/bf16 ratio (4.5 / 2.25)
-        peak *= 2.0
-        peak_note = f"{peak_src} bf16_tflops_sustained x 2 (nominal fp8/bf16 ratio; kernel runs inside a long step)"
+        # e4m3 contraction: the measured bf16 sustained peak times the measured fp8/bf16 burst
+        # ratio (nominal 2 when the e4m3 GEMM could not be timed)
+        ratio = (fp8_burst / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) if fp8_burst else 2.0
+        peak *= ratio
+        peak_note = (f"{peak_src} bf16_tflops_sustained x {ratio:.3f} (fp8/bf16 burst ratio"
+                     f"{', measured with torch._scaled_mm e4m3 8192^3' if fp8_burst else ', nominal'}; "
+                     f"kernel runs inside a long step)")
     launches = sum(n for _, n in prof.values())
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -370,6 +466,14 @@ def run_ours(args, rank, world, local_rank):
                 "api": "vdn_hybrid_attn_fwd_host, two streams", "max_abs_diff_vs_device_path": e2e_gap},
         "clocks": clk,
     }
+    if fp8_burst:
+        line["fp8_tflops_burst_measured"] = fp8_burst
+    if world == 1 and not args.no_dense_ref:
+        dense = dense_reference(s, dev)
+        if "layer_ms" in dense:
+            dense["layer_speedup_of_this_layer"] = dense["layer_ms"] / per_step_ms
+        line["dense_reference"] = dense
+    line["pages_context"] = PAGES_CONTEXT
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg, inp, args.cpu_rows)
     print(json.dumps(line), flush=True)
@@ -385,6 +489,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=48, help="query rows of the CPU oracle sample")
     ap.add_argument("--ref-rows", type=int, default=16, help="query rows per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense-ref", action="store_true", help="skip the dense cuDNN SDPA comparator")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

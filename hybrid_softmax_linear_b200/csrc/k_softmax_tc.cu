@@ -28,7 +28,7 @@ using namespace tc;
 constexpr int BM = 128;     // rows per Q tile
 constexpr int BN = 128;     // keys per K/V tile
 constexpr int NQ = 2;       // Q tiles per CTA
-constexpr int KST = 2, VST = 2;
+constexpr int KST = 2, VST = 3;  // V is refilled later in a step than K, so it gets the deeper ring
 constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
@@ -193,29 +193,40 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < C::BOXES; ++c)
           tma_load_2d(smem_u32(base + C::Q_OFF + w * C::TILE_BYTES + c * BM * 128), &tmQ, qb,
                       h * D + c * C::BOX_ELEMS, row0 + w * BM);
-      KvCursor cur;
-      cur.init(parts);
-      for (int j = 0; j < nkv; ++j) {
-        const int ks = j % KST, vs = j % VST;
-        const CUtensorMap *mk = parts.text[cur.part] ? &tmKt : &tmK;
-        const CUtensorMap *mv = parts.text[cur.part] ? &tmVt : &tmV;
-        if (!mbar_wait(smem_u32(&bars->k_empty[ks]), ((j / KST) & 1) ^ 1, abort_flag, st, K_SOFTMAX_TC, 1)) break;
+      // K runs one tile ahead of V: K_{j+1} is needed as soon as P_j V_j is issued, V_j only
+      // after the softmax of tile j
+      KvCursor ck, cv;
+      ck.init(parts);
+      cv.init(parts);
+      auto load_k = [&](int j) -> bool {
+        const int ks = j % KST;
+        if (!mbar_wait(smem_u32(&bars->k_empty[ks]), ((j / KST) & 1) ^ 1, abort_flag, st, K_SOFTMAX_TC, 1))
+          return false;
         const uint32_t kb = smem_u32(&bars->k_full[ks]);
         mbar_arrive_expect_tx(kb, C::TILE_BYTES);
+        const CUtensorMap *mk = parts.text[ck.part] ? &tmKt : &tmK;
         for (int c = 0; c < C::BOXES; ++c)
           tma_load_2d(smem_u32(base + C::K_OFF + ks * C::TILE_BYTES + c * BN * 128), mk, kb, h * D + c * C::BOX_ELEMS,
-                      cur.row);
+                      ck.row);
         armed_k |= 1u << ks;
         ph_k = (ph_k & ~(1u << ks)) | (((j / KST) & 1u) << ks);
+        ck.next(parts);
+        return true;
+      };
+      bool go = nkv > 0 && load_k(0);
+      for (int j = 0; go && j < nkv; ++j) {
+        if (j + 1 < nkv && !load_k(j + 1)) break;
+        const int vs = j % VST;
         if (!mbar_wait(smem_u32(&bars->v_empty[vs]), ((j / VST) & 1) ^ 1, abort_flag, st, K_SOFTMAX_TC, 2)) break;
         const uint32_t vb = smem_u32(&bars->v_full[vs]);
         mbar_arrive_expect_tx(vb, C::TILE_BYTES);
+        const CUtensorMap *mv = parts.text[cv.part] ? &tmVt : &tmV;
         for (int c = 0; c < C::BOXES; ++c)
           tma_load_2d(smem_u32(base + C::V_OFF + vs * C::TILE_BYTES + c * BN * 128), mv, vb, h * D + c * C::BOX_ELEMS,
-                      cur.row);
+                      cv.row);
         armed_v |= 1u << vs;
         ph_v = (ph_v & ~(1u << vs)) | (((j / VST) & 1u) << vs);
-        cur.next(parts);
+        cv.next(parts);
       }
       // loads issued here land before the block leaves (bounded waits)
       int no_abort = 0;
@@ -256,14 +267,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       for (int j = 0; ok && j < nkv; ++j) {
         const int vs = j % VST;
-        if (!mbar_wait(smem_u32(&bars->v_full[vs]), (j / VST) & 1, abort_flag, st, K_SOFTMAX_TC, 5)) break;
         const bool more = j + 1 < nkv;
-        if (more && !mbar_wait(smem_u32(&bars->k_full[(j + 1) % KST]), ((j + 1) / KST) & 1, abort_flag, st,
-                               K_SOFTMAX_TC, 6))
-          break;
         const uint32_t vbase = smem_u32(base + C::V_OFF + vs * C::TILE_BYTES);
         for (int w = 0; w < NQ && ok; ++w) {
+          // each wait sits right before the first MMA that needs it
           if (!mbar_wait(smem_u32(&bars->p_full[w]), j & 1, abort_flag, st, K_SOFTMAX_TC, 7)) { ok = false; break; }
+          if (w == 0 && !mbar_wait(smem_u32(&bars->v_full[vs]), (j / VST) & 1, abort_flag, st, K_SOFTMAX_TC, 5)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           // O_w += P_w V_j: P_w (two bf16 or four e4m3 per column) sits over the first columns
           // of S_w; each K-step takes 8 of those columns and KSTEP rows of V (128 bytes each)
@@ -279,8 +291,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             issue_s(1, 0);                               // staggered start of Q tile 1
             mma_commit(smem_u32(&bars->k_empty[0]));     // K tile 0 is free once both S of it complete
           }
-          if (more) issue_s(w, j + 1);
+          if (more) {
+            if (w == 0 && !mbar_wait(smem_u32(&bars->k_full[(j + 1) % KST]), ((j + 1) / KST) & 1, abort_flag, st,
+                                     K_SOFTMAX_TC, 6)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(w, j + 1);
+          }
         }
+        if (!ok) break;
         mma_commit(smem_u32(&bars->v_empty[vs]));
         if (more) mma_commit(smem_u32(&bars->k_empty[(j + 1) % KST]));
       }
