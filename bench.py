@@ -73,6 +73,38 @@ def load_peaks() -> tuple[dict, str]:
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "softmax_tc_dram_traffic.md")
+SOFTMAX_SRC = os.path.join(ROOT, "hybrid_softmax_linear_b200", "csrc", "k_softmax_tc.cu")
+
+
+def captured_traffic(s, fp8: bool) -> tuple[float | None, str]:
+    """DRAM bytes (read + write) of one softmax launch at this workload, from the committed
+    ncu capture, or None when the kernel source changed since that capture.  The capture
+    file holds lines `source_sha256: <hex>` and `<key>: <bytes> bytes over <units> units`,
+    key bf16 or e4m3, units = query rows x heads of the captured case."""
+    import hashlib
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no capture committed"
+    with open(SOFTMAX_SRC, "rb") as fh:
+        sha = hashlib.sha256(fh.read()).hexdigest()
+    fields = {}
+    with open(TRAFFIC_FILE) as fh:
+        for ln in fh:
+            if ":" in ln and not ln.startswith(("#", "|", " ")):
+                k, v = ln.split(":", 1)
+                fields[k.strip().strip("`")] = v.strip().strip("`")
+    if fields.get("source_sha256") != sha:
+        return None, "kernel source changed since the capture"
+    entry = fields.get("e4m3" if fp8 else "bf16")
+    if entry is None:
+        return None, "no capture of this dtype"
+    parts = entry.split()
+    nbytes, units = float(parts[0]), float(parts[3])
+    scale = s.n_video * s.heads / units
+    how = "measured at this size" if abs(scale - 1.0) < 1e-9 else f"scaled x{scale:.3f} by query rows x heads"
+    return nbytes * scale, how
+
+
 class ClockSampler:
     """SM clock, power and clock-event reasons sampled every 20 ms during the timed region
     (NVML through nvidia_ml_py, the GPU found by its UUID; nvidia-smi -lms 200 if NVML is
@@ -449,13 +481,15 @@ def run_ours(args, rank, world, local_rank):
         peak_note = (f"{peak_src} bf16_tflops_sustained x {ratio:.3f} (fp8/bf16 burst ratio"
                      f"{', measured with torch._scaled_mm e4m3 8192^3' if fp8_burst else ', nominal'}; "
                      f"kernel runs inside a long step)")
+    traffic, traffic_note = captured_traffic(s, w.softmax_fp8)
     launches = sum(n for _, n in prof.values())
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic", "config": workload_config(cfg),
         "roofline": {"kernel": sm_key, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                     "traffic_note": traffic_note,
                      "peak_source": peak_note,
                      "algorithmic_tflop_per_launch": fl["softmax"] / 1e12, "avg_launch_ms": sm_avg},
         "layer_tflops": sum(v for k, v in fl.items()) / (per_step_ms / 1e3) / 1e12,

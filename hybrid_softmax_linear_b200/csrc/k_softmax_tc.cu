@@ -28,7 +28,7 @@ using namespace tc;
 constexpr int BM = 128;     // rows per Q tile
 constexpr int BN = 128;     // keys per K/V tile
 constexpr int NQ = 2;       // Q tiles per CTA
-constexpr int KST = 2, VST = 3;  // V is refilled later in a step than K, so it gets the deeper ring
+constexpr int KST = 2, VST = 2;
 constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units

@@ -59,3 +59,23 @@ def test_softmax_flop_count_matches_brute_force():
     keys = sum(s.tokens_per_frame * (s.text_tokens + s.tokens_per_frame * int((M[f] == vo.SOFT).sum()))
                for f in range(s.frames))
     assert bench.softmax_flops(s) == 4.0 * s.head_dim * s.heads * keys
+
+
+def test_captured_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed capture only while the kernel source is the
+    one captured, scaled by query rows x heads."""
+    import hashlib
+    src = tmp_path / "k.cu"
+    src.write_text("kernel source\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    cap = tmp_path / "cap.md"
+    cap.write_text(f"# title\n\nsource_sha256: {sha}\nbf16: 1000 bytes over 10 units\n")
+    monkeypatch.setattr(bench, "SOFTMAX_SRC", str(src))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(cap))
+    shape = synth.Shape(2, 5, 1, 0, 2, 32)                     # 10 rows x 2 heads = 20 units
+    t, how = bench.captured_traffic(shape, fp8=False)
+    assert t == 2000.0 and "scaled" in how
+    assert bench.captured_traffic(shape, fp8=True)[0] is None  # no e4m3 entry
+    src.write_text("changed\n")
+    assert bench.captured_traffic(shape, fp8=False)[0] is None
+
