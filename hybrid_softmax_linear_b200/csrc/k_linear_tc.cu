@@ -242,24 +242,31 @@ __global__ void __launch_bounds__(256) read_stage_kernel(int64_t n_s8, int64_t n
 
 // ============================================================================ read (+ gate, RMSNorm)
 // One CTA per 128 query rows (half of a 256-row tile) and head; two CTAs fit on an SM.
-// Warp 0 loads Q, S_sum and W_l with TMA and one of its threads issues the MMAs: the gate
-// logits Q W_l as soon as Q lands, then num = feature * S_sum once the feature rows are
-// in place.  Warps 1-4 (one query row per thread) compute the feature row phi(q) (or
-// q/|q|), the normaliser phi(q).z and, with G_l = 1, the scalar gate, keep it in
-// registers until the gate MMA has consumed Q, and write it over Q; then they form
-// o = num / den and store o (plain) or A_l = g_l * gamma * o / rms(o) (layer).
+// Eight warps; each query row belongs to two threads (one per column half), and thread 0
+// also drives the copy engine and the tensor cores:
+//   1. thread 0 loads Q, S_sum and W_l with TMA; everyone waits for them;
+//   2. thread 0 issues the gate logits Q W_l (G_l = D) while every thread builds its half of
+//      the feature row phi(q) (or q/|q|), its part of the normaliser phi(q).z and, with
+//      G_l = 1, of the scalar gate logit;
+//   3. once the gate MMA has read Q the features go over it; thread 0 issues
+//      num = feature * S_sum;
+//   4. every thread forms its half of o = num / den and stores o, or
+//      A_l = g_l * gamma * o / rms(o) with the sum of squares shared between the halves.
+// The halves meet through shared memory at block barriers that every thread reaches
+// whatever happened before (a failed wait only turns the remaining work off).
 namespace rd {
-constexpr int D = 128, BM = 128, THREADS = 160;
+constexpr int D = 128, BM = 128, THREADS = 256, HC = D / 2;
 constexpr int TILE_BYTES = BM * D * 2;  // 32 KB: one 128-row bf16 tile (two 64-column boxes)
 constexpr int Q_OFF = 0, S_OFF = TILE_BYTES, W_OFF = 2 * TILE_BYTES;
 constexpr int BAR_OFF = 3 * TILE_BYTES;
 constexpr uint32_t IDESC_NUM = idesc_bf16(BM, D, false, true);   // A K-major, B MN-major
 constexpr uint32_t TMEM_COLS = 256;                               // num at 0, gate logits at 128
 struct alignas(8) Bars {
-  uint64_t in_full, gate_done, feat, acc, drain;
+  uint64_t in_full, gate_done, acc, drain;
   uint32_t tmem;
   int abort;
   float z[D], gamma[D], wg1[D];
+  float part[3][2][BM];  // per column half: normaliser, scalar-gate logit, sum of squares
 };
 constexpr size_t SMEM = 1024 + BAR_OFF + sizeof(Bars);
 }  // namespace rd
@@ -278,10 +285,10 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   Bars *bars = reinterpret_cast<Bars *>(base + BAR_OFF);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int *abort_flag = &bars->abort;
   __shared__ int skip;
-  if (threadIdx.x == 0) skip = *(volatile uint32_t *)&st->code != 0u;
+  if (tid == 0) skip = *(volatile uint32_t *)&st->code != 0u;
   __syncthreads();
   if (skip) return;
 
@@ -293,168 +300,188 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
   const int row0 = tr[1] + (int)(half_tile & 1) * BM, row_end = tr[2];
   if (row0 >= row_end) return;  // the second half of a short tile (block-uniform)
 
-  if (threadIdx.x == 0) {
+  const int quad = warp & 3, hf = warp >> 2;  // lane quarter (tensor-memory rule), column half
+  const int r = quad * 32 + lane;             // row within the tile
+  const int c0 = hf * HC;                     // first column of this thread's half
+  if (tid == 0) {
     mbar_init(smem_u32(&bars->in_full), 1);
     mbar_init(smem_u32(&bars->gate_done), 1);
-    mbar_init(smem_u32(&bars->feat), 4);
     mbar_init(smem_u32(&bars->acc), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x < D) {
-    bars->z[threadIdx.x] = delta ? 0.f : zsum[((int64_t)g * d.H + h) * D + threadIdx.x];
-    bars->gamma[threadIdx.x] = fused ? gamma[(int64_t)h * D + threadIdx.x] : 0.f;
-    bars->wg1[threadIdx.x] = (fused && !gate_mma) ? wgl[((int64_t)h * D + threadIdx.x) * G_l] : 0.f;
+  if (tid < D) {
+    bars->z[tid] = delta ? 0.f : zsum[((int64_t)g * d.H + h) * D + tid];
+    bars->gamma[tid] = fused ? gamma[(int64_t)h * D + tid] : 0.f;
+    bars->wg1[tid] = (fused && !gate_mma) ? wgl[((int64_t)h * D + tid) * G_l] : 0.f;
   }
   if (warp == 0) { tmem_alloc(smem_u32(&bars->tmem), TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
+  const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+  const uint32_t qa = smem_u32(base + Q_OFF), sb_ = smem_u32(base + S_OFF), wb = smem_u32(base + W_OFF);
+  const uint32_t fb = smem_u32(&bars->in_full);
+  bool issued = false;  // thread 0: MMAs in flight that must drain before the block exits
 
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint32_t fb = smem_u32(&bars->in_full);
-      mbar_arrive_expect_tx(fb, (2 + (gate_mma ? 1 : 0)) * TILE_BYTES);
-      for (int b = 0; b < 2; ++b) {
-        tma_load_2d(smem_u32(base + Q_OFF + b * BM * 128), &tmQ, fb, h * D + b * 64, row0);
-        tma_load_2d(smem_u32(base + S_OFF + b * BM * 128), &tmS, fb, b * 64, (g * d.H + h) * D);
-        if (gate_mma) tma_load_2d(smem_u32(base + W_OFF + b * BM * 128), &tmW, fb, b * 64, h * D);
-      }
-      bool ok = mbar_wait(fb, 0, abort_flag, st, K_READ, 1);
-      if (ok) {
-        tc_fence_after();
-        const uint32_t qa = smem_u32(base + Q_OFF), sb_ = smem_u32(base + S_OFF), wb = smem_u32(base + W_OFF);
-        if (gate_mma) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + 128, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc(wb + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
-        }
-        mma_commit(smem_u32(&bars->gate_done));  // Q may be overwritten once this arrives
-        if (mbar_wait(smem_u32(&bars->feat), 0, abort_flag, st, K_READ, 3)) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc(sb_ + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
-          mma_commit(smem_u32(&bars->acc));
-        }
-      }
-      mma_commit(smem_u32(&bars->drain));
-      int no_abort = 0;
-      mbar_wait(fb, 0, &no_abort, st, K_READ, 2);
-      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_READ, 4);
+  // ---- 1. operands
+  if (tid == 0) {
+    mbar_arrive_expect_tx(fb, (2 + (gate_mma ? 1 : 0)) * TILE_BYTES);
+    for (int b = 0; b < 2; ++b) {
+      tma_load_2d(smem_u32(base + Q_OFF + b * BM * 128), &tmQ, fb, h * D + b * 64, row0);
+      tma_load_2d(smem_u32(base + S_OFF + b * BM * 128), &tmS, fb, b * 64, (g * d.H + h) * D);
+      if (gate_mma) tma_load_2d(smem_u32(base + W_OFF + b * BM * 128), &tmW, fb, b * 64, h * D);
     }
-  } else {
-    const int quad = warp & 3, r = quad * 32 + lane;
-    const int row = row0 + r;
-    const bool valid = row < row_end;
-    uint8_t *qt = base + Q_OFF;
-    const bool got = mbar_wait(smem_u32(&bars->in_full), 0, abort_flag, st, K_READ, 5);
-    bool ok = __all_sync(0xffffffffu, got);
-    float den = 0.f, gate1 = 0.f;
-    if (ok) {
-      // feature row in registers (bf16 pairs): phi(q), or q/|q| for the delta rule
-      uint32_t fr[D / 2];
-      float inv_norm = 1.f;
-      const bool scalar_gate = fused && !gate_mma;
-      if (delta) {
-        float ss = 0.f;
+  }
+  bool ok = __syncthreads_and(mbar_wait(fb, 0, abort_flag, st, K_READ, 1)) != 0;
+
+  // ---- 2. gate logits on the tensor cores; the feature half-row in registers
+  if (ok && tid == 0) {
+    tc_fence_after();
+    if (gate_mma) {
 #pragma unroll
-        for (int cl = 0; cl < D / 8; ++cl) {
-          float f[8];
-          unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ss(tmem + 128, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
+               sdesc(wb + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
+    }
+    mma_commit(smem_u32(&bars->gate_done));  // Q may be overwritten once this arrives
+    issued = true;
+  }
+  __syncwarp();
+  uint8_t *qt = base + Q_OFF;
+  uint32_t fr[HC / 2];
+  float den = 0.f, gate1 = 0.f, ssq = 0.f;
+  if (ok) {
+    if (delta) {
+      // |q|^2 over the whole row: this half's share now, the other's through part[2]
 #pragma unroll
-          for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
-        }
-        inv_norm = ss > 0.f ? rsqrtf(ss) : 0.f;
-      }
-#pragma unroll
-      for (int cl = 0; cl < D / 8; ++cl) {
+      for (int cl = c0 / 8; cl < (c0 + HC) / 8; ++cl) {
         float f[8];
         unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (scalar_gate) gate1 = fmaf(f[e], bars->wg1[cl * 8 + e], gate1);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (delta) {
-            f[e] *= inv_norm;
-          } else {
-            f[e] = f[e] > 0.f ? f[e] + 1.f : __expf(f[e]);
-            den = fmaf(f[e], bars->z[cl * 8 + e], den);
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) fr[cl * 4 + e] = pack_bf16(f[2 * e], f[2 * e + 1]);
-      }
-      // Q is the A operand of the gate MMA: write the features over it only afterwards
-      const bool gd = mbar_wait(smem_u32(&bars->gate_done), 0, abort_flag, st, K_READ, 7);
-      ok = __all_sync(0xffffffffu, gd);
-      if (ok) {
-#pragma unroll
-        for (int cl = 0; cl < D / 8; ++cl)
-          *reinterpret_cast<uint4 *>(qt + swz_off(r, cl, BM)) =
-              make_uint4(fr[cl * 4], fr[cl * 4 + 1], fr[cl * 4 + 2], fr[cl * 4 + 3]);
-        fence_proxy_async();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->feat));
-        const bool done = mbar_wait(smem_u32(&bars->acc), 0, abort_flag, st, K_READ, 6);
-        ok = __all_sync(0xffffffffu, done);
+        for (int e = 0; e < 8; ++e) ssq = fmaf(f[e], f[e], ssq);
       }
     }
-    if (ok) {
-      tc_fence_after();
-      const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-      const float scale = delta ? 1.f : (den > 0.f ? 1.f / den : 0.f);
-      __nv_bfloat16 *orow = out + (int64_t)row * out_stride + (int64_t)h * D;
-      // the accumulator is read twice (sum of squares, then the output) to keep registers low
-      float rinv = 1.f;
-      if (fused) {
-        float ss = 0.f;
+    bars->part[2][hf][r] = ssq;
+  }
+  __syncthreads();
+  float inv_norm = 1.f;
+  if (ok && delta) {
+    const float qq = bars->part[2][0][r] + bars->part[2][1][r];
+    inv_norm = qq > 0.f ? rsqrtf(qq) : 0.f;
+  }
+  if (ok) {
+    const bool scalar_gate = fused && !gate_mma;
 #pragma unroll
-        for (int c = 0; c < D; c += 64) {
-          uint32_t u0[32], u1[32];
-          tmem_ld32(tmem + lane_off + c, u0);
-          tmem_ld32(tmem + lane_off + c + 32, u1);
-          tmem_wait_ld();
+    for (int i = 0; i < HC / 8; ++i) {
+      const int cl = c0 / 8 + i;
+      float f[8];
+      unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
+      if (scalar_gate) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float a = __uint_as_float(u0[i]) * scale, b = __uint_as_float(u1[i]) * scale;
-            ss = fmaf(a, a, ss);
-            ss = fmaf(b, b, ss);
-          }
-        }
-        rinv = rsqrtf(ss / (float)D + eps);
+        for (int e = 0; e < 8; ++e) gate1 = fmaf(f[e], bars->wg1[cl * 8 + e], gate1);
       }
-      const float gs = fast_sigmoid(gate1);
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        uint32_t u[32], ug[32];
-        tmem_ld32(tmem + lane_off + c, u);
-        if (fused && gate_mma) tmem_ld32(tmem + lane_off + 128 + c, ug);
-        tmem_wait_ld();
-        if (valid) {
+      for (int e = 0; e < 8; ++e) {
+        if (delta) {
+          f[e] *= inv_norm;
+        } else {
+          f[e] = f[e] > 0.f ? f[e] + 1.f : __expf(f[e]);
+          den = fmaf(f[e], bars->z[cl * 8 + e], den);
+        }
+      }
 #pragma unroll
-          for (int v = 0; v < 32; v += 8) {
-            float a[8];
+      for (int e = 0; e < 4; ++e) fr[i * 4 + e] = pack_bf16(f[2 * e], f[2 * e + 1]);
+    }
+  }
+  // ---- 3. features over Q once the gate MMA has read it; then num
+  ok = __syncthreads_and(ok && mbar_wait(smem_u32(&bars->gate_done), 0, abort_flag, st, K_READ, 2)) != 0;
+  if (ok) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float o = __uint_as_float(u[v + e]) * scale;
-              if (!fused) {
-                a[e] = o;
-              } else {
-                const float gl = gate_mma ? fast_sigmoid(__uint_as_float(ug[v + e])) : gs;
-                a[e] = gl * bars->gamma[c + v + e] * o * rinv;
-              }
+    for (int i = 0; i < HC / 8; ++i)
+      *reinterpret_cast<uint4 *>(qt + swz_off(r, c0 / 8 + i, BM)) =
+          make_uint4(fr[i * 4], fr[i * 4 + 1], fr[i * 4 + 2], fr[i * 4 + 3]);
+    fence_proxy_async();
+  }
+  bars->part[0][hf][r] = den;
+  bars->part[1][hf][r] = gate1;
+  __syncthreads();
+  if (ok && tid == 0) {
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      mma_ss(tmem, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
+             sdesc(sb_ + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
+    mma_commit(smem_u32(&bars->acc));
+  }
+  __syncwarp();
+  ok = __syncthreads_and(ok && mbar_wait(smem_u32(&bars->acc), 0, abort_flag, st, K_READ, 3)) != 0;
+
+  // ---- 4. epilogue on this thread's half of the row
+  const float den_row = bars->part[0][0][r] + bars->part[0][1][r];
+  const float g1_row = bars->part[1][0][r] + bars->part[1][1][r];
+  const float scale = delta ? 1.f : (den_row > 0.f ? 1.f / den_row : 0.f);
+  const uint32_t acc = tmem + lane_off + (uint32_t)c0;
+  float ss = 0.f;
+  if (ok) {
+    tc_fence_after();
+    if (fused) {
+      uint32_t u0[32], u1[32];
+      tmem_ld32(acc, u0);
+      tmem_ld32(acc + 32, u1);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float a = __uint_as_float(u0[i]) * scale, b = __uint_as_float(u1[i]) * scale;
+        ss = fmaf(a, a, ss);
+        ss = fmaf(b, b, ss);
+      }
+    }
+  }
+  __syncthreads();  // part[2] held the |q|^2 halves of the delta rule: all read before reuse
+  bars->part[2][hf][r] = ss;
+  __syncthreads();
+  if (ok) {
+    const int row = row0 + r;
+    const bool valid = row < row_end;
+    const float rinv = fused ? rsqrtf((bars->part[2][0][r] + bars->part[2][1][r]) / (float)D + eps) : 1.f;
+    const float f_row = scale * rinv;  // o / rms(o) = num * scale * rinv
+    const float gs = fast_sigmoid(g1_row);
+    __nv_bfloat16 *orow = out + (int64_t)row * out_stride + (int64_t)h * D + c0;
+#pragma unroll
+    for (int c = 0; c < HC; c += 32) {
+      uint32_t u[32], ug[32];
+      tmem_ld32(acc + c, u);
+      if (fused && gate_mma) tmem_ld32(acc + 128 + c, ug);
+      tmem_wait_ld();
+      if (valid) {
+#pragma unroll
+        for (int v = 0; v < 32; v += 8) {
+          float o8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float o = __uint_as_float(u[v + e]) * f_row;
+            if (!fused) {
+              o8[e] = o;
+            } else {
+              const float gl = gate_mma ? fast_sigmoid(__uint_as_float(ug[v + e])) : gs;
+              o8[e] = gl * bars->gamma[c0 + c + v + e] * o;
             }
-            *reinterpret_cast<uint4 *>(orow + c + v) = pack8(a);
           }
+          *reinterpret_cast<uint4 *>(orow + c + v) = pack8(o8);
         }
       }
+    }
+  }
+  // ---- drain: no copy or MMA of this block may be in flight when it exits
+  if (tid == 0) {
+    int no_abort = 0;
+    mbar_wait(fb, 0, &no_abort, st, K_READ, 4);
+    if (issued) {
+      mma_commit(smem_u32(&bars->drain));
+      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_READ, 5);
     }
   }
   tc_fence_before();
