@@ -33,6 +33,10 @@ __device__ __forceinline__ uint32_t swz_off(int r, int cl, int box_rows) {
   return (uint32_t)((cl >> 3) * box_rows * 128 + r * 128 + ((((cl & 7) ^ (r & 7))) << 4));
 }
 
+// phi(x) = elu(x) + 1 without a branch: max(x, 0) + e^min(x, 0) is x + 1 for x > 0 (e^0 = 1
+// exactly) and e^x otherwise, and keeps the warp converged whatever the signs
+__device__ __forceinline__ float phi_fast(float x) { return fmaxf(x, 0.f) + __expf(fminf(x, 0.f)); }
+
 __device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
   const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
 #pragma unroll
@@ -168,7 +172,7 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           // phi enters the MMA in bf16, so the fast exponential is accurate enough
-          const float ph = valid ? (f[e] > 0.f ? f[e] + 1.f : __expf(f[e])) : 0.f;
+          const float ph = valid ? phi_fast(f[e]) : 0.f;
           zacc[e] += ph;
           f[e] = ph;
         }
@@ -261,14 +265,18 @@ constexpr int Q_OFF = 0, S_OFF = TILE_BYTES, W_OFF = 2 * TILE_BYTES;
 constexpr int BAR_OFF = 3 * TILE_BYTES;
 constexpr uint32_t IDESC_NUM = idesc_bf16(BM, D, false, true);   // A K-major, B MN-major
 constexpr uint32_t TMEM_COLS = 256;                               // num at 0, gate logits at 128
-struct alignas(8) Bars {
+struct alignas(16) Bars {
+  float z[D], gamma[D], wg1[D];
+  float part[3][2][BM];  // per column half: normaliser, scalar-gate logit, sum of squares
   uint64_t in_full, gate_done, acc, drain;
   uint32_t tmem;
   int abort;
-  float z[D], gamma[D], wg1[D];
-  float part[3][2][BM];  // per column half: normaliser, scalar-gate logit, sum of squares
 };
 constexpr size_t SMEM = 1024 + BAR_OFF + sizeof(Bars);
+// Output rows are staged in shared memory (over Q and S, free once num is complete) with a
+// 16-byte pad per row, then written out two whole rows per warp instruction.
+constexpr int OUT_PITCH = D * 2 + 16;
+static_assert(BM * OUT_PITCH <= 2 * TILE_BYTES, "output staging must fit over Q and S");
 }  // namespace rd
 
 // 1 / (1 + 2^(-x log2 e)) with the hardware exp2 and reciprocal approximations (relative
@@ -366,7 +374,7 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
     }
     bars->part[2][hf][r] = ssq;
   }
-  __syncthreads();
+  if (delta) __syncthreads();  // block-uniform: the |q|^2 halves meet (delta rule only)
   float inv_norm = 1.f;
   if (ok && delta) {
     const float qq = bars->part[2][0][r] + bars->part[2][1][r];
@@ -388,9 +396,15 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
         if (delta) {
           f[e] *= inv_norm;
         } else {
-          f[e] = f[e] > 0.f ? f[e] + 1.f : __expf(f[e]);
-          den = fmaf(f[e], bars->z[cl * 8 + e], den);
+          f[e] = phi_fast(f[e]);
         }
+      }
+      if (!delta) {
+        const float4 za = *reinterpret_cast<const float4 *>(&bars->z[cl * 8]);
+        const float4 zb = *reinterpret_cast<const float4 *>(&bars->z[cl * 8 + 4]);
+        den = fmaf(f[0], za.x, den); den = fmaf(f[1], za.y, den); den = fmaf(f[2], za.z, den);
+        den = fmaf(f[3], za.w, den); den = fmaf(f[4], zb.x, den); den = fmaf(f[5], zb.y, den);
+        den = fmaf(f[6], zb.z, den); den = fmaf(f[7], zb.w, den);
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) fr[i * 4 + e] = pack_bf16(f[2 * e], f[2 * e + 1]);
@@ -434,45 +448,55 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
       tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float a = __uint_as_float(u0[i]) * scale, b = __uint_as_float(u1[i]) * scale;
+        const float a = __uint_as_float(u0[i]), b = __uint_as_float(u1[i]);
         ss = fmaf(a, a, ss);
         ss = fmaf(b, b, ss);
       }
+      ss *= scale * scale;
     }
   }
   __syncthreads();  // part[2] held the |q|^2 halves of the delta rule: all read before reuse
   bars->part[2][hf][r] = ss;
   __syncthreads();
+  uint8_t *stage = base + Q_OFF;  // Q, F and S are no longer read once num is complete
   if (ok) {
-    const int row = row0 + r;
-    const bool valid = row < row_end;
     const float rinv = fused ? rsqrtf((bars->part[2][0][r] + bars->part[2][1][r]) / (float)D + eps) : 1.f;
     const float f_row = scale * rinv;  // o / rms(o) = num * scale * rinv
     const float gs = fast_sigmoid(g1_row);
-    __nv_bfloat16 *orow = out + (int64_t)row * out_stride + (int64_t)h * D + c0;
+    uint8_t *srow = stage + r * OUT_PITCH + c0 * 2;
 #pragma unroll
     for (int c = 0; c < HC; c += 32) {
       uint32_t u[32], ug[32];
       tmem_ld32(acc + c, u);
       if (fused && gate_mma) tmem_ld32(acc + 128 + c, ug);
       tmem_wait_ld();
-      if (valid) {
 #pragma unroll
-        for (int v = 0; v < 32; v += 8) {
-          float o8[8];
+      for (int v = 0; v < 32; v += 8) {
+        float o8[8];
+        if (fused) {
+          const float4 ga = *reinterpret_cast<const float4 *>(&bars->gamma[c0 + c + v]);
+          const float4 gb = *reinterpret_cast<const float4 *>(&bars->gamma[c0 + c + v + 4]);
+          const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float o = __uint_as_float(u[v + e]) * f_row;
-            if (!fused) {
-              o8[e] = o;
-            } else {
-              const float gl = gate_mma ? fast_sigmoid(__uint_as_float(ug[v + e])) : gs;
-              o8[e] = gl * bars->gamma[c0 + c + v + e] * o;
-            }
+            const float gl = gate_mma ? fast_sigmoid(__uint_as_float(ug[v + e])) : gs;
+            o8[e] = gl * gg[e] * (__uint_as_float(u[v + e]) * f_row);
           }
-          *reinterpret_cast<uint4 *>(orow + c + v) = pack8(o8);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o8[e] = __uint_as_float(u[v + e]) * f_row;
         }
+        *reinterpret_cast<uint4 *>(srow + (c + v) * 2) = pack8(o8);
       }
+    }
+  }
+  __syncthreads();
+  if (ok) {
+    // two rows per warp instruction: lanes 0-15 one row, 16-31 the next (256 bytes each)
+    const int nrows = min(BM, row_end - row0);
+    for (int rr = warp * 2 + (lane >> 4); rr < nrows; rr += 2 * (THREADS / 32)) {
+      const uint4 val = *reinterpret_cast<const uint4 *>(stage + rr * OUT_PITCH + (lane & 15) * 16);
+      *reinterpret_cast<uint4 *>(out + (int64_t)(row0 + rr) * out_stride + (int64_t)h * D + (lane & 15) * 8) = val;
     }
   }
   // ---- drain: no copy or MMA of this block may be in flight when it exits

@@ -269,7 +269,8 @@ template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
-__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
+// elu(x) + 1 as max(x, 0) + e^min(x, 0): no branch, the same value (e^0 = 1 exactly)
+__device__ __forceinline__ float phi_elu1(float x) { return fmaxf(x, 0.f) + expf(fminf(x, 0.f)); }
 
 // ---------------------------------------------------------------- launchers
 struct Dims {
