@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(256) scan_delta_kernel(Dims d, const float *__
 
 // Segmented scan of the ELU1 memories.  A block owns 128 consecutive entries (32 lanes x
 // float4) of the flattened [D*D | D] state of one head.  Its warps first sum the frames
-// of each segment (the frames between two consecutive memory boundaries; four loads in
+// of each segment (the frames between two consecutive memory boundaries; eight loads in
 // flight per lane), then warp 0 forms the exclusive prefix sums and warp 1 the suffix
 // sums over the segments, and every group's memories are read off those:
 // S_fwd = S_txt/2 + prefix[ie_g], S_bwd = S_txt/2 + suffix[ib_g].  With SUM the block
@@ -408,16 +408,16 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_seg_kernel(Dims d, const fl
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     if (valid) {
       const int hi = bnd[j + 1];
-      int f = bnd[j];
-      for (; f + 4 <= hi; f += 4) {
-        const float4 x0 = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)f * fstride));
-        const float4 x1 = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(f + 1) * fstride));
-        const float4 x2 = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(f + 2) * fstride));
-        const float4 x3 = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(f + 3) * fstride));
-        a = f4add(a, f4add(x0, x1));
-        b = f4add(b, f4add(x2, x3));
+      // eight frames per round trip: a segment of up to eight frames costs one memory latency
+      for (int f = bnd[j]; f < hi; f += 8) {
+        float4 x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          x[k] = f + k < hi ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(f + k) * fstride))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        a = f4add(a, f4add(f4add(x[0], x[1]), f4add(x[2], x[3])));
+        b = f4add(b, f4add(f4add(x[4], x[5]), f4add(x[6], x[7])));
       }
-      for (; f < hi; ++f) a = f4add(a, __ldg(reinterpret_cast<const float4 *>(src + (int64_t)f * fstride)));
     }
     seg[j * 32 + lane] = f4add(a, b);
   }
