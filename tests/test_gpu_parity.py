@@ -315,3 +315,45 @@ def test_host_entry_point_matches_device_entry_point(kind_dtype):
     ref = vo.layer(oracle_inputs(inp), s.frames, s.tokens_per_frame, s.chunk_frames, rows=np.arange(s.n_video),
                    linear="delta" if kind == vdn.DELTA else "elu1")
     assert rel_l2(got, ref["y"]) <= (3e-2 if cdt == vdn.E4M3 else 5e-3)
+
+
+# ----------------------------------------------------------------------------- read-kernel modes
+@pytest.mark.parametrize("kind", [vdn.ELU1, vdn.DELTA])
+def test_scalar_linear_gate_tensor_core_path(kind):
+    """G_l = 1 on the D = 128 tensor-core path (the scalar-gate instantiation of the read)."""
+    shape = synth.Shape(12, 300, 5, 40, 2, 128)
+    inp = synth.make_inputs(shape, "bf16", seed=6, gate_l_cols=1, with_beta=kind == vdn.DELTA)
+    run = Run(shape, inp, "bf16", kind=kind)
+    s = run.shape
+    rows = np.arange(s.n_video)
+    o = oracle_inputs(inp)
+    y = run.layer()
+    HD = s.heads * s.head_dim
+    A = to_numpy(run.intermediate(2, (s.n_video, 2 * HD), torch.bfloat16))
+    ref = vo.layer(o, s.frames, s.tokens_per_frame, s.chunk_frames, rows=rows,
+                   linear="delta" if kind == vdn.DELTA else "elu1")
+    assert_close("A_l (scalar gate)", A[:, HD:], ref["a"][:, HD:], "bf16")
+    assert_close("y", to_numpy(y), ref["y"], "bf16")
+
+
+def test_delta_plain_read_tensor_core_path():
+    """vdn_linear_read with the delta rule at D = 128 (the plain delta instantiation)."""
+    s = synth.Shape(12, 300, 5, 40, 2, 128)
+    F, T, C, L, H, D = 12, 300, 5, 40, 2, 128
+    inp = synth.make_inputs(s, "bf16", seed=23, with_beta=True)
+    d = {n: to_device(a) for n, a in inp.items()}
+    o = oracle_inputs(inp)
+    ws = workspace(vdn.step_workspace_size(s))
+    vdn.workspace_init(ws)
+    rSf, rSb = vo.delta_memory(o["k"], o["v"], o["kt"], o["vt"], o["beta"], F, T, C)
+    _, gtab = vdn.mask_layout_build(s)
+    G = vdn.max_groups(s)
+    Sf = torch.zeros((G, H, D, D), dtype=torch.float32, device="cuda")
+    Sb = torch.zeros((G, H, D, D), dtype=torch.float32, device="cuda")
+    first = [int(r[0]) for r in gtab]
+    Sf[:len(gtab)] = torch.from_numpy(rSf[first].astype(np.float32)).cuda()
+    Sb[:len(gtab)] = torch.from_numpy(rSb[first].astype(np.float32)).cuda()
+    o_l = empty((s.n_video, H, D), "bf16")
+    vdn.linear_read(s, vdn.DELTA, vdn.BF16, d["q"], Sf, Sb, None, None, o_l, ws)
+    vdn.check_device_status(ws)
+    assert_close("delta read (tensor cores)", to_numpy(o_l), vo.delta_read(o["q"], rSf, rSb, T), "bf16")
