@@ -220,6 +220,59 @@ __global__ void __launch_bounds__(D) delta_stats_kernel(Dims d, const T *__restr
   vbar[((int64_t)f * d.H + h) * D + i] = sv;
 }
 
+// Frame means for the delta rule, bf16 and D = 128: 16 threads cover a token row of one
+// head with 16-byte loads (8 values each) and the block's 16 token slices are summed
+// through shared memory; then kbar is L2-normalised.
+constexpr int DS_THREADS = 256, DS_SLICES = DS_THREADS / 16;
+__global__ void __launch_bounds__(DS_THREADS) delta_stats_bf16_kernel(Dims d, const __nv_bfloat16 *__restrict__ k,
+                                                                      const __nv_bfloat16 *__restrict__ v,
+                                                                      float *__restrict__ kbar,
+                                                                      float *__restrict__ vbar) {
+  constexpr int D = 128;
+  __shared__ float acc[2][DS_SLICES][D];
+  __shared__ float nrm;
+  const int f = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int c8 = (tid & 15) * 8, sl = tid >> 4;
+  const int64_t HD = (int64_t)d.H * D;
+  const __nv_bfloat16 *kb = k + (int64_t)f * d.T * HD + h * D + c8;
+  const __nv_bfloat16 *vb = v + (int64_t)f * d.T * HD + h * D + c8;
+  float sk[8], sv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) sk[e] = sv[e] = 0.f;
+#pragma unroll 4
+  for (int t = sl; t < d.T; t += DS_SLICES) {
+    float a[8], b[8];
+    load8(kb + (int64_t)t * HD, a);
+    load8(vb + (int64_t)t * HD, b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { sk[e] += a[e]; sv[e] += b[e]; }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { acc[0][sl][c8 + e] = sk[e]; acc[1][sl][c8 + e] = sv[e]; }
+  __syncthreads();
+  float mk = 0.f, mv = 0.f;
+  if (tid < D) {
+#pragma unroll
+    for (int q = 0; q < DS_SLICES; ++q) { mk += acc[0][q][tid]; mv += acc[1][q][tid]; }
+    mk /= (float)d.T;
+    mv /= (float)d.T;
+  }
+  const float ss = warp_sum(tid < D ? mk * mk : 0.f);
+  __syncthreads();  // acc is reused for the per-warp sums of squares
+  if ((tid & 31) == 0) acc[0][0][tid >> 5] = ss;
+  __syncthreads();
+  if (tid == 0) {
+    float tot = 0.f;
+    for (int w = 0; w < DS_THREADS / 32; ++w) tot += acc[0][0][w];
+    nrm = tot > 0.f ? rsqrtf(tot) : 0.f;
+  }
+  __syncthreads();
+  if (tid < D) {
+    kbar[((int64_t)f * d.H + h) * D + tid] = mk * nrm;
+    vbar[((int64_t)f * d.H + h) * D + tid] = mv;
+  }
+}
+
 template <typename T, int D>
 static cudaError_t state_build_t(const Dims &d, vdn_lin_kind kind, const void *k, const void *v, const void *kt,
                                  const void *vt, float *S, float *z, float *St, float *zt, cudaStream_t st) {
@@ -228,7 +281,10 @@ static cudaError_t state_build_t(const Dims &d, vdn_lin_kind kind, const void *k
                                                                  (const T *)vt, S, z, St, zt, d.F, 0);
     return cudaGetLastError();
   }
-  delta_stats_kernel<T, D><<<dim3(d.F, d.H), D, 0, st>>>(d, (const T *)k, (const T *)v, S, z);
+  if constexpr (D == 128 && sizeof(T) == 2)
+    delta_stats_bf16_kernel<<<dim3(d.F, d.H), DS_THREADS, 0, st>>>(d, (const T *)k, (const T *)v, S, z);
+  else
+    delta_stats_kernel<T, D><<<dim3(d.F, d.H), D, 0, st>>>(d, (const T *)k, (const T *)v, S, z);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // text init only: one block per head, with L2-normalised text keys
@@ -304,14 +360,103 @@ __global__ void __launch_bounds__(256) scan_elu1_kernel(Dims d, const float *__r
   }
 }
 
-// Delta-rule scan: block per (head, direction); the D x D state lives in shared memory.
-// Step with frame f: u = S^T kbar; S += beta kbar (vbar - u)^T, which is
-// S <- (I - beta kbar kbar^T) S + beta kbar vbar^T.
-__global__ void __launch_bounds__(256) scan_delta_kernel(Dims d, const float *__restrict__ kbar,
-                                                         const float *__restrict__ vbar, const float *__restrict__ St,
-                                                         const float *__restrict__ beta, float *__restrict__ Sf,
-                                                         float *__restrict__ Sb, const int32_t *__restrict__ gtab,
-                                                         int G) {
+// Delta-rule scan.  The update S <- (I - beta kbar kbar^T) S + beta kbar vbar^T acts on each
+// column of S separately (u_j = kbar . S[:, j]; S[:, j] += beta kbar (vbar_j - u_j)), so a
+// block owns DCB columns of one head's state in one direction, walks the frames in order and
+// emits its slice of every group's memory when the walk reaches the group's boundary.  The
+// frame means of the head and the block's value columns are staged in shared memory first;
+// each thread keeps 8 state entries (one column, 8 rows) in registers, and a step needs one
+// block barrier (the column sums u are reduced through a parity-double-buffered array).
+constexpr int DCB = 16;            // state columns per block
+constexpr int DELTA_THREADS = 256;
+
+template <int D>
+__global__ void __launch_bounds__(DELTA_THREADS) scan_delta_kernel(Dims d, const float *__restrict__ kbar,
+                                                                   const float *__restrict__ vbar,
+                                                                   const float *__restrict__ St,
+                                                                   const float *__restrict__ beta,
+                                                                   float *__restrict__ Sf, float *__restrict__ Sb,
+                                                                   const int32_t *__restrict__ gtab, int G) {
+  constexpr int RPT = D / (2 * DELTA_THREADS / 32);  // rows per thread: 16 row groups of 8 (D = 128)
+  static_assert(RPT * 2 * (DELTA_THREADS / 32) == D, "row split");
+  extern __shared__ float sm[];
+  const int h = blockIdx.x, dir = blockIdx.y, j0 = blockIdx.z * DCB;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int col = lane & 15;                       // column j0 + col
+  const int rg = (lane >> 4) + 2 * warp;           // row group: rows rg * RPT .. + RPT - 1
+  const int F = d.F;
+  float *kb = sm;                                  // [F][D]
+  float *vb = kb + (size_t)F * D;                  // [F][DCB]
+  float *bt = vb + (size_t)F * DCB;                // [F]
+  float *part = bt + F;                            // [2][8 warps][DCB]
+  int *bound = reinterpret_cast<int *>(part + 2 * (DELTA_THREADS / 32) * DCB);  // [G]
+  int *any = bound + G;                            // [F]: some group's memory ends at this frame
+  for (int e = tid; e < F * D; e += DELTA_THREADS) kb[e] = kbar[((int64_t)(e / D) * d.H + h) * D + e % D];
+  for (int e = tid; e < F * DCB; e += DELTA_THREADS)
+    vb[e] = vbar[((int64_t)(e / DCB) * d.H + h) * D + j0 + e % DCB];
+  for (int e = tid; e < F; e += DELTA_THREADS) bt[e] = beta[(int64_t)e * d.H + h];
+  for (int e = tid; e < F; e += DELTA_THREADS) any[e] = 0;
+  __syncthreads();
+  for (int g = tid; g < G; g += DELTA_THREADS) {
+    const int32_t *r = gtab + g * 16;
+    const int b = dir == 0 ? (r[13] > r[12] ? r[13] : 1) : (r[15] > r[14] ? r[14] : F - 1);
+    bound[g] = b;
+    any[b] = 1;
+  }
+  float sreg[RPT];
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) sreg[m] = 0.5f * St[((int64_t)h * D + rg * RPT + m) * D + j0 + col];
+  __syncthreads();
+  float *dst = dir == 0 ? Sf : Sb;
+  auto emit = [&](int f) {
+    if (f < F && !any[f]) return;  // the forward walk ends at frame F-1 (frame 1 when F = 1)
+    for (int g = 0; g < G; ++g)
+      if (bound[g] == f) {
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) dst[(((int64_t)g * d.H + h) * D + rg * RPT + m) * D + j0 + col] = sreg[m];
+      }
+  };
+  int par = 0;
+  auto step = [&](int f) {
+    const float *k = kb + (size_t)f * D + rg * RPT;
+    float u = 0.f;
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) u = fmaf(k[m], sreg[m], u);
+    u += __shfl_xor_sync(0xffffffffu, u, 16);      // the two row groups of this warp
+    float *pp = part + par * (DELTA_THREADS / 32) * DCB;
+    if (lane < 16) pp[warp * DCB + col] = u;
+    __syncthreads();
+    float uj = 0.f;
+#pragma unroll
+    for (int w = 0; w < DELTA_THREADS / 32; ++w) uj += pp[w * DCB + col];
+    const float c = bt[f] * (vb[(size_t)f * DCB + col] - uj);
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) sreg[m] = fmaf(k[m], c, sreg[m]);
+    par ^= 1;
+  };
+  if (dir == 0) {
+    for (int f = 1;; ++f) {
+      emit(f);
+      if (f > F - 2) break;
+      step(f);
+    }
+  } else {
+    for (int f = F - 1;; --f) {
+      emit(f);
+      if (f - 1 < 1) break;
+      step(f - 1);
+    }
+  }
+}
+
+// Fallback for head dims without the column split: one block per (head, direction), the
+// whole D x D state in shared memory.
+__global__ void __launch_bounds__(256) scan_delta_small_kernel(Dims d, const float *__restrict__ kbar,
+                                                               const float *__restrict__ vbar,
+                                                               const float *__restrict__ St,
+                                                               const float *__restrict__ beta, float *__restrict__ Sf,
+                                                               float *__restrict__ Sb,
+                                                               const int32_t *__restrict__ gtab, int G) {
   extern __shared__ float sm[];
   const int D = d.D, h = blockIdx.x, dir = blockIdx.y, tid = threadIdx.x;
   const int DD = D * D;
@@ -492,10 +637,21 @@ cudaError_t launch_state_scan(const Dims &d, vdn_lin_kind kind, const float *S, 
     scan_elu1_kernel<<<grid, 256, 0, st>>>(d, S, z, St, zt, Sf, Sb, zf, zb, gtab, G);
     return cudaGetLastError();
   }
+  // column-split recurrence for D = 128 while the frame means fit in shared memory
+  const size_t smem_cols = ((size_t)d.F * (d.D + DCB + 1) + 2 * (DELTA_THREADS / 32) * DCB) * sizeof(float) +
+                           ((size_t)max_groups(d.F, d.C) + d.F) * sizeof(int);
+  if (d.D == 128 && smem_cols <= 200 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(scan_delta_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_cols);
+    if (e != cudaSuccess) return e;
+    scan_delta_kernel<128><<<dim3(d.H, 2, 128 / DCB), DELTA_THREADS, smem_cols, st>>>(d, S, z, St, beta, Sf, Sb, gtab,
+                                                                                      G);
+    return cudaGetLastError();
+  }
   size_t smem = ((size_t)d.D * d.D + 3 * d.D) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(scan_delta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(scan_delta_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  scan_delta_kernel<<<dim3(d.H, 2), 256, smem, st>>>(d, S, z, St, beta, Sf, Sb, gtab, G);
+  scan_delta_small_kernel<<<dim3(d.H, 2), 256, smem, st>>>(d, S, z, St, beta, Sf, Sb, gtab, G);
   return cudaGetLastError();
 }
 

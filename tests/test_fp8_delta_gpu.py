@@ -120,9 +120,10 @@ def test_delta_layer_bf16_softmax():
     assert_close("y", yr, ref["y"], "bf16")
 
 
-def test_delta_step_entry_points():
-    s = synth.Shape(17, 50, 3, 6, 2, 64)
-    F, T, C, L, H, D = 17, 50, 3, 6, 2, 64
+@pytest.mark.parametrize("D", [64, 128])   # 128: the column-split recurrence and vectorised frame means
+def test_delta_step_entry_points(D):
+    F, T, C, L, H = 17, 50, 3, 6, 2
+    s = synth.Shape(F, T, C, L, H, D)
     inp = synth.make_inputs(s, "bf16", seed=22, with_beta=True)
     d = {n: to_device(a) for n, a in inp.items()}
     o = oracle_inputs(inp)
