@@ -65,6 +65,61 @@ def layer_flops(shape: synth.Shape) -> dict:
     }
 
 
+def kernel_work(shape: synth.Shape, linear: str, fp8: bool) -> dict:
+    """Algorithmic work of each library kernel per layer call: ("tensor", FLOP) for the
+    contractions, ("hbm", bytes that must cross HBM) for the memory-bound steps."""
+    import hybrid_softmax_linear_b200 as vdn
+    Nv, H, D = shape.n_video, shape.heads, shape.head_dim
+    F, L = shape.frames, shape.text_tokens
+    G = len(vdn.mask_layout_build(shape)[1])
+    HD = H * D
+    act = 2  # bf16 activations
+    fl = layer_flops(shape)
+    work = {
+        "softmax_tc": ("tensor", fl["softmax"]),
+        "out_proj_tc": ("tensor", fl["out_proj"]),
+        # q in, the linear half of A out
+        "read_tc": ("hbm", 2.0 * Nv * HD * act),
+    }
+    if linear == "elu1":
+        # k, v and text in; per-frame S, z and the text state out
+        work["state_build_tc"] = ("hbm", 2.0 * (Nv + L) * HD * act + (F + 1) * H * (D * D + D) * 4.0)
+        # per-frame states in; bf16 S_fwd + S_bwd and float z_fwd + z_bwd per group out
+        work["scan"] = ("hbm", (F + 1) * H * (D * D + D) * 4.0 + G * H * (D * D * 2.0 + D * 4.0))
+    else:
+        # k, v in (frame means out, negligible); the recurrence writes both memories per group
+        work["state_build"] = ("hbm", 2.0 * (Nv + L) * HD * act)
+        work["scan"] = ("hbm", 2.0 * G * H * D * D * 4.0)
+    if fp8:
+        # q, k, v (and text) read once, e4m3 copies written once
+        work["fp8_quant"] = ("hbm", 3.0 * Nv * HD * (act + 1) + 2.0 * L * HD * (act + 1))
+    return work
+
+
+def kernel_rooflines(prof: dict, steps: int, shape, linear: str, fp8: bool, peaks: dict, fp8_ratio: float) -> dict:
+    """Per kernel: live ms per call, achieved TFLOP/s or GB/s, and its fractions of the
+    measured burst and sustained tensor peaks (the e4m3 softmax: times the e4m3/bf16 ratio)
+    or of the measured HBM bandwidth."""
+    out = {}
+    work = kernel_work(shape, linear, fp8)
+    for name, (ms_total, n) in prof.items():
+        if name not in work or n == 0:
+            continue
+        ms = ms_total / n
+        kind, amount = work[name]
+        if kind == "tensor":
+            tf = amount / (ms / 1e3) / 1e12
+            scale = fp8_ratio if (fp8 and name == "softmax_tc") else 1.0
+            out[name] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                         "frac_of_burst": round(tf / (peaks["bf16_tflops"] * scale), 3),
+                         "frac_of_sustained": round(tf / (peaks["bf16_tflops_sustained"] * scale), 3)}
+        else:
+            gbs = amount / (ms / 1e3) / 1e9
+            out[name] = {"ms": round(ms, 4), "gb_per_s": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3),
+                         "algorithmic_gb": round(amount / 1e9, 4)}
+    return out
+
+
 def load_peaks() -> tuple[dict, str]:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -473,10 +528,12 @@ def run_ours(args, rank, world, local_rank):
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_note = f"{peak_src} bf16_tflops_sustained (kernel runs inside a long step)"
     fp8_burst = fp8_peak(dev) if w.softmax_fp8 else None
+    fp8_ratio = 1.0
     if w.softmax_fp8:
         # e4m3 contraction: the measured bf16 sustained peak times the measured fp8/bf16 burst
         # ratio (nominal 2 when the e4m3 GEMM could not be timed)
         ratio = (fp8_burst / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) if fp8_burst else 2.0
+        fp8_ratio = ratio
         peak *= ratio
         peak_note = (f"{peak_src} bf16_tflops_sustained x {ratio:.3f} (fp8/bf16 burst ratio"
                      f"{', measured with torch._scaled_mm e4m3 8192^3' if fp8_burst else ', nominal'}; "
@@ -494,6 +551,8 @@ def run_ours(args, rank, world, local_rank):
                      "algorithmic_tflop_per_launch": fl["softmax"] / 1e12, "avg_launch_ms": sm_avg},
         "layer_tflops": sum(v for k, v in fl.items()) / (per_step_ms / 1e3) / 1e12,
         "per_kernel_ms_per_step": {k: round(v[0] / max(args.steps, 1), 4) for k, v in prof.items()},
+        "kernels": kernel_rooflines(prof, args.steps, s, w.linear, w.softmax_fp8, dict(FALLBACK_PEAKS) | peaks,
+                                    fp8_ratio),
         "gpu_launches": launches,
         "e2e": {"value": whole_job_value(world, s.n_video, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,

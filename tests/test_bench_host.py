@@ -79,3 +79,21 @@ def test_captured_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     src.write_text("changed\n")
     assert bench.captured_traffic(shape, fp8=False)[0] is None
 
+
+
+def test_kernel_rooflines_use_the_algorithmic_work():
+    """Per-kernel rates divide the stated algorithmic work by the live time per call."""
+    shape = synth.CONFIGS[2].shape
+    work = bench.kernel_work(shape, "elu1", fp8=False)
+    Nv, HD = shape.n_video, shape.heads * shape.head_dim
+    assert work["read_tc"] == ("hbm", 2.0 * Nv * HD * 2)
+    assert work["softmax_tc"] == ("tensor", bench.softmax_flops(shape))
+    peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 800.0, "hbm_gbs": 5000.0}
+    prof = {"read_tc": (2.0, 4), "softmax_tc": (10.0, 2), "tables": (0.1, 2)}
+    k = bench.kernel_rooflines(prof, 2, shape, "elu1", False, peaks, 1.0)
+    assert set(k) == {"read_tc", "softmax_tc"}                 # no work figure for the tables
+    gbs = work["read_tc"][1] / 0.5e-3 / 1e9
+    assert abs(k["read_tc"]["gb_per_s"] - round(gbs, 1)) < 0.11
+    tf = work["softmax_tc"][1] / 5e-3 / 1e12
+    assert abs(k["softmax_tc"]["frac_of_sustained"] - round(tf / 800.0, 3)) < 1e-3
+    assert "fp8_quant" in bench.kernel_work(shape, "delta", fp8=True)

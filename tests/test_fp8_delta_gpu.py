@@ -159,3 +159,15 @@ def test_config5_full_size_fp8_delta_sampled():
     assert_close("A_l (delta, bf16)", A[:, HD:], ref["a"][:, HD:], "bf16")
     assert rel_l2(yr, ref["y"]) <= FP8_TOL
     assert np.all(np.isfinite(yr))
+
+
+@pytest.mark.parametrize("shape", [(1, 70, 5, 3, 2, 128),    # one frame (both anchors)
+                                   (2, 40, 5, 0, 1, 128),    # two anchors, no text
+                                   (87, 20, 5, 8, 2, 128)])  # ragged last chunk
+def test_delta_layer_edge_shapes(shape):
+    s = synth.Shape(*shape)
+    inp = synth.make_inputs(s, "bf16", seed=31 + shape[0], with_beta=True)
+    run = Run(s, inp, "bf16", kind=vdn.DELTA)
+    A, yr, ref, HD = _layer(run, np.arange(s.n_video))
+    assert_close("A_l (delta)", A[:, HD:], ref["a"][:, HD:], "bf16")
+    assert_close("y", yr, ref["y"], "bf16")
