@@ -8,13 +8,15 @@
 //   phi = elu+1 in place in shared memory (masking tokens past the frame) and sum z;
 //   one thread issues tcgen05.mma with both operands MN-major (M = key feature, N =
 //   value dim, K = tokens) into a 128x128 fp32 accumulator in tensor memory.
-// read_stage: S_fwd + S_bwd of every group summed into bf16 (the MMA B operand), the
-//   normalisers summed, the linear-gate weights converted to bf16.
-// read_tc: 256 query rows of one group and head per CTA (two 128-row halves).  Four
-//   warps per half write phi(q) (or q/|q| for the delta rule) next to q in shared memory
-//   and the normaliser phi(q).z; one thread issues num = phi(Q) S_sum and, for the fused
-//   layer, the gate logits Q W_l; the same warps then form o = num / den and either
-//   store o or the gated, RMS-normalised A_l straight into the linear half of A.
+// read_stage: the linear-gate weights converted to bf16 and, where the scan left fp32
+//   memories (step entry points, delta rule), S_fwd + S_bwd of every group summed into
+//   bf16 (the MMA B operand) and the normalisers summed.
+// read_tc: 128 query rows of one group and head per CTA, two CTAs per SM.  Two threads per
+//   row (one per column half) build phi(q) (or q/|q| for the delta rule) and the
+//   normaliser phi(q).z while thread 0's MMA forms the gate logits Q W_l, write the
+//   features over Q, and after num = phi(Q) S_sum form o = num / den and store o or the
+//   gated, RMS-normalised A_l (staged in shared memory, whole rows per store) into the
+//   linear half of A.
 #include "tc_common.cuh"
 
 namespace vdn {
