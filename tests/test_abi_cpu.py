@@ -117,3 +117,27 @@ def test_argument_checks_precede_cuda():
     st = L.vdn_hybrid_attn_fwd(ctypes.byref(s), 7, vdn.F32, 16, 16, 16, 16, 16, None, 16, 16, 32, 16, 1e-6, 16, 16,
                                16, 256, 1 << 30, None)
     assert st == 1  # unknown kind
+
+
+def test_host_entry_point_checks_and_sizes():
+    """The host-buffer layer: its workspace adds the staging area; missing host tensors and a
+    short workspace are reported before any device work."""
+    s = synth.Shape(90, 1008, 5, 512, 40, 128)
+    nv, hd = 90 * 1008, 40 * 128
+    full = vdn.hybrid_attn_workspace_size(s, vdn.ELU1, vdn.BF16)
+    host = vdn.hybrid_attn_host_workspace_size(s, vdn.ELU1, vdn.BF16)
+    # q, k, v, y (bf16) plus text k/v staged behind the layer's workspace
+    assert host >= full + 4 * nv * hd * 2 + 2 * 512 * hd * 2
+    assert vdn.hybrid_attn_host_workspace_size(s, vdn.DELTA, vdn.BF16) >= \
+        vdn.hybrid_attn_workspace_size(s, vdn.DELTA, vdn.BF16) + 4 * nv * hd * 2 + 90 * 40 * 4
+    t = vdn.Shape(15, 16, 1, 4, 2, 32)
+    L = vdn.lib()
+    args = [ctypes.byref(t), vdn.ELU1, vdn.F32, 16, 16, 16, 16, 16, None, 16, 16, 32, 16, 1e-6, 16, 16, 16, 256]
+    big = vdn.hybrid_attn_host_workspace_size(t, vdn.ELU1, vdn.F32)
+    a = list(args); a[3] = None
+    assert L.vdn_hybrid_attn_fwd_host(*a, big, None) == 1 and b"host" in L.vdn_last_error()
+    a = list(args); a[6] = None                                    # text k with L > 0
+    assert L.vdn_hybrid_attn_fwd_host(*a, big, None) == 1
+    assert L.vdn_hybrid_attn_fwd_host(*args, big - 256, None) == 3   # workspace too small
+    a = list(args); a[1] = vdn.DELTA                               # the delta rule needs beta
+    assert L.vdn_hybrid_attn_fwd_host(*a, vdn.hybrid_attn_host_workspace_size(t, vdn.DELTA, vdn.F32), None) == 1
