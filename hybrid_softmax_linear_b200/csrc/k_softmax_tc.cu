@@ -7,8 +7,9 @@
 // that share every K/V tile.  Warp 0 streams Q once and the group's K/V tiles (128 keys,
 // text first, then the merged video segments) with TMA into 2-stage rings.  One thread
 // of warp 1 issues tcgen05.mma: S_w = Q_w K_j^T (M=128, N=128) into tensor memory, then,
-// once softmax warpgroup w has written P_w (bf16, over S_w's columns) and rescaled its
-// output, O_w += P_w V_j (A operand from tensor memory, V as an MN-major operand).
+// once softmax warpgroup w has rescaled its output and written P_w (bf16 or e4m3, over
+// S_w's columns; e4m3 in two pieces of 64 keys, each handed over as soon as it is
+// written), O_w += P_w V_j (A operand from tensor memory, V as an MN-major operand).
 // Warpgroups 0 and 1 (warps 2-5 and 6-9) run the online softmax of Q0 and Q1, one row
 // per thread, so while one warpgroup exponentiates, the tensor cores work for the
 // other.  The running maximum is only moved (and O rescaled) when it grows by more than
@@ -32,6 +33,8 @@ constexpr int KST = 2, VST = 2;
 constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+// P of a tile is handed to the tensor cores in up to MAX_P_PARTS pieces (Cfg::P_PARTS)
+constexpr int MAX_P_PARTS = 2;
 
 // FP8 = false: bf16 Q/K/V and P (kind::f16, K = 16 per MMA).  FP8 = true: e4m3 Q/K/V
 // with per-head scales and e4m3 P at unit scale (kind::f8f6f4, K = 32 per MMA).  A
@@ -51,13 +54,20 @@ struct Cfg {
   static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
   static constexpr uint32_t IDESC_S = FP8 ? idesc_e4m3(BM, BN, false, false) : idesc_bf16(BM, BN, false, false);
   static constexpr uint32_t IDESC_O = FP8 ? idesc_e4m3(BM, D, false, true) : idesc_bf16(BM, D, false, true);
+  // e4m3: P goes to the tensor cores in two pieces of 64 keys, so the P.V MMA of the first
+  // overlaps the exponentials of the second (5% faster, measured).  bf16: in one piece; its
+  // P.V takes twice as long and a wait in its middle holds up the single MMA issuer (2%
+  // slower in two pieces, 8% in four).
+  static constexpr int P_PARTS = FP8 ? 2 : 1;
+  static_assert(P_PARTS <= MAX_P_PARTS && (P_PARTS == 1 || P_PARTS == 2 || P_PARTS == 4), "P is written in 32-key chunks");
   // tensor memory columns: S_0, S_1, O_0, O_1
   __device__ static constexpr uint32_t s_col(int w) { return (uint32_t)w * 128u; }
   __device__ static constexpr uint32_t o_col(int w) { return 256u + (uint32_t)w * 128u; }
 };
 
 struct alignas(8) Bars {
-  uint64_t q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[NQ], p_full[NQ], o_done, drain;
+  uint64_t q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[NQ], p_ready[NQ][MAX_P_PARTS], o_done,
+      drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -170,7 +180,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(smem_u32(&bars->q_full), 1);
     for (int s = 0; s < KST; ++s) { mbar_init(smem_u32(&bars->k_full[s]), 1); mbar_init(smem_u32(&bars->k_empty[s]), 1); }
     for (int s = 0; s < VST; ++s) { mbar_init(smem_u32(&bars->v_full[s]), 1); mbar_init(smem_u32(&bars->v_empty[s]), 1); }
-    for (int w = 0; w < NQ; ++w) { mbar_init(smem_u32(&bars->s_full[w]), 1); mbar_init(smem_u32(&bars->p_full[w]), 4); }
+    for (int w = 0; w < NQ; ++w) {
+      mbar_init(smem_u32(&bars->s_full[w]), 1);
+      for (int i = 0; i < C::P_PARTS; ++i) mbar_init(smem_u32(&bars->p_ready[w][i]), 4);
+    }
     mbar_init(smem_u32(&bars->o_done), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
@@ -271,22 +284,33 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t vbase = smem_u32(base + C::V_OFF + vs * C::TILE_BYTES);
         for (int w = 0; w < NQ && ok; ++w) {
           // each wait sits right before the first MMA that needs it
-          if (!mbar_wait(smem_u32(&bars->p_full[w]), j & 1, abort_flag, st, K_SOFTMAX_TC, 7)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&bars->p_ready[w][0]), j & 1, abort_flag, st, K_SOFTMAX_TC, 7)) { ok = false; break; }
           if (w == 0 && !mbar_wait(smem_u32(&bars->v_full[vs]), (j / VST) & 1, abort_flag, st, K_SOFTMAX_TC, 5)) {
             ok = false;
             break;
           }
           tc_fence_after();
           // O_w += P_w V_j: P_w (two bf16 or four e4m3 per column) sits over the first columns
-          // of S_w; each K-step takes 8 of those columns and KSTEP rows of V (128 bytes each)
+          // of S_w; each K-step takes 8 of those columns and KSTEP rows of V (128 bytes each).
+          // Each piece of P goes as soon as it is written, while the softmax warps still
+          // exponentiate the next.
+          constexpr int KSTEPS = BN / C::KSTEP, KPART = KSTEPS / C::P_PARTS;
 #pragma unroll
-          for (int kk = 0; kk < BN / C::KSTEP; ++kk) {
+          for (int kk = 0; kk < KSTEPS; ++kk) {
+            if (kk > 0 && kk % KPART == 0) {
+              if (!mbar_wait(smem_u32(&bars->p_ready[w][kk / KPART]), j & 1, abort_flag, st, K_SOFTMAX_TC, 15)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
             const uint64_t bdesc = sdesc(vbase + kk * (C::KSTEP * 128), BM * 128, 1024);
             if (FP8)
               mma_ts_f8(tmem + C::o_col(w), tmem + C::s_col(w) + kk * 8, bdesc, C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
             else
               mma_ts(tmem + C::o_col(w), tmem + C::s_col(w) + kk * 8, bdesc, C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
           }
+          if (!ok) break;
           if (j == 0 && w == 0) {
             issue_s(1, 0);                               // staggered start of Q tile 1
             mma_commit(smem_u32(&bars->k_empty[0]));     // K tile 0 is free once both S of it complete
@@ -368,6 +392,29 @@ __global__ void __launch_bounds__(THREADS, 1)
         alpha = ex2(m - m_new);   // 0 on the first tile (m = -inf)
         m = m_new;
       }
+      if (need && j > 0) {
+        // O_w was last written by P V of tile j-1, which completed before S_w of tile j; it
+        // is rescaled before any P of tile j is handed to the tensor cores
+#pragma unroll 1
+        for (int c = 0; c < D; c += 8) {  // 8 columns at a time: the row of S is still live
+          uint32_t u[8];
+          tmem_ld8(o_addr + c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          tmem_st8(o_addr + c, u);
+        }
+      }
+      // P of keys [0, c + 32) (and the rescaled O) handed to the MMA thread at the end of
+      // each piece
+      auto hand_piece = [&](int c) {
+        if ((c + 32) % (BN / C::P_PARTS) == 0) {
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[w][(c + 32) / (BN / C::P_PARTS) - 1]));
+        }
+      };
       float rs8[8];               // row sum in eight independent chains
 #pragma unroll
       for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
@@ -390,6 +437,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             pk[i] = (lo & 0xffffu) | (hi << 16);
           }
           tmem_st8(s_addr + (c >> 2), pk);
+          hand_piece(c);
         }
       } else {
 #pragma unroll
@@ -404,26 +452,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             pk[i] = pack_bf16(p0, p1);
           }
           tmem_st16(s_addr + (c >> 1), pk);
-        }
-      }
-      if (need && j > 0) {
-        // O_w was last written by P V of tile j-1, which completed before S_w of tile j
-#pragma unroll 1
-        for (int c = 0; c < D; c += 16) {
-          uint32_t u[16];
-          tmem_ld16(o_addr + c, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st16(o_addr + c, u);
+          hand_piece(c);
         }
       }
       const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l = l * alpha + rs;
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[w]));
     }
     // ------------------------------------------------------------ epilogue
     const bool done = ok && mbar_wait(smem_u32(&bars->o_done), 0, abort_flag, st, K_SOFTMAX_TC, 13);
