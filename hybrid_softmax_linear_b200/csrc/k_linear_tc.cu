@@ -64,7 +64,7 @@ struct alignas(8) Bars {
   uint64_t full[NS], phi[NS], empty[NS], acc, drain;
   uint32_t tmem;
   int abort;
-  float zred[D];
+  float zpart[PHI_WARPS][D];  // z of each phi warp, summed in a fixed order (repeatable bits)
 };
 constexpr size_t SMEM = 1024 + NS * STAGE_BYTES + sizeof(Bars);
 }  // namespace sb
@@ -104,7 +104,6 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x < D) bars->zred[threadIdx.x] = 0.f;
   if (warp == 1) { tmem_alloc(smem_u32(&bars->tmem), 128); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -184,8 +183,13 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->phi[s]));
     }
+    // lanes l and l ^ 16 hold the same columns: pair them, then one row per warp
 #pragma unroll
-    for (int e = 0; e < 8; ++e) atomicAdd(&bars->zred[cl * 8 + e], zacc[e]);
+    for (int e = 0; e < 8; ++e) zacc[e] += __shfl_xor_sync(0xffffffffu, zacc[e], 16);
+    if (lane < 16) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) bars->zpart[warp - 2][cl * 8 + e] = zacc[e];
+    }
     const int quad = warp & 3, c_lo = ((warp - 2) >> 2) * (D / 2);  // lane quarter; column half
     const int i = quad * 32 + lane;  // key feature = accumulator row = tensor-memory lane
     float *So = text ? St + (int64_t)h * D * D : S + ((int64_t)fr * d.H + h) * D * D;
@@ -210,10 +214,14 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
     } else {
       for (int cc = 0; cc < D / 2; ++cc) So[i * D + c_lo + cc] = 0.f;
     }
-    named_bar_sync(1, 32 * PHI_WARPS);  // every phi thread has added its share of z
+    named_bar_sync(1, 32 * PHI_WARPS);  // every phi warp has written its share of z
     float *zo = text ? zt : z;
-    if (zo != nullptr && tid < D)
-      zo[(text ? (int64_t)h * D : ((int64_t)fr * d.H + h) * D) + tid] = bars->zred[tid];
+    if (zo != nullptr && tid < D) {
+      float zs = 0.f;
+#pragma unroll
+      for (int pw = 0; pw < PHI_WARPS; ++pw) zs += bars->zpart[pw][tid];
+      zo[(text ? (int64_t)h * D : ((int64_t)fr * d.H + h) * D) + tid] = zs;
+    }
   }
   tc_fence_before();
   __syncthreads();
