@@ -141,3 +141,40 @@ def test_host_entry_point_checks_and_sizes():
     assert L.vdn_hybrid_attn_fwd_host(*args, big - 256, None) == 3   # workspace too small
     a = list(args); a[1] = vdn.DELTA                               # the delta rule needs beta
     assert L.vdn_hybrid_attn_fwd_host(*a, vdn.hybrid_attn_host_workspace_size(t, vdn.DELTA, vdn.F32), None) == 1
+
+
+@pytest.mark.parametrize("shape,kind,cdt,states", [
+    ((90, 1008, 5, 512, 40, 128), vdn.ELU1, vdn.BF16, False),   # segmented scan: bf16 sum only
+    ((90, 1008, 5, 512, 40, 128), vdn.DELTA, vdn.E4M3, True),
+    ((12, 300, 5, 40, 2, 128), vdn.ELU1, vdn.F32, True),         # CUDA-core path: O_s, O_l too
+    ((130, 4, 1, 3, 1, 128), vdn.ELU1, vdn.BF16, True),          # 127 segments: per-group states
+    ((15, 16, 1, 4, 2, 64), vdn.DELTA, vdn.BF16, True),
+])
+def test_workspace_regions_disjoint_aligned_in_bounds(shape, kind, cdt, states):
+    """The intermediates the layer exposes sit inside its workspace, 256-byte aligned, and
+    do not overlap (pointer arithmetic only: a fake base address, no device)."""
+    s = synth.Shape(*shape)
+    F, T, C, L, H, D = shape
+    base = 1 << 40
+    total = vdn.hybrid_attn_workspace_size(s, kind, cdt)
+    G = vdn.max_groups(s)
+    act = 4 if cdt == vdn.F32 else 2
+    nv = F * T
+    sizes = {0: nv * H * D * act, 1: nv * H * D * act, 2: nv * 2 * H * D * act, 3: G * H * D * D * 4,
+             4: G * H * D * D * 4, 5: F * 8 * 4, 6: G * 16 * 4, 7: 8 * 4, 8: 2 * 4, 9: (4 + F + 1 + 2 * G) * 4}
+    regions = []
+    for which, n in sizes.items():
+        p = vdn.hybrid_attn_intermediate(s, kind, cdt, base, which)
+        if p == 0:
+            continue
+        assert (p - base) % 256 == 0, which
+        assert base <= p and p + n <= base + total, which
+        regions.append((p, p + n, which))
+    regions.sort()
+    for (_, a1, wa), (b0, _, wb) in zip(regions, regions[1:]):
+        assert a1 <= b0, (wa, wb)
+    fused = cdt in (vdn.BF16, vdn.E4M3) and D == 128
+    assert (vdn.hybrid_attn_intermediate(s, kind, cdt, base, 0) == 0) == fused
+    assert (vdn.hybrid_attn_intermediate(s, kind, cdt, base, 3) != 0) == states
+    assert vdn.hybrid_attn_intermediate(s, kind, cdt, base, 10) == 0
+    assert vdn.hybrid_attn_intermediate(s, kind, cdt, None, 2) == 0
