@@ -5,7 +5,9 @@ kernels; torch is used for device memory and streams.
 The functions carry the C entry points' names without the ``vdn_`` prefix and accept
 torch tensors (their ``data_ptr()`` is passed) or raw integer device pointers.  A
 non-zero status raises :class:`VdnError` with the library's message.  If libvdn.so is
-missing, :func:`lib` raises: there is no fallback path.
+missing, :func:`lib` raises: there is no fallback path.  The whole-layer calls check each
+torch tensor's element count, element size, contiguity and placement first and raise
+ValueError on a mismatch.
 """
 from __future__ import annotations
 
@@ -209,8 +211,52 @@ def out_proj(shape, dtype, a, w_os, w_ol, y, ws, stream=None):
                               _nbytes(ws), _stream(stream)))
 
 
+def _need(name: str, t, numel: int, esize: int, where: str | None):
+    """Checks a torch tensor argument of the whole-layer calls before its pointer is passed:
+    the library sees only addresses, so a short or strided buffer would be read or written
+    out of bounds.  Raw integer pointers and None go through unchecked (the library checks
+    for NULL).  where: "device", "host" or None (no placement check)."""
+    if t is None or isinstance(t, int):
+        return
+    if where == "device" and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if where == "host" and t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.element_size() != esize:
+        raise ValueError(f"{name}: {esize}-byte elements expected, got {t.dtype}")
+    if t.numel() != numel:
+        raise ValueError(f"{name}: {numel} elements expected, got {t.numel()}")
+
+
+def _check_layer_args(shape, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma, w_os, w_ol, y,
+                      io: str | None, weights: str | None):
+    """Element counts and sizes of the layer's tensors (vdn.h, whole layer): q, k, v, y
+    [N_v][H][D], kt, vt [L][H][D] and w_os, w_ol [HD][HD] in float (VDN_F32) or bf16; beta
+    float[F][H]; w_gate_s, gamma float[H][D]; w_gate_l float[H][D][G_l].  io places the
+    per-call tensors, weights the weights."""
+    s = Shape.of(shape)
+    nv, hd = s.frames * s.tokens_per_frame, s.heads * s.head_dim
+    act = 4 if dtype == F32 else 2
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(name, t, nv * hd, act, io)
+    for name, t in (("kt", kt), ("vt", vt)):
+        _need(name, t, s.text_tokens * hd, act, io)
+    _need("beta", beta, s.frames * s.heads, 4, io)
+    _need("y", y, nv * hd, act, io)
+    _need("w_gate_s", w_gate_s, hd, 4, weights)
+    if isinstance(G_l, int) and G_l > 0:
+        _need("w_gate_l", w_gate_l, hd * G_l, 4, weights)
+    _need("gamma", gamma, hd, 4, weights)
+    _need("w_os", w_os, hd * hd, act, weights)
+    _need("w_ol", w_ol, hd * hd, act, weights)
+
+
 def hybrid_attn_fwd(shape, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma, eps, w_os, w_ol, y,
                     ws, stream=None):
+    _check_layer_args(shape, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma, w_os, w_ol, y,
+                      "device", "device")
     _check(lib().vdn_hybrid_attn_fwd(ctypes.byref(Shape.of(shape)), kind, dtype, _p(q), _p(k), _p(v), _p(kt),
                                      _p(vt), _p(beta), _p(w_gate_s), _p(w_gate_l), G_l, _p(gamma), eps, _p(w_os),
                                      _p(w_ol), _p(y), _p(ws), _nbytes(ws), _stream(stream)))
@@ -224,6 +270,8 @@ def hybrid_attn_fwd_host(shape, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_
                          w_ol, y, ws, stream=None):
     """The layer with q, k, v, kt, vt, beta and y in (page-locked) host memory; weights on
     the device.  Asynchronous on `stream`: y is complete when the stream is."""
+    _check_layer_args(shape, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma, w_os, w_ol, y,
+                      "host", "device")
     _check(lib().vdn_hybrid_attn_fwd_host(ctypes.byref(Shape.of(shape)), kind, dtype, _p(q), _p(k), _p(v), _p(kt),
                                           _p(vt), _p(beta), _p(w_gate_s), _p(w_gate_l), G_l, _p(gamma), eps,
                                           _p(w_os), _p(w_ol), _p(y), _p(ws), _nbytes(ws), _stream(stream)))
