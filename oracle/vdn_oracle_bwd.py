@@ -1,5 +1,6 @@
-"""Float64 CPU oracle of the VDN-H3 hybrid attention layer, backward pass (elu+1 linear
-branch): the gradients of a loss L(y) with respect to every input of the forward oracle.
+"""Float64 CPU oracle of the VDN-H3 hybrid attention layer, backward pass (elu+1 and
+delta-rule linear branches): the gradients of a loss L(y) with respect to every input of
+the forward oracle.
 
 TEST INFRASTRUCTURE, like the forward oracle in vdn_oracle.py: only the test suite may
 import it; the CUDA library shares no code with it.
@@ -16,6 +17,9 @@ same notation; the pages define only the forward ([ART] æŠ€æœ¯è§£è¯»: å±€éƒ¨ç²¾ç
   Num_f = S_txt + sum_{fk in FWD(f) u BWD(f)} S_fk,  Den_f likewise with z
           (the two text halves of the forward and backward memories add up to one, R5)
   S_fk  = sum_{t in fk} phi(k_t) v_t^T,  z_fk = sum_{t in fk} phi(k_t)
+  delta rule ([BLOG] III; R12, R13): O_l = (S_f + S_b)^T q_hat, each memory the recurrence
+          S <- S - beta kb (kb^T S) + beta kb vb^T over its frames from
+          S_0 = 1/2 sum_text k_hat v^T, with kb = normalised frame-mean key, vb = frame-mean value
 
 phi = elu + 1 has the continuous derivative phi'(x) = 1 for x > 0, e^x otherwise.
 The gradients are pinned against central finite differences of the forward oracle and,
@@ -166,15 +170,93 @@ def linear_branch_bwd(q, k, v, kt, vt, F, T, C, do_l):
     return dq, dk, dv, dkt, dvt
 
 
-def layer_bwd(inp: dict, dy, F, T, C, eps=1e-6, scale=None) -> dict:
-    """Gradients of sum(y * dy) for the whole layer over all video rows (elu+1 linear
-    branch), with respect to q, k, v, kt, vt, w_gate_s, w_gate_l, gamma, w_os, w_ol."""
+def l2_normalize_bwd(x, dy, axis=-1):
+    """y = x / ||x||  ->  dx = (dy - y (y . dy)) / ||x||; zero where x is zero (R13)."""
+    x = np.asarray(x, np.float64)
+    n = np.sqrt((x * x).sum(axis=axis, keepdims=True))
+    y = np.where(n > 0, x / np.where(n > 0, n, 1.0), 0.0)
+    g = dy - y * (y * dy).sum(axis=axis, keepdims=True)
+    return np.where(n > 0, g / np.where(n > 0, n, 1.0), 0.0)
+
+
+def delta_update_bwd(S, kb, vb, beta, dS1):
+    """Backward of one delta step S1 = S - beta kb (kb^T S) + beta kb vb^T (all heads):
+    dS = (I - beta kb kb^T) dS1 (the factor is symmetric);
+    dkb = -beta (dS1 S^T + S dS1^T) kb + beta dS1 vb;  dvb = beta dS1^T kb;
+    dbeta = kb^T dS1 (vb - S^T kb).  Shapes S, dS1 [H, D, D]; kb, vb [H, D]; beta [H]."""
+    H, D = kb.shape
+    b = np.asarray(beta, np.float64)
+    A = np.eye(D)[None] - b[:, None, None] * kb[:, :, None] * kb[:, None, :]
+    dS = np.matmul(A, dS1)
+    Stk = np.einsum("hde,hd->he", S, kb)                                  # S^T kb
+    dkb = (-b[:, None] * (np.einsum("hde,hfe,hf->hd", dS1, S, kb) + np.einsum("hde,hfe,hf->hd", S, dS1, kb))
+           + b[:, None] * np.einsum("hde,he->hd", dS1, vb))
+    dvb = b[:, None] * np.einsum("hde,hd->he", dS1, kb)
+    dbeta = np.einsum("hd,hde,he->h", kb, dS1, vb - Stk)
+    return dS, dkb, dvb, dbeta
+
+
+def delta_branch_bwd(q, k, v, kt, vt, beta, F, T, C, do_l):
+    """Backward of the delta-rule linear branch for all video query rows
+    (o = (S_f + S_b)^T q_hat, [BLOG] III; R12, R13).  The memory gradient of every distinct
+    frame sequence is summed over the query frames that read it and taken back through
+    its recurrence once, to the text init, the frame statistics and beta.
+    Returns dq, dk, dv [N, H, D], dkt, dvt [L, H, D], dbeta [F, H]."""
+    N, H, D = q.shape
+    L = kt.shape[0]
+    M = vo.frame_mask(F, C)
+    kb_raw = np.stack([np.asarray(k[f * T:(f + 1) * T], np.float64).mean(axis=0) for f in range(F)])
+    kb, vb = vo.delta_frame_stats(k, v, F, T)
+    S0 = vo.delta_text_init(kt, vt)
+    beta = np.asarray(beta, np.float64)
+    Sf, Sb = vo.delta_memory(k, v, kt, vt, beta, F, T, C)
+    dq = np.zeros((N, H, D))
+    dmem = {}                                                            # frame sequence -> dS
+    for f in range(F):
+        rows = np.arange(f * T, (f + 1) * T)
+        qr = np.asarray(q[rows], np.float64)
+        qh = vo.l2_normalize(qr)
+        dO = np.asarray(do_l[rows], np.float64)
+        dq[rows] = l2_normalize_bwd(qr, np.einsum("hde,nhe->nhd", Sf[f] + Sb[f], dO))
+        dS = np.einsum("nhd,nhe->hde", qh, dO)
+        for frames in (np.nonzero(M[f] == vo.FWD)[0], np.nonzero(M[f] == vo.BWD)[0][::-1]):
+            key = tuple(frames.tolist())
+            dmem[key] = dmem.get(key, 0.0) + dS
+    dS0 = np.zeros((H, D, D)); dkb = np.zeros((F, H, D)); dvb = np.zeros((F, H, D)); dbeta = np.zeros((F, H))
+    for key, dS in dmem.items():
+        states = [S0]
+        for f in key:
+            states.append(vo.delta_update(states[-1], kb[f], vb[f], beta[f]))
+        for i in range(len(key) - 1, -1, -1):
+            f = key[i]
+            dS, gk, gv, gb = delta_update_bwd(states[i], kb[f], vb[f], beta[f], dS)
+            dkb[f] += gk; dvb[f] += gv; dbeta[f] += gb
+        dS0 += dS
+    # frame statistics: kb = normalise(mean k), vb = mean v
+    dkraw = l2_normalize_bwd(kb_raw, dkb)
+    dk = np.repeat(dkraw / T, T, axis=0)
+    dv = np.repeat(dvb / T, T, axis=0)
+    # text init S0 = 1/2 sum k_hat v^T
+    ktr, vtr = np.asarray(kt, np.float64), np.asarray(vt, np.float64)
+    kth = vo.l2_normalize(ktr)
+    dkt = l2_normalize_bwd(ktr, 0.5 * np.einsum("hde,nhe->nhd", dS0, vtr))
+    dvt = 0.5 * np.einsum("hde,nhd->nhe", dS0, kth)
+    return dq, dk, dv, dkt, dvt, dbeta
+
+
+def layer_bwd(inp: dict, dy, F, T, C, eps=1e-6, scale=None, linear="elu1") -> dict:
+    """Gradients of sum(y * dy) for the whole layer over all video rows, with respect to
+    q, k, v, kt, vt, w_gate_s, w_gate_l, gamma, w_os, w_ol (and beta for the delta rule)."""
     q, k, v, kt, vt = (np.asarray(inp[n], np.float64) for n in ("q", "k", "v", "kt", "vt"))
-    fwd = vo.layer(inp, F, T, C, eps=eps, scale=scale)
+    fwd = vo.layer(inp, F, T, C, linear=linear, eps=eps, scale=scale)
     da, dwos, dwol = out_proj_bwd(fwd["a"], inp["w_os"], inp["w_ol"], dy)
     dq, do_s, do_l, dws, dwl, dgamma = hybrid_fuse_bwd(q, fwd["o_s"], fwd["o_l"], inp["w_gate_s"], inp["w_gate_l"],
                                                        inp["gamma"], da, eps)
     sq, sk, sv, skt, svt = softmax_branch_bwd(q, k, v, kt, vt, F, T, C, do_s, scale)
-    lq, lk, lv, lkt, lvt = linear_branch_bwd(q, k, v, kt, vt, F, T, C, do_l)
-    return {"q": dq + sq + lq, "k": sk + lk, "v": sv + lv, "kt": skt + lkt, "vt": svt + lvt,
-            "w_gate_s": dws, "w_gate_l": dwl, "gamma": dgamma, "w_os": dwos, "w_ol": dwol}
+    out = {"w_gate_s": dws, "w_gate_l": dwl, "gamma": dgamma, "w_os": dwos, "w_ol": dwol}
+    if linear == "delta":
+        lq, lk, lv, lkt, lvt, out["beta"] = delta_branch_bwd(q, k, v, kt, vt, inp["beta"], F, T, C, do_l)
+    else:
+        lq, lk, lv, lkt, lvt = linear_branch_bwd(q, k, v, kt, vt, F, T, C, do_l)
+    out.update(q=dq + sq + lq, k=sk + lk, v=sv + lv, kt=skt + lkt, vt=svt + lvt)
+    return out

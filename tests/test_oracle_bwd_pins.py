@@ -5,7 +5,8 @@ is pinned on its own (tests/test_oracle_pins.py).  The checks use a random direc
 input tensor (all of its entries at once) plus a few single entries, in float64.  The
 softmax branch with every key visible is also checked against torch's autograd of dense
 attention, a library routine.  The shapes cover chunk windows, both anchors, forward and
-backward memories, text and no text, one-frame chunks, and the scalar linear gate."""
+backward memories, text and no text, one-frame chunks, the scalar linear gate, and both
+linear branches (elu+1 and the delta rule)."""
 import numpy as np
 import pytest
 import torch
@@ -69,6 +70,17 @@ def test_layer_gradients_match_finite_differences(F, T, C, L, H, D, G_l):
 
 
 @pytest.mark.parametrize("F,T,C,L,H,D,G_l", SHAPES[:2])
+def test_delta_layer_gradients_match_finite_differences(F, T, C, L, H, D, G_l):
+    """The layer with the delta-rule linear branch: beta is an input too."""
+    inp = _inputs(F, T, L, H, D, G_l, seed=13)
+    inp["beta"] = 1.0 / (1.0 + np.exp(-np.random.default_rng(14).standard_normal((F, H))))
+    dy = np.random.default_rng(15).standard_normal((F * T, H * D))
+    grads = vb.layer_bwd(inp, dy, F, T, C, linear="delta")
+    _check_fd(lambda: float((vo.layer(inp, F, T, C, linear="delta")["y"] * dy).sum()), inp, grads,
+              NAMES + ("beta",))
+
+
+@pytest.mark.parametrize("F,T,C,L,H,D,G_l", SHAPES[:2])
 def test_branch_gradients_match_finite_differences(F, T, C, L, H, D, G_l):
     """Each branch alone, so a mistake is located at its branch."""
     inp = _inputs(F, T, L, H, D, G_l, seed=3)
@@ -85,6 +97,14 @@ def test_branch_gradients_match_finite_differences(F, T, C, L, H, D, G_l):
     _check_fd(soft, inp, dict(zip(names, g)), names)
     g = vb.linear_branch_bwd(inp["q"], inp["k"], inp["v"], inp["kt"], inp["vt"], F, T, C, do)
     _check_fd(lin, inp, dict(zip(names, g)), names)
+    inp["beta"] = np.random.default_rng(9).uniform(0.05, 0.95, (F, H))
+
+    def delta():
+        return float((vo.delta_branch(inp["q"], inp["k"], inp["v"], inp["kt"], inp["vt"], inp["beta"], F, T, C)
+                      * do).sum())
+
+    g = vb.delta_branch_bwd(inp["q"], inp["k"], inp["v"], inp["kt"], inp["vt"], inp["beta"], F, T, C, do)
+    _check_fd(delta, inp, dict(zip(names + ("beta",), g)), names + ("beta",))
 
 
 @pytest.mark.parametrize("G_l", [None, 1])
@@ -138,7 +158,8 @@ def test_out_proj_gradients_are_the_transposed_products():
     np.testing.assert_allclose(dwol, twl.grad.numpy(), rtol=1e-12)
 
 
-@pytest.mark.parametrize("slip", ["text_once", "rms_sign", "phi_prime", "gate_prime", "no_center"])
+@pytest.mark.parametrize("slip", ["text_once", "rms_sign", "phi_prime", "gate_prime", "no_center",
+                                  "delta_transpose"])
 def test_planted_backward_mistakes_are_caught(monkeypatch, slip):
     """Plausible slips in the backward oracle fail the finite-difference pin."""
     F, T, C, L, H, D = 7, 2, 2, 3, 1, 4
@@ -170,7 +191,19 @@ def test_planted_backward_mistakes_are_caught(monkeypatch, slip):
         monkeypatch.setattr(vb, "hybrid_fuse_bwd", bad)
     elif slip == "no_center":    # the softmax Jacobian without its -dO.o term
         monkeypatch.setattr(vb, "attention_ds", lambda p, dO, o, V: p * (dO @ V.T))
-    grads = vb.layer_bwd(inp, dy, F, T, C)
+    elif slip == "delta_transpose":  # only one of the two S terms of dkb in the delta step
+        orig_step = vb.delta_update_bwd
+
+        def bad(S, kb, vb_, beta, dS1):
+            dS, dkb, dvb, dbeta = orig_step(S, kb, vb_, beta, dS1)
+            return dS, dkb + np.asarray(beta)[:, None] * np.einsum("hde,hfe,hf->hd", S, dS1, kb), dvb, dbeta
+        monkeypatch.setattr(vb, "delta_update_bwd", bad)
+    linear = "delta" if slip == "delta_transpose" else "elu1"
+    names = NAMES
+    if linear == "delta":
+        inp["beta"] = np.random.default_rng(23).uniform(0.05, 0.95, (F, H))
+        names = NAMES + ("beta",)
+    grads = vb.layer_bwd(inp, dy, F, T, C, linear=linear)
     monkeypatch.undo()
     with pytest.raises(AssertionError):
-        _check_fd(lambda: float((vo.layer(inp, F, T, C)["y"] * dy).sum()), inp, grads, NAMES)
+        _check_fd(lambda: float((vo.layer(inp, F, T, C, linear=linear)["y"] * dy).sum()), inp, grads, names)
