@@ -1,6 +1,7 @@
 """Host logic of the benchmark on CPU: the replica (data-parallel) layout with two ranks
 over gloo.  Each rank draws its own batch, the timing reduction takes the max over
-ranks, and the whole-job value counts every rank's tokens."""
+ranks, and the whole-job value counts every rank's tokens.  Also the traffic lookup, the
+per-kernel rooflines, and the reference arm's JSON line."""
 import os
 import socket
 
@@ -97,3 +98,31 @@ def test_kernel_rooflines_use_the_algorithmic_work():
     tf = work["softmax_tc"][1] / 5e-3 / 1e12
     assert abs(k["softmax_tc"]["frac_of_sustained"] - round(tf / 800.0, 3)) < 1e-3
     assert "fp8_quant" in bench.kernel_work(shape, "delta", fp8=True)
+
+
+def _bench_reference(env_extra):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **env_extra)
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config", "1",
+                        "--steps", "2", "--warmup", "1"], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    return [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_reference_arm_prints_the_contract_line_on_rank_0_only():
+    """--impl reference times the CPU oracle on rank 0 and prints one JSON line with the
+    arm's keys; another rank of a multi-rank launch exits 0 without work."""
+    lines = _bench_reference({"RANK": "0", "WORLD_SIZE": "1"})
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["metric"] == bench.METRIC and d["unit"] == bench.UNIT and d["steps"] == 2 and d["warmup"] == 1
+    assert d["config"]["workload"] == synth.CONFIGS[1].name
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert _bench_reference({"RANK": "1", "WORLD_SIZE": "2"}) == []
