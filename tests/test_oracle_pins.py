@@ -276,6 +276,50 @@ def test_delta_exact_write_at_beta_one():
         np.testing.assert_allclose(kb[h] @ S1[h], vb[h], rtol=1e-12, atol=1e-12)   # k^T S_new = v^T
 
 
+def test_delta_frame_stats_single_token_frames():
+    # T = 1: the frame mean is the token itself, so kb = k / ||k|| and vb = v exactly
+    rng = np.random.default_rng(31)
+    F, H, D = 5, 3, 7
+    k, v = rng.standard_normal((F, H, D)) * 3, rng.standard_normal((F, H, D))
+    kb, vb = vo.delta_frame_stats(k, v, F, 1)
+    np.testing.assert_allclose(kb, k / np.linalg.norm(k, axis=-1, keepdims=True), rtol=1e-15)
+    np.testing.assert_array_equal(vb, v)
+
+
+def test_delta_frame_stats_closed_forms():
+    F, T, H, D = 3, 2, 1, 2
+    k = np.zeros((F * T, H, D)); v = np.zeros((F * T, H, D))
+    # frame 0: keys (3, 0) and (0, 1): mean (1.5, 0.5), normalised (3, 1) / sqrt(10); taking
+    # each key's direction first would give (1, 1) / sqrt(2)
+    k[0, 0] = [3.0, 0.0]; k[1, 0] = [0.0, 1.0]
+    v[0, 0] = [2.0, -4.0]; v[1, 0] = [4.0, 8.0]
+    # frame 1: two identical tokens: kb = k / ||k||, vb = v
+    k[2, 0] = k[3, 0] = [-6.0, 8.0]
+    v[2, 0] = v[3, 0] = [0.5, 0.25]
+    # frame 2: keys k and -k: zero mean, which normalises to zero (R13)
+    k[4, 0] = [1.0, 2.0]; k[5, 0] = [-1.0, -2.0]
+    kb, vb = vo.delta_frame_stats(k, v, F, T)
+    np.testing.assert_allclose(kb[0, 0], np.array([3.0, 1.0]) / np.sqrt(10.0), rtol=1e-15)
+    np.testing.assert_allclose(vb[0, 0], [3.0, 2.0], rtol=1e-15)
+    np.testing.assert_allclose(kb[1, 0], [-0.6, 0.8], rtol=1e-15)
+    np.testing.assert_allclose(vb[1, 0], [0.5, 0.25], rtol=1e-15)
+    np.testing.assert_array_equal(kb[2, 0], [0.0, 0.0])
+
+
+def test_delta_frame_stats_matches_torch_composition():
+    # frame-major rows [F*T, H, D]: frame f is rows f*T .. f*T+T-1; the mean runs over the
+    # tokens of a frame, separately for every head and feature
+    F, T, H, D = 6, 5, 3, 4
+    rng = np.random.default_rng(32)
+    k = rng.standard_normal((F * T, H, D)) * rng.uniform(0.1, 5.0, (F * T, H, 1))
+    v = rng.standard_normal((F * T, H, D))
+    kb, vb = vo.delta_frame_stats(k, v, F, T)
+    tk, tv = torch.from_numpy(k).view(F, T, H, D), torch.from_numpy(v).view(F, T, H, D)
+    ref_kb = torch.nn.functional.normalize(tk.mean(dim=1), dim=-1)
+    np.testing.assert_allclose(kb, ref_kb.numpy(), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(vb, tv.mean(dim=1).numpy(), rtol=1e-13, atol=1e-15)
+
+
 def test_delta_per_group_rerun_equals_single_pass_snapshots():
     F, T, C, L, H, D = 33, 2, 5, 3, 2, 8
     x = _inputs(F, T, L, H, D, seed=19)
@@ -391,6 +435,9 @@ def _pins_hold():
         lambda: test_delta_single_update_from_zero(),
         lambda: test_delta_exact_write_at_beta_one(),
         lambda: test_delta_per_group_rerun_equals_single_pass_snapshots(),
+        lambda: test_delta_frame_stats_single_token_frames(),
+        lambda: test_delta_frame_stats_closed_forms(),
+        lambda: test_delta_frame_stats_matches_torch_composition(),
         lambda: test_softmax_matches_masked_sdpa(23, 3, 5, 2),
     ]
     for c in checks:
@@ -440,12 +487,33 @@ def _softmax_without_text(q, k, v, kt, vt, F, T, C, scale=None, rows=None):
     return vo.__dict__["_orig_softmax_branch"](q, k, v, kt[:0], vt[:0], F, T, C, scale, rows)
 
 
+def _delta_stats_tokens_normalised_first(k, v, F, T):
+    kb, vb = vo.__dict__["_orig_delta_frame_stats"](vo.l2_normalize(k), v, F, T)
+    return kb, vb                                         # each key's direction averaged
+
+
+def _delta_stats_unnormalised(k, v, F, T):
+    N, H, D = k.shape
+    kb = np.asarray(k, np.float64).reshape(F, T, H, D).mean(axis=1)   # mean key, left unnormalised
+    return kb, np.asarray(v, np.float64).reshape(F, T, H, D).mean(axis=1)
+
+
+def _delta_stats_strided_frames(k, v, F, T):
+    # frame f taken as rows f, f+F, f+2F, ... (token-major reading of frame-major rows)
+    N, H, D = k.shape
+    kb = vo.l2_normalize(np.asarray(k, np.float64).reshape(T, F, H, D).mean(axis=0))
+    return kb, np.asarray(v, np.float64).reshape(T, F, H, D).mean(axis=0)
+
+
 @pytest.mark.parametrize("attr,bad", [
     ("frame_mask", _mask_without_anchor_reads),
     ("frame_mask", _mask_swapped),
     ("text_state", _text_state_full),
     ("delta_update", _delta_update_wrong_sign),
     ("softmax_branch", _softmax_without_text),
+    ("delta_frame_stats", _delta_stats_tokens_normalised_first),
+    ("delta_frame_stats", _delta_stats_unnormalised),
+    ("delta_frame_stats", _delta_stats_strided_frames),
 ])
 def test_planted_mistake_is_caught(monkeypatch, attr, bad):
     monkeypatch.setattr(vo, "_orig_" + attr, getattr(vo, attr), raising=False)
