@@ -126,6 +126,8 @@ struct ProfScope {
   ~ProfScope() { prof_mark(kid, false, st); }
 };
 
+constexpr uint32_t DEBUG_MAX_POLLS = 1000000u;
+
 float scale_log2_of(float sm_scale, int D) {
   const float s = sm_scale > 0.f ? sm_scale : 1.f / std::sqrt((float)D);
   return s * 1.4426950408889634f;
@@ -177,6 +179,22 @@ vdn_status out_proj_dispatch(const Dims &d, vdn_dtype act, const void *a, const 
 namespace vdn {
 // lets entry points defined in other files report through vdn_last_error()
 void set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+// the checks every softmax-branch entry point applies, shared so that they accept exactly
+// the same arguments (each reports through vdn_last_error())
+vdn_status softmax_args_check(const vdn_shape *shape, vdn_dtype dtype, const void *q, const void *k, const void *v,
+                              const void *kt, const void *vt, const float *scales, float sm_scale, const void *o_s) {
+  VDN_TRY(check_shape(shape));
+  if (dtype != VDN_F32 && dtype != VDN_BF16 && dtype != VDN_E4M3)
+    return fail(VDN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  VDN_TRY(need(q, "q")); VDN_TRY(need(k, "k")); VDN_TRY(need(v, "v")); VDN_TRY(need(o_s, "o_s"));
+  if (shape->text_tokens > 0) { VDN_TRY(need(kt, "kt")); VDN_TRY(need(vt, "vt")); }
+  if ((dtype == VDN_E4M3) != (scales != nullptr))
+    return fail(VDN_ERR_INVALID_ARG, "scales must be given exactly when dtype is VDN_E4M3");
+  if (!std::isfinite(sm_scale)) return fail(VDN_ERR_INVALID_ARG, "sm_scale is not finite");
+  return VDN_OK;
+}
+vdn_status device_check() { return check_device(); }
+float softmax_scale_log2(float sm_scale, int D) { return scale_log2_of(sm_scale, D); }
 }  // namespace vdn
 
 extern "C" {
@@ -222,14 +240,7 @@ vdn_status vdn_workspace_init(void *ws, size_t ws_bytes, vdn_stream stream) {
 vdn_status vdn_softmax_branch_fwd(const vdn_shape *shape, vdn_dtype dtype, const void *q, const void *k,
                                   const void *v, const void *kt, const void *vt, const float *scales, float sm_scale,
                                   void *o_s, float *lse, void *ws, size_t ws_bytes, vdn_stream stream) {
-  VDN_TRY(check_shape(shape));
-  if (dtype != VDN_F32 && dtype != VDN_BF16 && dtype != VDN_E4M3)
-    return fail(VDN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
-  VDN_TRY(need(q, "q")); VDN_TRY(need(k, "k")); VDN_TRY(need(v, "v")); VDN_TRY(need(o_s, "o_s"));
-  if (shape->text_tokens > 0) { VDN_TRY(need(kt, "kt")); VDN_TRY(need(vt, "vt")); }
-  if ((dtype == VDN_E4M3) != (scales != nullptr))
-    return fail(VDN_ERR_INVALID_ARG, "scales must be given exactly when dtype is VDN_E4M3");
-  if (!std::isfinite(sm_scale)) return fail(VDN_ERR_INVALID_ARG, "sm_scale is not finite");
+  VDN_TRY(softmax_args_check(shape, dtype, q, k, v, kt, vt, scales, sm_scale, o_s));
   const WsPlan p = plan_workspace(*shape, VDN_LIN_ELU1, VDN_BF16);
   VDN_TRY(check_ws(ws, ws_bytes, p.step_end));
   VDN_TRY(check_device());
@@ -589,7 +600,9 @@ vdn_status vdn_profile_end(float *ms, int32_t *launches, int32_t n) {
 
 vdn_status vdn_debug_unset_flag_wait(void *ws, size_t ws_bytes, uint32_t max_polls, vdn_stream stream) {
   VDN_TRY(check_ws(ws, ws_bytes, 256));
-  if (max_polls == 0) return fail(VDN_ERR_INVALID_ARG, "max_polls must be >= 1");
+  // at about 64 ns a poll, 10^6 polls keep the test wait near 64 ms
+  if (max_polls == 0 || max_polls > DEBUG_MAX_POLLS)
+    return fail(VDN_ERR_INVALID_ARG, "max_polls must be in [1, %u]", DEBUG_MAX_POLLS);
   VDN_TRY(check_device());
   VDN_CUDA(launch_debug_wait((char *)ws, max_polls, (cudaStream_t)stream), "debug wait launch");
   return ok();

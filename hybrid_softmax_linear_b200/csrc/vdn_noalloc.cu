@@ -8,24 +8,26 @@
 //
 // The array is a file-scope __device__ array: each GPU that loads the library holds
 // it until the process exits.  Host code cannot use the array's name as a device
-// address, so the address is looked up once per device with cudaGetSymbolAddress
-// (on the first call made on that device) and passed to the kernels.
+// address: every call looks the address up with cudaGetSymbolAddress in the context
+// current at that moment (a host-side lookup) and passes it to the kernels, so a caller
+// that switches contexts never gets an address that belongs to another one.  The first
+// call on a device (or in a new context) also loads the library's device code there,
+// which is why that first call should come before any stream capture.
 #include <cstdio>
-#include <mutex>
 
 #include "vdn_internal.cuh"
 
 namespace vdn {
 void set_last_error(const char *msg);  // vdn_api.cu
+vdn_status softmax_args_check(const vdn_shape *shape, vdn_dtype dtype, const void *q, const void *k, const void *v,
+                              const void *kt, const void *vt, const float *scales, float sm_scale, const void *o_s);
+vdn_status device_check();
+float softmax_scale_log2(float sm_scale, int D);
 
 namespace {
 
 constexpr size_t NOALLOC_SCRATCH_BYTES = 256u * 1024u;  // 256 KiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
-
-constexpr int MAX_DEVICES = 64;
-std::mutex g_mu;
-void *g_scratch_ptr[MAX_DEVICES] = {nullptr};
 
 // messages go to the library's vdn_last_error()
 vdn_status noalloc_fail(vdn_status code, const char *msg, cudaError_t e = cudaSuccess) {
@@ -38,21 +40,13 @@ vdn_status noalloc_fail(vdn_status code, const char *msg, cudaError_t e = cudaSu
   return code;
 }
 
-// Device address of the scratch array on the current device (looked up once per device).
+// Device address of the scratch array in the current context.
 vdn_status scratch_address(char **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return noalloc_fail(VDN_ERR_CUDA, "cudaGetDevice", e);
-  if (dev < 0 || dev >= MAX_DEVICES) return noalloc_fail(VDN_ERR_UNSUPPORTED, "device index out of range");
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return noalloc_fail(VDN_ERR_CUDA, "cudaGetSymbolAddress of the static scratch array", e);
-    g_scratch_ptr[dev] = p;
-  }
-  *out = (char *)g_scratch_ptr[dev];
+  void *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr)
+    return noalloc_fail(VDN_ERR_CUDA, "cudaGetSymbolAddress of the static scratch array", e);
+  *out = (char *)p;
   return VDN_OK;
 }
 
@@ -66,42 +60,31 @@ extern "C" VDN_API vdn_status vdn_softmax_branch_fwd_noalloc(const vdn_shape *sh
                                                              const void *vt, float sm_scale, void *o_s, float *lse,
                                                              vdn_stream stream) {
   set_last_error("");
-  if (shape == nullptr) return noalloc_fail(VDN_ERR_INVALID_ARG, "shape is NULL");
-  const vdn_shape &s = *shape;
-  if (s.frames < 1 || s.tokens_per_frame < 1 || s.chunk_frames < 1 || s.text_tokens < 0 || s.heads < 1)
-    return noalloc_fail(VDN_ERR_INVALID_ARG, "shape out of range");
-  if (s.head_dim != 32 && s.head_dim != 64 && s.head_dim != 128)
-    return noalloc_fail(VDN_ERR_UNSUPPORTED, "head_dim not in {32, 64, 128}");
-  if ((int64_t)s.frames * s.tokens_per_frame + s.text_tokens >= ((int64_t)1 << 31))
-    return noalloc_fail(VDN_ERR_INVALID_ARG, "shape too large");
+  // the same argument checks as vdn_softmax_branch_fwd; e4m3 needs its scales, which this
+  // entry point does not take
   if (dtype != VDN_F32 && dtype != VDN_BF16)
     return noalloc_fail(VDN_ERR_UNSUPPORTED, "dtype must be VDN_F32 or VDN_BF16");
-  auto bad = [](const void *p) { return p == nullptr || ((uintptr_t)p & 15u) != 0; };
-  if (bad(q) || bad(k) || bad(v) || bad(o_s) || (s.text_tokens > 0 && (bad(kt) || bad(vt))))
-    return noalloc_fail(VDN_ERR_INVALID_ARG, "a tensor pointer is NULL or not 16-byte aligned");
+  vdn_status rs = softmax_args_check(shape, dtype, q, k, v, kt, vt, nullptr, sm_scale, o_s);
+  if (rs != VDN_OK) return rs;
+  const vdn_shape &s = *shape;
   const WsPlan p = plan_workspace(s, VDN_LIN_ELU1, VDN_BF16);
   if (p.step_end > NOALLOC_SCRATCH_BYTES)
     return noalloc_fail(VDN_ERR_WORKSPACE,
                         "shape needs more scratch than the fixed 256 KiB array (tables and query-tile list); "
                         "use vdn_softmax_branch_fwd with a workspace");
-  int dev = 0, major = 0, minor = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  if (e != cudaSuccess) return noalloc_fail(VDN_ERR_CUDA, "device query", e);
-  if (major != 10 || minor != 0) return noalloc_fail(VDN_ERR_UNSUPPORTED, "libvdn is built for sm_100a (B200) only");
+  rs = device_check();
+  if (rs != VDN_OK) return rs;
   char *scratch = nullptr;
-  vdn_status rs = scratch_address(&scratch);
+  rs = scratch_address(&scratch);
   if (rs != VDN_OK) return rs;
   cudaStream_t st = (cudaStream_t)stream;
   const Dims d = dims_of(s);
   // the status word must start at zero; the tables and tile list are rewritten below
-  e = cudaMemsetAsync(scratch + p.status, 0, 256, st);
+  cudaError_t e = cudaMemsetAsync(scratch + p.status, 0, 256, st);
   if (e != cudaSuccess) return noalloc_fail(VDN_ERR_CUDA, "clearing the scratch status word", e);
   e = launch_tables(d, scratch, p, st);
   if (e != cudaSuccess) return noalloc_fail(VDN_ERR_CUDA, "tables launch", e);
-  const float scale = sm_scale > 0.f ? sm_scale : 1.f / sqrtf((float)s.head_dim);
-  const float sl2 = scale * 1.4426950408889634f;
+  const float sl2 = softmax_scale_log2(sm_scale, s.head_dim);
   if (softmax_tc_supported(d, dtype))
     e = launch_softmax_tc(d, dtype, q, k, v, kt, vt, nullptr, sl2, o_s, lse, scratch, p, st);
   else

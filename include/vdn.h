@@ -141,17 +141,25 @@ VDN_API vdn_status vdn_softmax_branch_fwd(const vdn_shape *shape, vdn_dtype dtyp
  * (status word, layout tables, query-tile list) in a fixed 256 KiB array that the
  * library holds in device memory on every GPU that loads it, until the process exits.
  * Nothing is allocated or freed: no cudaMalloc, no cudaFree, no allocating library call.
- *   - Arguments and results as vdn_softmax_branch_fwd, for dtype VDN_F32 or VDN_BF16.
- *   - Shapes whose tables and tile list need more than the 256 KiB (about 16k query
- *     tiles of 256 rows) are rejected with VDN_ERR_WORKSPACE.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Arguments, checks and results as vdn_softmax_branch_fwd, for dtype VDN_F32 or
+ *     VDN_BF16 (both entry points run the same argument checks).
+ *   - Capacity: the array holds the layout tables (about 80 bytes per frame) and the
+ *     query-tile list (32 bytes per tile of at most 256 query rows).  At 1008 tokens per
+ *     frame in 5-frame chunks that is up to 1343 frames (about 1.35M video tokens); at 256
+ *     tokens per frame, 2604 frames.  Larger shapes are rejected with VDN_ERR_WORKSPACE
+ *     before any device work.
+ *   - Every call looks up the array's device address in the context current at that
+ *     moment (cudaGetSymbolAddress, a host-side lookup).  The first call on a device, or
+ *     in a new context, also loads the library's device code there: make that first
+ *     call before any stream capture.
  *   - Every call shares the one array, which keeps the last call's contents; each call
  *     clears the status word and rewrites the tables before its kernels run.  Calls
  *     that overlap on the GPU (other streams, other host threads) race on the array and
  *     must be serialised by the caller.
- *   - Device-side wait timeouts are recorded in the array's status word but not
- *     reported: the call never synchronises.  Launch errors are returned. */
+ *   - Device-side errors (a wait timeout, or a layout-table error that makes the softmax
+ *     kernel skip its work and leave o_s and lse unwritten) are recorded in the array's
+ *     status word but not reported: the call never synchronises.  Launch errors are
+ *     returned. */
 VDN_API vdn_status vdn_softmax_branch_fwd_noalloc(const vdn_shape *shape, vdn_dtype dtype, const void *q,
                                                   const void *k, const void *v, const void *kt, const void *vt,
                                                   float sm_scale, void *o_s, float *lse, vdn_stream stream);
@@ -280,7 +288,8 @@ VDN_API void *vdn_hybrid_attn_intermediate(const vdn_shape *shape, vdn_lin_kind 
 VDN_API vdn_status vdn_check_device_status(void *ws, size_t ws_bytes, vdn_stream stream);
 
 /* Test hook for the bounded device wait: launches one block that waits on a flag in ws
- * that nothing sets, giving up after `max_polls` polls and recording VDN_ERR_TIMEOUT in
+ * that nothing sets, giving up after `max_polls` polls (1 <= max_polls <= 10^6, about
+ * 64 ms at most; other values give VDN_ERR_INVALID_ARG) and recording VDN_ERR_TIMEOUT in
  * the status word.  Read the outcome with vdn_check_device_status. */
 VDN_API vdn_status vdn_debug_unset_flag_wait(void *ws, size_t ws_bytes, uint32_t max_polls, vdn_stream stream);
 

@@ -117,6 +117,37 @@ def test_argument_checks_precede_cuda():
     st = L.vdn_hybrid_attn_fwd(ctypes.byref(s), 7, vdn.F32, 16, 16, 16, 16, 16, None, 16, 16, 32, 16, 1e-6, 16, 16,
                                16, 256, 1 << 30, None)
     assert st == 1  # unknown kind
+    for polls in (0, 1000001, 0xFFFFFFFF):
+        assert L.vdn_debug_unset_flag_wait(256, 1 << 20, polls, None) == 1  # the test wait stays short
+
+
+def test_noalloc_checks_match_the_workspace_entry_point():
+    """The no-allocation softmax entry point rejects exactly what vdn_softmax_branch_fwd
+    rejects, before any device work, and refuses shapes whose scratch exceeds its fixed
+    256 KiB array (2604 frames of 256 tokens in 5-frame chunks fit, 2605 do not)."""
+    L = vdn.lib()
+    ok = vdn.Shape(15, 16, 1, 4, 2, 32)
+    cases = [
+        (ok, 0.0, (None, 16, 16, 16, 16), 1),                      # q NULL
+        (ok, 0.0, (24, 16, 16, 16, 16), 1),                        # q misaligned
+        (ok, float("inf"), (16, 16, 16, 16, 16), 1),               # non-finite scale
+        (ok, float("nan"), (16, 16, 16, 16, 16), 1),
+        (vdn.Shape(4, 4, 1, 0, 1025, 64), 0.0, (16, 16, 16, 16, 16), 1),   # H*D > 65536
+        (vdn.Shape(4, 4, 1, 0, 1, 48), 0.0, (16, 16, 16, 16, 16), 2),      # head_dim 48
+        (vdn.Shape(0, 4, 1, 0, 1, 32), 0.0, (16, 16, 16, 16, 16), 1),      # no frames
+    ]
+    for sh, scale, (q, k, v, kt, vt), want in cases:
+        a = L.vdn_softmax_branch_fwd(ctypes.byref(sh), vdn.BF16, q, k, v, kt, vt, None, scale, 16, None, 256, 1 << 30,
+                                     None)
+        b = L.vdn_softmax_branch_fwd_noalloc(ctypes.byref(sh), vdn.BF16, q, k, v, kt, vt, scale, 16, None, None)
+        assert a == b == want, (sh.frames, sh.heads, sh.head_dim, scale, a, b)
+    st = L.vdn_softmax_branch_fwd_noalloc(ctypes.byref(ok), vdn.E4M3, 16, 16, 16, 16, 16, 0.0, 16, None, None)
+    assert st == 2  # e4m3 needs scales, which this entry point does not take
+    fits, over = vdn.Shape(2604, 256, 5, 16, 1, 64), vdn.Shape(2605, 256, 5, 16, 1, 64)
+    st = L.vdn_softmax_branch_fwd_noalloc(ctypes.byref(fits), vdn.BF16, 16, 16, 16, 16, 16, 0.0, 16, None, None)
+    assert st not in (0, 1, 3)  # passes every argument check; fails only for want of a GPU here
+    st = L.vdn_softmax_branch_fwd_noalloc(ctypes.byref(over), vdn.BF16, 16, 16, 16, 16, 16, 0.0, 16, None, None)
+    assert st == 3 and b"256 KiB" in L.vdn_last_error()
 
 
 def test_host_entry_point_checks_and_sizes():

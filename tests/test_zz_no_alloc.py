@@ -26,32 +26,68 @@ CASES = [
 ]
 
 
+def _setup(case, seed):
+    F, T, C, L, H, D, dt = case
+    s = synth.Shape(F, T, C, L, H, D)
+    inp = synth.make_inputs(s, dt, seed=seed)
+    return s, {n: to_device(a) for n, a in inp.items()}
+
+
+def _workspace_reference(s, dt, d):
+    cdt = vdn.F32 if dt == "f32" else vdn.BF16
+    ws = workspace(vdn.step_workspace_size(s))
+    vdn.workspace_init(ws)
+    ref = empty((s.n_video, s.heads, s.head_dim), dt)
+    ref_lse = torch.empty((s.n_video, s.heads), dtype=torch.float32, device="cuda")
+    vdn.softmax_branch_fwd(s, cdt, d["q"], d["k"], d["v"], d["kt"], d["vt"], ref, ws, lse=ref_lse)
+    vdn.check_device_status(ws)
+    return to_numpy(ref), ref_lse.cpu().numpy(), ref.dtype
+
+
+def _noalloc_call(s, dt, d, out_dtype):
+    cdt = vdn.F32 if dt == "f32" else vdn.BF16
+    out = torch.full((s.n_video, s.heads, s.head_dim), float("nan"), dtype=out_dtype, device="cuda")
+    lse = torch.full((s.n_video, s.heads), float("nan"), dtype=torch.float32, device="cuda")
+    vdn.softmax_branch_fwd_noalloc(s, cdt, d["q"], d["k"], d["v"], d["kt"], d["vt"], out, lse=lse)
+    torch.cuda.synchronize()
+    return to_numpy(out), lse.cpu().numpy()
+
+
 @pytest.mark.parametrize("case", CASES)
 def test_noalloc_matches_workspace_entry_point_twice(case):
     assert torch.cuda.is_available(), "GPU test needs a CUDA device"
-    F, T, C, L, H, D, dt = case
-    s = synth.Shape(F, T, C, L, H, D)
-    cdt = vdn.F32 if dt == "f32" else vdn.BF16
-    tol = "f32" if dt == "f32" else "bf16"
-    inp = synth.make_inputs(s, dt, seed=77 + F)
-    d = {n: to_device(a) for n, a in inp.items()}
-    Nv = s.n_video
-
-    ws = workspace(vdn.step_workspace_size(s))
-    vdn.workspace_init(ws)
-    ref = empty((Nv, H, D), dt)
-    ref_lse = torch.empty((Nv, H), dtype=torch.float32, device="cuda")
-    vdn.softmax_branch_fwd(s, cdt, d["q"], d["k"], d["v"], d["kt"], d["vt"], ref, ws, lse=ref_lse)
-    vdn.check_device_status(ws)
-    ref_np, ref_lse_np = to_numpy(ref), ref_lse.cpu().numpy()
-
+    dt = case[-1]
+    s, d = _setup(case, 77 + case[0])
+    ref_np, ref_lse_np, odt = _workspace_reference(s, dt, d)
     for call in range(2):
-        out = torch.full((Nv, H, D), float("nan"), dtype=ref.dtype, device="cuda")
-        lse = torch.full((Nv, H), float("nan"), dtype=torch.float32, device="cuda")
-        vdn.softmax_branch_fwd_noalloc(s, cdt, d["q"], d["k"], d["v"], d["kt"], d["vt"], out, lse=lse)
-        torch.cuda.synchronize()
-        assert_close(f"no-alloc output, call {call + 1}", to_numpy(out), ref_np, tol)
-        np.testing.assert_allclose(lse.cpu().numpy(), ref_lse_np, rtol=1e-5, atol=1e-5)
+        out, lse = _noalloc_call(s, dt, d, odt)
+        assert_close(f"no-alloc output, call {call + 1}", out, ref_np, "f32" if dt == "f32" else "bf16")
+        np.testing.assert_allclose(lse, ref_lse_np, rtol=1e-5, atol=1e-5)
+
+
+def test_noalloc_after_a_larger_call_with_other_tables():
+    # the shared array keeps the previous call's tables and tile list: a smaller shape with
+    # another frame count, chunk size and text length must not read any of them
+    big = (40, 300, 4, 70, 4, 128, "bf16")
+    small = (11, 130, 3, 9, 3, 128, "bf16")
+    s_big, d_big = _setup(big, 5)
+    s_small, d_small = _setup(small, 6)
+    ref_np, ref_lse_np, odt = _workspace_reference(s_small, "bf16", d_small)
+    _noalloc_call(s_big, "bf16", d_big, odt)
+    out, lse = _noalloc_call(s_small, "bf16", d_small, odt)
+    assert_close("no-alloc output after a larger call", out, ref_np, "bf16")
+    np.testing.assert_allclose(lse, ref_lse_np, rtol=1e-5, atol=1e-5)
+
+
+def test_noalloc_at_the_size_limit():
+    # 2604 frames of 256 tokens in 5-frame chunks is the largest frame count whose tables and
+    # query-tile list fit the 256 KiB array (2605 is rejected, see tests/test_abi_cpu.py)
+    case = (2604, 256, 5, 16, 1, 64, "bf16")
+    s, d = _setup(case, 8)
+    ref_np, ref_lse_np, odt = _workspace_reference(s, "bf16", d)
+    out, lse = _noalloc_call(s, "bf16", d, odt)
+    assert_close("no-alloc output at the size limit", out, ref_np, "bf16")
+    np.testing.assert_allclose(lse, ref_lse_np, rtol=1e-5, atol=1e-5)
 
 
 def test_noalloc_rejects_shapes_beyond_the_fixed_scratch():
