@@ -2,6 +2,7 @@
 over gloo.  Each rank draws its own batch, the timing reduction takes the max over
 ranks, and the whole-job value counts every rank's tokens.  Also the traffic lookup, the
 per-kernel rooflines, and the reference arm's JSON line."""
+import json
 import os
 import socket
 
@@ -69,8 +70,8 @@ def test_captured_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     src = tmp_path / "k.cu"
     src.write_text("kernel source\n")
     sha = hashlib.sha256(src.read_bytes()).hexdigest()
-    cap = tmp_path / "cap.md"
-    cap.write_text(f"# title\n\nsource_sha256: {sha}\nbf16: 1000 bytes over 10 units\n")
+    cap = tmp_path / "cap.json"
+    cap.write_text(json.dumps({"source_sha256": sha, "bf16": {"bytes": 1000, "units": 10}}))
     monkeypatch.setattr(bench, "SOFTMAX_SRC", str(src))
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(cap))
     shape = synth.Shape(2, 5, 1, 0, 2, 32)                     # 10 rows x 2 heads = 20 units
