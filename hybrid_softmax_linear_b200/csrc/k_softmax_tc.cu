@@ -10,15 +10,20 @@
 // once softmax warpgroup w has rescaled its output and written P_w (bf16 or e4m3, over
 // S_w's columns; e4m3 in two pieces of 64 keys, each handed over as soon as it is
 // written), O_w += P_w V_j (A operand from tensor memory, V as an MN-major operand).
-// Warpgroups 0 and 1 (warps 2-5 and 6-9) run the online softmax of Q0 and Q1, one row
+// Warpgroups 1 and 2 (warps 4-7 and 8-11) run the online softmax of Q0 and Q1, one row
 // per thread, so while one warpgroup exponentiates, the tensor cores work for the
-// other.  The running maximum is only moved (and O rescaled) when it grows by more than
+// other.  Warpgroup 0 (the TMA and MMA warps and two idle ones) hands most of its
+// registers to the softmax warpgroups (setmaxnreg), which keep a whole row of S in
+// registers and work on pairs of values with the packed fp32 instructions of sm_100.
+// (A share of the exponentials can run as a polynomial on the FMA pipe instead of the
+// exponential unit, VDN_SOFTMAX_POLY_PAIRS; measured slower at every share, so off.)
+// The running maximum is only moved (and O rescaled) when it grows by more than
 // 2^8; the final normalisation uses the same stale maximum, so the result is exact.
 // Keys past the end of a segment are masked in the last tile of that segment.
 #include "tc_common.cuh"
 
-#ifndef VDN_SOFTMAX_POLY_EIGHTHS
-#define VDN_SOFTMAX_POLY_EIGHTHS 0
+#ifndef VDN_SOFTMAX_POLY_PAIRS
+#define VDN_SOFTMAX_POLY_PAIRS 0
 #endif
 
 namespace vdn {
@@ -30,7 +35,9 @@ constexpr int BM = 128;     // rows per Q tile
 constexpr int BN = 128;     // keys per K/V tile
 constexpr int NQ = 2;       // Q tiles per CTA
 constexpr int KST = 2, VST = 2;
-constexpr int THREADS = 320;
+constexpr int THREADS = 384;      // 12 warps: warpgroup 0 = TMA, MMA, 2 idle; warpgroups 1, 2 = softmax
+// registers per thread after the split: 128 x 64 + 256 x 216 = 63488, within the launch's 384 x 168
+constexpr uint32_t REGS_CTRL = 64, REGS_SOFTMAX = 216;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 // P of a tile is handed to the tensor cores in up to MAX_P_PARTS pieces (Cfg::P_PARTS)
@@ -65,18 +72,22 @@ struct Cfg {
   __device__ static constexpr uint32_t o_col(int w) { return 256u + (uint32_t)w * 128u; }
 };
 
-struct alignas(8) Bars {
-  uint64_t q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[NQ], p_ready[NQ][MAX_P_PARTS], o_done,
-      drain;
-  uint32_t tmem_base;
-  int abort;
-};
-
 // The key tiles of a group: text rows first, then video rows, each merged segment of the
 // group cut into 128-key tiles.
 struct KvParts {
   int n;
   int text[5], lo[5], hi[5];
+};
+
+struct alignas(8) Bars {
+  uint64_t q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[NQ], p_ready[NQ][MAX_P_PARTS], o_done,
+      drain;
+  uint32_t tmem_base;
+  int abort;
+  // this block's work, decoded once by thread 0; each role reads it after the register
+  // split, so that nothing computed before the split stays live across it
+  int h, row0, row_end, nkv;
+  KvParts parts;
 };
 
 __device__ __forceinline__ void kv_parts(const int32_t *g, int L, KvParts &p) {
@@ -110,27 +121,45 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA and integer pipes, for a share of the exponentials, so that the
-// hardware exponential unit (shared by both softmax warpgroups) is not the only path.
+// 2^x on the FMA and integer pipes for a share of the exponentials (pairs of values,
+// packed fp32 instructions), so that the hardware exponential unit is not the only path.
 // Range reduction: x = n + f with n = round(x) (read from the low mantissa bits after
 // adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial, fitted here for
 // minimal relative error on [-1/2, 1/2] (iteratively reweighted least squares, Lawson's
 // method; max relative error 7.5e-5, below bf16's 2^-9); 2^n is added to the exponent
-// field.  x is clamped to -125 so that the result stays a normal float (~1e-38 there).
-constexpr int POLY_EIGHTHS = VDN_SOFTMAX_POLY_EIGHTHS;  // eighths of the exponentials computed this way
+// field.  x is clamped to -125 so that the result stays a normal float (~2e-38 there).
+constexpr int POLY_PAIRS = VDN_SOFTMAX_POLY_PAIRS;  // pairs of every 16 computed this way
+static_assert(POLY_PAIRS >= 0 && POLY_PAIRS <= 16, "pairs per 32-key chunk");
 
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float j = x + 12582912.f;
-  const float n = j - 12582912.f;
-  const float f = x - n;
-  const float p = fmaf(fmaf(fmaf(0.05517132f, f, 0.24261054f), f, 0.69326097f), f, 0.99992812f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(j) << 23));
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 j = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(j, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(0.05517132f, 0.05517132f), f, make_float2(0.24261054f, 0.24261054f));
+  p = __ffma2_rn(p, f, make_float2(0.69326097f, 0.69326097f));
+  p = __ffma2_rn(p, f, make_float2(0.99992812f, 0.99992812f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
 }
 
-// element idx of a row (a compile-time constant once the loops are unrolled)
-__device__ __forceinline__ float exp2_mixed(float x, int idx) {
-  return (idx & 7) < POLY_EIGHTHS ? exp2_poly(x) : ex2(x);
+// pair i of a 16-pair chunk goes through the polynomial (spread evenly over the chunk;
+// a compile-time constant once the loops are unrolled)
+__device__ __forceinline__ constexpr bool poly_pair(int i) {
+  return ((i + 1) * POLY_PAIRS) / 16 > (i * POLY_PAIRS) / 16;
+}
+
+__device__ __forceinline__ float2 exp2_pair(float2 x, int i) {
+  if (poly_pair(i)) return exp2_poly2(x);
+  return make_float2(ex2(x.x), ex2(x.y));
+}
+
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_CTRL));
+}
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
 }
 
 // three-input max of sm_100 (half the instructions of a pairwise max tree)
@@ -159,23 +188,20 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if (skip) return;
 
-  // Blocks [H*first, H*(first+count)) belong to the group whose tiles are first..first+count-1
-  // in the tile list; inside that range the head varies slowest, so the blocks that run
-  // together share one head's keys and values in L2.
-  const int32_t *t0 = tiles + (int64_t)(blockIdx.x / d.H) * TILE_REC;
-  const int first = t0[4], count = t0[5];
-  const int rel = (int)(blockIdx.x - (unsigned)first * d.H);
-  const int h = rel / count;
-  const int32_t *tr = tiles + (int64_t)(first + rel % count) * TILE_REC;
-  const int g = tr[0], row0 = tr[1], row_end = tr[2];
-  const int32_t *grow = gtab + g * 16;
-  // e4m3: scores carry s_q * s_k, the output s_v (per-head dequantisation scales)
-  if (FP8) sl2 *= scales[h] * scales[d.H + h];
-  const float out_scale = FP8 ? scales[2 * d.H + h] : 1.f;
-  KvParts parts;
-  kv_parts(grow, d.L, parts);
-  const int nkv = kv_tiles(parts);
-
+  if (threadIdx.x == 0) {
+    // Blocks [H*first, H*(first+count)) belong to the group whose tiles are
+    // first..first+count-1 in the tile list; inside that range the head varies slowest, so
+    // the blocks that run together share one head's keys and values in L2.
+    const int32_t *t0 = tiles + (int64_t)(blockIdx.x / d.H) * TILE_REC;
+    const int first = t0[4], count = t0[5];
+    const int rel = (int)(blockIdx.x - (unsigned)first * d.H);
+    const int32_t *tr = tiles + (int64_t)(first + rel % count) * TILE_REC;
+    bars->h = rel / count;
+    bars->row0 = tr[1];
+    bars->row_end = tr[2];
+    kv_parts(gtab + tr[0] * 16, d.L, bars->parts);
+    bars->nkv = kv_tiles(bars->parts);
+  }
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
     for (int s = 0; s < KST; ++s) { mbar_init(smem_u32(&bars->k_full[s]), 1); mbar_init(smem_u32(&bars->k_empty[s]), 1); }
@@ -196,9 +222,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  if (warp < 4) {
+  reg_dealloc();
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
+      const int h = bars->h, row0 = bars->row0, nkv = bars->nkv;
+      const KvParts &parts = bars->parts;
       uint32_t armed_k = 0, ph_k = 0, armed_v = 0, ph_v = 0;
       const uint32_t qb = smem_u32(&bars->q_full);
       mbar_arrive_expect_tx(qb, NQ * C::TILE_BYTES);
@@ -252,6 +282,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
+      const int nkv = bars->nkv;
       const uint32_t qa = smem_u32(base + C::Q_OFF);
       auto issue_s = [&](int w, int j) {
         const uint32_t kbase = smem_u32(base + C::K_OFF + (j % KST) * C::TILE_BYTES);
@@ -334,9 +365,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       int no_abort = 0;
       mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_SOFTMAX_TC, 8);
     }
+  }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
-    const int w = (warp - 2) >> 2;          // Q tile of this warpgroup
+    reg_alloc();
+    const int h = bars->h, row0 = bars->row0, row_end = bars->row_end, nkv = bars->nkv;
+    const KvParts &parts = bars->parts;
+    // e4m3: scores carry s_q * s_k, the output s_v (per-head dequantisation scales)
+    if (FP8) sl2 *= scales[h] * scales[d.H + h];
+    const float out_scale = FP8 ? scales[2 * d.H + h] : 1.f;
+    const int w = (warp >> 2) - 1;          // Q tile of this warpgroup
     const int quad = warp & 3;              // tensor-memory lane quadrant
     const int r = quad * 32 + lane;         // row within the Q tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -353,8 +391,49 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool got = mbar_wait(smem_u32(&bars->s_full[w]), j & 1, abort_flag, st, K_SOFTMAX_TC, 9);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      // the whole row of S in one round trip: four loads in flight, one wait
       float s[BN];
+      float alpha = 1.f;
+      float2 rs2[4];              // row sum in four independent pair chains
+#pragma unroll
+      for (int i = 0; i < 4; ++i) rs2[i] = make_float2(0.f, 0.f);
+      const float2 sl2v = make_float2(sl2, sl2);
+      // P of keys [0, c + 32) (and the rescaled O) handed to the MMA thread at the end of
+      // each piece
+      auto hand_piece = [&](int c) {
+        if ((c + 32) % (BN / C::P_PARTS) == 0) {
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[w][(c + 32) / (BN / C::P_PARTS) - 1]));
+        }
+      };
+      // O_w was last written by P V of tile j-1, which completed before S_w of tile j; it is
+      // rescaled before any P of tile j is handed to the tensor cores
+      auto rescale_o = [&]() {
+#pragma unroll 1
+        for (int c = 0; c < D; c += 8) {  // 8 columns at a time: the row of S is still live
+          uint32_t u[8];
+          tmem_ld8(o_addr + c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          tmem_st8(o_addr + c, u);
+        }
+      };
+      // bf16: x = s * scale - m, 2^x and the row sum of one 32-key chunk on pairs of values
+      // (packed fp32 instructions), P over the chunk's first 16 columns
+      auto exp_chunk_bf16 = [&](int c, float2 negm) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 p = exp2_pair(__ffma2_rn(make_float2(s[c + 2 * i], s[c + 2 * i + 1]), sl2v, negm), i);
+          rs2[i & 3] = __fadd2_rn(rs2[i & 3], p);
+          pk[i] = pack_bf16(p.x, p.y);
+        }
+        tmem_st16(s_addr + (c >> 1), pk);
+      };
+      {
+      // the whole row of S in one round trip: four loads in flight, one wait
       {
         uint32_t u0[32], u1[32], u2[32], u3[32];
         tmem_ld32(s_addr + 0, u0);
@@ -387,38 +466,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float mx = fmaxf(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], max3(mx8[5], mx8[6], mx8[7])));
       const float m_new = fmaxf(m, mx * sl2);
       const bool need = __any_sync(0xffffffffu, m_new > m + RESCALE_THRESHOLD);
-      float alpha = 1.f;
       if (need) {
         alpha = ex2(m - m_new);   // 0 on the first tile (m = -inf)
         m = m_new;
       }
-      if (need && j > 0) {
-        // O_w was last written by P V of tile j-1, which completed before S_w of tile j; it
-        // is rescaled before any P of tile j is handed to the tensor cores
-#pragma unroll 1
-        for (int c = 0; c < D; c += 8) {  // 8 columns at a time: the row of S is still live
-          uint32_t u[8];
-          tmem_ld8(o_addr + c, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 8; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st8(o_addr + c, u);
-        }
-      }
-      // P of keys [0, c + 32) (and the rescaled O) handed to the MMA thread at the end of
-      // each piece
-      auto hand_piece = [&](int c) {
-        if ((c + 32) % (BN / C::P_PARTS) == 0) {
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[w][(c + 32) / (BN / C::P_PARTS) - 1]));
-        }
-      };
-      float rs8[8];               // row sum in eight independent chains
-#pragma unroll
-      for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
-      const float neg_m = -m;
+      if (need && j > 0) rescale_o();
+      const float2 negm = make_float2(-m, -m);
       if (FP8) {
         // e4m3 P at unit scale, four per tensor-memory column (p <= 2^8 < 448)
 #pragma unroll
@@ -426,14 +479,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            float p[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              p[e] = exp2_mixed(fmaf(s[c + 4 * i + e], sl2, neg_m), 4 * i + e);
-              rs8[(4 * i + e) & 7] += p[e];
-            }
-            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p[0], p[1]), __NV_SATFINITE, __NV_E4M3);
-            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p[2], p[3]), __NV_SATFINITE, __NV_E4M3);
+            const float2 p0 = exp2_pair(__ffma2_rn(make_float2(s[c + 4 * i], s[c + 4 * i + 1]), sl2v, negm), 2 * i);
+            const float2 p1 =
+                exp2_pair(__ffma2_rn(make_float2(s[c + 4 * i + 2], s[c + 4 * i + 3]), sl2v, negm), 2 * i + 1);
+            rs2[(2 * i) & 3] = __fadd2_rn(rs2[(2 * i) & 3], p0);
+            rs2[(2 * i + 1) & 3] = __fadd2_rn(rs2[(2 * i + 1) & 3], p1);
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(p0, __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(p1, __NV_SATFINITE, __NV_E4M3);
             pk[i] = (lo & 0xffffu) | (hi << 16);
           }
           tmem_st8(s_addr + (c >> 2), pk);
@@ -442,20 +494,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
 #pragma unroll
         for (int c = 0; c < BN; c += 32) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = exp2_mixed(fmaf(s[c + 2 * i], sl2, neg_m), 2 * i);
-            const float p1 = exp2_mixed(fmaf(s[c + 2 * i + 1], sl2, neg_m), 2 * i + 1);
-            rs8[(2 * i) & 7] += p0;
-            rs8[(2 * i + 1) & 7] += p1;
-            pk[i] = pack_bf16(p0, p1);
-          }
-          tmem_st16(s_addr + (c >> 1), pk);
+          exp_chunk_bf16(c, negm);
           hand_piece(c);
         }
       }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      }
+      const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+      const float rs = rsa.x + rsa.y;
       l = l * alpha + rs;
     }
     // ------------------------------------------------------------ epilogue
