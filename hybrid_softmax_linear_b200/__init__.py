@@ -17,16 +17,17 @@ import os
 import numpy as np
 
 __all__ = [
-    "VdnError", "Shape", "lib", "F32", "BF16", "E4M3", "ELU1", "DELTA",
+    "VdnError", "Shape", "lib", "F32", "BF16", "E4M3", "E4M3_PROJ", "ELU1", "DELTA",
     "mask_layout_build", "max_groups", "hybrid_attn_workspace_size", "step_workspace_size", "workspace_init",
     "softmax_branch_fwd", "linear_state_build", "linear_state_scan", "linear_read", "hybrid_fuse", "out_proj",
     "hybrid_attn_fwd", "hybrid_attn_host_workspace_size", "hybrid_attn_fwd_host", "hybrid_attn_intermediate", "check_device_status", "debug_unset_flag_wait", "version",
     "profile_begin", "profile_end", "fp8_quant_per_head", "softmax_branch_fwd_noalloc",
+    "out_proj_e4m3", "out_proj_e4m3_workspace_size", "hybrid_attn_fwd_partial",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdn.so")
 
-F32, BF16, E4M3 = 0, 1, 2
+F32, BF16, E4M3, E4M3_PROJ = 0, 1, 2, 3
 ELU1, DELTA = 0, 1
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT", 6: "DEVICE"}
 
@@ -70,8 +71,12 @@ _SIGS = {
                                        _vp]),
     "vdn_hybrid_fuse": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _f32, _vp, _vp]),
     "vdn_out_proj": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "vdn_out_proj_e4m3_workspace_size": (_sz, [_SP]),
+    "vdn_out_proj_e4m3": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "vdn_hybrid_attn_fwd": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                            _i32, _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "vdn_hybrid_attn_fwd_partial": (ctypes.c_int, [_SP, _i32, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
+                                                   _vp, _vp, _vp, _i32, _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "vdn_hybrid_attn_host_workspace_size": (_sz, [_SP, ctypes.c_int, ctypes.c_int]),
     "vdn_hybrid_attn_fwd_host": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                 _vp, _i32, _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -211,6 +216,17 @@ def out_proj(shape, dtype, a, w_os, w_ol, y, ws, stream=None):
                               _nbytes(ws), _stream(stream)))
 
 
+def out_proj_e4m3_workspace_size(shape) -> int:
+    return lib().vdn_out_proj_e4m3_workspace_size(ctypes.byref(Shape.of(shape)))
+
+
+def out_proj_e4m3(shape, a8, a_scales, w_os, w_ol, y, ws, stream=None):
+    """y = A W_os^T + A W_ol^T from e4m3 A codes (uint8 [N_v][2HD]) with per-(branch half,
+    head) scales a_scales float[2][H]; bf16 weights and y."""
+    _check(lib().vdn_out_proj_e4m3(ctypes.byref(Shape.of(shape)), _p(a8), _p(a_scales), _p(w_os), _p(w_ol), _p(y),
+                                   _p(ws), _nbytes(ws), _stream(stream)))
+
+
 def _need(name: str, t, numel: int, esize: int, where: str | None):
     """Checks a torch tensor argument of the whole-layer calls before its pointer is passed:
     the library sees only addresses, so a short or strided buffer would be read or written
@@ -260,6 +276,30 @@ def hybrid_attn_fwd(shape, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_
     _check(lib().vdn_hybrid_attn_fwd(ctypes.byref(Shape.of(shape)), kind, dtype, _p(q), _p(k), _p(v), _p(kt),
                                      _p(vt), _p(beta), _p(w_gate_s), _p(w_gate_l), G_l, _p(gamma), eps, _p(w_os),
                                      _p(w_ol), _p(y), _p(ws), _nbytes(ws), _stream(stream)))
+
+
+def hybrid_attn_fwd_partial(shape, out_features, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma,
+                            eps, w_os, w_ol, y_partial, ws, stream=None):
+    """One rank's share of the head-split layer: shape.heads = this rank's heads, inputs are
+    their slices, w_os/w_ol [out_features][H_r D] bf16, y_partial float [N_v][out_features]."""
+    s = Shape.of(shape)
+    nv, hd = s.frames * s.tokens_per_frame, s.heads * s.head_dim
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(name, t, nv * hd, 2, "device")
+    for name, t in (("kt", kt), ("vt", vt)):
+        _need(name, t, s.text_tokens * hd, 2, "device")
+    _need("beta", beta, s.frames * s.heads, 4, "device")
+    _need("w_gate_s", w_gate_s, hd, 4, "device")
+    if isinstance(G_l, int) and G_l > 0:
+        _need("w_gate_l", w_gate_l, hd * G_l, 4, "device")
+    _need("gamma", gamma, hd, 4, "device")
+    _need("w_os", w_os, out_features * hd, 2, "device")
+    _need("w_ol", w_ol, out_features * hd, 2, "device")
+    _need("y_partial", y_partial, nv * out_features, 4, "device")
+    _check(lib().vdn_hybrid_attn_fwd_partial(ctypes.byref(s), out_features, kind, dtype, _p(q), _p(k), _p(v), _p(kt),
+                                             _p(vt), _p(beta), _p(w_gate_s), _p(w_gate_l), G_l, _p(gamma), eps,
+                                             _p(w_os), _p(w_ol), _p(y_partial), _p(ws), _nbytes(ws),
+                                             _stream(stream)))
 
 
 def hybrid_attn_host_workspace_size(shape, kind: int, dtype: int) -> int:

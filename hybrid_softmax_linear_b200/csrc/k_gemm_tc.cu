@@ -4,12 +4,19 @@
 // projections of the two branches, summed).  One GEMM with K = 2*H*D: the K loop reads
 // W_os for the first H*D columns of A and W_ol for the rest.
 //
-// Persistent, warp-specialised: warp 0 issues TMA loads of 128x64 A and 256x64 W tiles
-// (128-byte swizzle) into a 4-stage ring; one thread of warp 1 issues tcgen05.mma
-// (M=128, N=256, K=16) into one of two 128x256 fp32 accumulators in tensor memory;
-// warps 2-5 drain the other accumulator (tcgen05.ld), round to bf16 and store y, so the
-// epilogue of tile i overlaps the main loop of tile i+1.  Tiles are visited in groups of
-// 16 row blocks so that concurrently running CTAs share A rows and W columns in L2.
+// Persistent, warp-specialised: warp 0 issues TMA loads of 128-row A and 256-row W tiles
+// of 128 bytes per row (64 bf16 or 128 e4m3; 128-byte swizzle) into a 4-stage ring; one
+// thread of warp 1 issues tcgen05.mma (M=128, N=256, K=16 bf16 or K=32 e4m3) into one of
+// two 128x256 fp32 accumulators in tensor memory; warps 2-5 drain the other accumulator
+// (tcgen05.ld), round to bf16 and store y, so the epilogue of tile i overlaps the main
+// loop of tile i+1.  Tiles are visited in groups of 16 row blocks so that concurrently
+// running CTAs share A rows and W columns in L2.
+//
+// e4m3 form (the model card's "Inference with Diffusers" runs every wide Linear in fp8
+// e4m3): A holds e4m3 codes whose dequantisation scale depends only on the column's
+// branch and head; w8_prep folds those scales into a copy of [W_os | W_ol], which it
+// quantises with one scale per output column n (its amax / 448), so that one fp32
+// accumulator sums both halves and the epilogue multiplies column n by that scale.
 #include <mutex>
 
 #include "tc_common.cuh"
@@ -57,11 +64,10 @@ namespace {
 
 using namespace tc;
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, GROUP_M = 16;
-constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BM = 128, BN = 256, BKB = 128, STAGES = 4, GROUP_M = 16;  // BKB: bytes of a K tile row
+constexpr int A_BYTES = BM * BKB, B_BYTES = BN * BKB, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC = idesc_bf16(BM, BN, false, false);
 
 struct alignas(8) Bars {
   uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
@@ -78,10 +84,18 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &m,
   n = idx / gm;
 }
 
+// FP8 = false: bf16 A and W, the K loop switching from W_os (tmW1) to W_ol (tmW2) at HD.
+// FP8 = true: e4m3 A and the prepared e4m3 [W_os | W_ol] copy (tmW1 only); column scales
+// wsc[N] applied in the epilogue.
+template <bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
     out_proj_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW1,
-                       const __grid_constant__ CUtensorMap tmW2, __nv_bfloat16 *__restrict__ y, int M, int N,
-                       int KH, DevStatus *st) {
+                       const __grid_constant__ CUtensorMap tmW2, void *__restrict__ y, int M, int N,
+                       int KH, const float *__restrict__ wsc, int y_f32, DevStatus *st) {
+  constexpr int EB = FP8 ? 1 : 2;          // bytes per element
+  constexpr int BK = BKB / EB;             // K elements per stage
+  constexpr int KSTEP = 32 / EB;           // K elements per MMA (32 bytes of a row)
+  constexpr uint32_t IDESC = FP8 ? idesc_e4m3(BM, BN, false, false) : idesc_bf16(BM, BN, false, false);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t *base = smem_raw + ((1024 - (raw & 1023)) & 1023);
@@ -110,7 +124,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = bars->tmem_base;
 
   const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN, tiles = num_m * num_n;
-  const int ktiles = 2 * KH / BK;
+  const int ktiles = 2 * KH / BK;  // K = 2 * KH elements
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
@@ -126,7 +140,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive_expect_tx(fb, STAGE_BYTES);
         const int kx = kt * BK;
         tma_load_2d(smem_u32(sa + s * A_BYTES), &tmA, fb, kx, m * BM);
-        if (kx < KH) tma_load_2d(smem_u32(sb + s * B_BYTES), &tmW1, fb, kx, n * BN);
+        if (FP8 || kx < KH) tma_load_2d(smem_u32(sb + s * B_BYTES), &tmW1, fb, kx, n * BN);
         else tma_load_2d(smem_u32(sb + s * B_BYTES), &tmW2, fb, kx - KH, n * BN);
         armed |= 1u << s;
         armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
@@ -151,8 +165,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t a0 = smem_u32(sa + s * A_BYTES), b0 = smem_u32(sb + s * B_BYTES);
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k) {
-          mma_ss(d, sdesc(a0 + k * 32, 16, 1024), sdesc(b0 + k * 32, 16, 1024), IDESC, (kt | k) != 0);
+        for (int k = 0; k < BK / KSTEP; ++k) {
+          if (FP8)
+            mma_ss_f8(d, sdesc(a0 + k * 32, 16, 1024), sdesc(b0 + k * 32, 16, 1024), IDESC, (kt | k) != 0);
+          else
+            mma_ss(d, sdesc(a0 + k * 32, 16, 1024), sdesc(b0 + k * 32, 16, 1024), IDESC, (kt | k) != 0);
         }
         mma_commit(smem_u32(&bars->empty[s]));
         if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -178,22 +195,40 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const int row = m * BM + q * 32 + lane;
-      __nv_bfloat16 *yr = y + (int64_t)row * N + n * BN;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c0), r);
         tmem_wait_ld();
         if (row < M && n * BN + c0 < N) {
-          uint4 *dst = reinterpret_cast<uint4 *>(yr + c0);
+          float f[32];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 o;
-            o.x = pack_bf16(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-            o.y = pack_bf16(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-            o.z = pack_bf16(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-            o.w = pack_bf16(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-            dst[v] = o;
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]);
+          if (FP8) {
+            const float4 *sc = reinterpret_cast<const float4 *>(wsc + n * BN + c0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 c = __ldg(sc + i);
+              f[4 * i] *= c.x; f[4 * i + 1] *= c.y; f[4 * i + 2] *= c.z; f[4 * i + 3] *= c.w;
+            }
+          }
+          const int64_t o = (int64_t)row * N + n * BN + c0;
+          if (y_f32) {
+            // float partial sums (the head-sharded layer reduces them across ranks)
+            float4 *dst = reinterpret_cast<float4 *>((float *)y + o);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) dst[v] = make_float4(f[4 * v], f[4 * v + 1], f[4 * v + 2], f[4 * v + 3]);
+          } else {
+            uint4 *dst = reinterpret_cast<uint4 *>((__nv_bfloat16 *)y + o);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w4;
+              w4.x = pack_bf16(f[8 * v + 0], f[8 * v + 1]);
+              w4.y = pack_bf16(f[8 * v + 2], f[8 * v + 3]);
+              w4.z = pack_bf16(f[8 * v + 4], f[8 * v + 5]);
+              w4.w = pack_bf16(f[8 * v + 6], f[8 * v + 7]);
+              dst[v] = w4;
+            }
           }
         }
       }
@@ -209,41 +244,147 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
+
+// w8[n][c] = e4m3(w'[n][c] / wsc[n]) with w'[n][c] = [W_os | W_ol][n][c] * ascale[c / D] (the
+// dequantisation scale of A's column c: its branch half and head) and wsc[n] =
+// max_c |w'[n][c]| / 448 (1 for an all-zero row).  One block per output row.
+__global__ void __launch_bounds__(256) w8_prep_kernel(const __nv_bfloat16 *__restrict__ wos,
+                                                      const __nv_bfloat16 *__restrict__ wol, int HD, int D,
+                                                      const float *__restrict__ ascale, uint8_t *__restrict__ w8,
+                                                      float *__restrict__ wsc) {
+  __shared__ float red[8];
+  const int n = blockIdx.x, tid = threadIdx.x;
+  const int K = 2 * HD;
+  float mx = 0.f;
+  // pass 1: amax of the scaled row (8 elements per step: 16-byte loads of each half)
+  for (int c = tid * 8; c < K; c += 256 * 8) {
+    const __nv_bfloat16 *src = c < HD ? wos + (int64_t)n * HD + c : wol + (int64_t)n * HD + (c - HD);
+    const float sc = ascale[c / D];
+    const uint4 raw = *reinterpret_cast<const uint4 *>(src);
+    const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(hp[e]);
+      mx = fmaxf(mx, fmaxf(fabsf(f.x * sc), fabsf(f.y * sc)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  mx = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) mx = fmaxf(mx, red[i]);
+  const float scale = mx > 0.f ? mx / 448.f : 1.f;
+  const float inv = 1.f / scale;
+  if (tid == 0) wsc[n] = scale;
+  // pass 2: the codes (the row is in L1/L2 from pass 1)
+  for (int c = tid * 8; c < K; c += 256 * 8) {
+    const __nv_bfloat16 *src = c < HD ? wos + (int64_t)n * HD + c : wol + (int64_t)n * HD + (c - HD);
+    const float sc = ascale[c / D] * inv;
+    const uint4 raw = *reinterpret_cast<const uint4 *>(src);
+    const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+    uint32_t q[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float2 f0 = __bfloat1622float2(hp[2 * e]), f1 = __bfloat1622float2(hp[2 * e + 1]);
+      const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f0.x * sc, f0.y * sc), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f1.x * sc, f1.y * sc), __NV_SATFINITE, __NV_E4M3);
+      q[e] = (lo & 0xffffu) | (hi << 16);
+    }
+    *reinterpret_cast<uint2 *>(w8 + (int64_t)n * K + c) = make_uint2(q[0], q[1]);
+  }
+}
+
+// Per-(branch half, head) dequantisation scales of A in the e4m3 layer, from static bounds:
+// A_s = g_s O_s is a gated convex combination of V rows, so |A_s| <= amax(V_h), the e4m3
+// V scale's 448 (its scale is then that of V); A_l = g_l gamma O_l / rms(O_l) has
+// |A_l| <= max|gamma_h| sqrt(D), so its scale is that / 448.
+__global__ void a8_scale_kernel(int H, int D, const float *__restrict__ vscale, const float *__restrict__ gamma,
+                                float *__restrict__ ascale) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= H) return;
+  float g = 0.f;
+  for (int i = 0; i < D; ++i) g = fmaxf(g, fabsf(gamma[(int64_t)h * D + i]));
+  ascale[h] = vscale[h];
+  const float b = g * sqrtf((float)D) / 448.f;
+  ascale[H + h] = b > 0.f ? b : 1.f;
+}
+
 }  // namespace
 
 bool out_proj_tc_supported(const Dims &d) {
   const int HD = d.H * d.D;
-  return HD % BK == 0 && HD % 8 == 0 && HD >= BK;
+  return HD % 64 == 0 && HD % 8 == 0 && HD >= 64;
 }
 
 cudaError_t launch_out_proj_tc(const Dims &d, const void *a, const void *wos, const void *wol, void *y, char *ws,
-                               const WsPlan &p, cudaStream_t st) {
-  const int HD = d.H * d.D;
+                               const WsPlan &p, cudaStream_t st, int n_out, bool y_f32) {
+  const int HD = d.H * d.D;                 // K of each projection (this call's heads)
+  const int N = n_out > 0 ? n_out : HD;     // output features
   const int64_t M = d.Nv();
   CUtensorMap tmA, tmW1, tmW2;
   {
     uint64_t dims[2] = {(uint64_t)(2 * HD), (uint64_t)M}, strides[1] = {(uint64_t)(2 * HD) * 2};
-    uint32_t box[2] = {BK, BM};
+    uint32_t box[2] = {BKB / 2, BM};
     if (!encode_tmap(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
   {
-    uint64_t dims[2] = {(uint64_t)HD, (uint64_t)HD}, strides[1] = {(uint64_t)HD * 2};
-    uint32_t box[2] = {BK, BN};
+    uint64_t dims[2] = {(uint64_t)HD, (uint64_t)N}, strides[1] = {(uint64_t)HD * 2};
+    uint32_t box[2] = {BKB / 2, BN};
     if (!encode_tmap(&tmW1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wos, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_tmap(&tmW2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wol, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(out_proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(out_proj_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int tiles = (int)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  out_proj_tc_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmW1, tmW2, y, (int)M, N, HD, nullptr,
+                                                               y_f32 ? 1 : 0, (DevStatus *)(ws + p.status));
+  return cudaGetLastError();
+}
+
+bool out_proj_e4m3_supported(const Dims &d) {
+  const int HD = d.H * d.D;
+  return HD % 256 == 0 && HD >= 256;
+}
+
+cudaError_t launch_a8_scales(const Dims &d, const float *vscale, const float *gamma, float *ascale, cudaStream_t st) {
+  a8_scale_kernel<<<(d.H + 127) / 128, 128, 0, st>>>(d.H, d.D, vscale, gamma, ascale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_out_proj_e4m3(const Dims &d, const void *a8, const float *ascale, const void *wos, const void *wol,
+                                 void *y, uint8_t *w8, float *wsc, DevStatus *status, cudaStream_t st) {
+  const int HD = d.H * d.D;
+  const int64_t M = d.Nv();
+  w8_prep_kernel<<<HD, 256, 0, st>>>((const __nv_bfloat16 *)wos, (const __nv_bfloat16 *)wol, HD, d.D, ascale, w8, wsc);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap tmA, tmW;
+  {
+    uint64_t dims[2] = {(uint64_t)(2 * HD), (uint64_t)M}, strides[1] = {(uint64_t)(2 * HD)};
+    uint32_t box[2] = {BKB, BM};
+    if (!encode_tmap(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a8, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t dims[2] = {(uint64_t)(2 * HD), (uint64_t)HD}, strides[1] = {(uint64_t)(2 * HD)};
+    uint32_t box[2] = {BKB, BN};
+    if (!encode_tmap(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w8, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  e = cudaFuncSetAttribute(out_proj_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int tiles = (int)((M + BM - 1) / BM) * ((HD + BN - 1) / BN);
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  out_proj_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmW1, tmW2, (__nv_bfloat16 *)y, (int)M, HD, HD,
-                                                        (DevStatus *)(ws + p.status));
+  out_proj_tc_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmW, tmW, y, (int)M, HD, HD, wsc, 0, status);
   return cudaGetLastError();
 }
 

@@ -25,9 +25,6 @@ namespace {
 using namespace tc;
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 
 // 16-byte chunk `cl` (8 bf16 of columns 8cl..8cl+7) of row r in a tile stored as
 // 64-column boxes of `box_rows` rows with the 128-byte swizzle
@@ -286,6 +283,7 @@ constexpr size_t SMEM = 1024 + BAR_OFF + sizeof(Bars);
 // Output rows are staged in shared memory (over Q and S, free once num is complete) with a
 // 16-byte pad per row, then written out two whole rows per warp instruction.
 constexpr int OUT_PITCH = D * 2 + 16;
+constexpr int OUT_PITCH8 = D + 16;  // e4m3 output rows
 static_assert(BM * OUT_PITCH <= 2 * TILE_BYTES, "output staging must fit over Q and S");
 }  // namespace rd
 
@@ -310,7 +308,8 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
     read_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                    const __grid_constant__ CUtensorMap tmW, Dims d, const float *__restrict__ zsum,
                    const float *__restrict__ wgl, int G_l, const float *__restrict__ gamma, float eps,
-                   __nv_bfloat16 *__restrict__ out, int64_t out_stride, const int32_t *__restrict__ tiles,
+                   void *__restrict__ out, int64_t out_stride, const int32_t *__restrict__ tiles,
+                   const float *__restrict__ a8_scale,
                    DevStatus *st) {
   using namespace rd;
   constexpr bool delta = DELTA, fused = FUSED, gate_mma = FUSED && GATE_MMA;
@@ -489,7 +488,10 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
     const float rinv = fused ? rsqrtf((bars->part[2][0][r] + bars->part[2][1][r]) / (float)D + eps) : 1.f;
     const float f_row = scale * rinv;  // o / rms(o) = num * scale * rinv
     const float gs = fast_sigmoid(g1_row);
-    uint8_t *srow = stage + r * OUT_PITCH + c0 * 2;
+    // e4m3 output (fused only): codes of A_l in units of its per-head scale a8_scale[h]
+    const bool out8 = fused && a8_scale != nullptr;
+    const float f_out = out8 ? f_row / a8_scale[h] : f_row;
+    uint8_t *srow = stage + (out8 ? r * OUT_PITCH8 + c0 : r * OUT_PITCH + c0 * 2);
 #pragma unroll
     for (int c = 0; c < HC; c += 32) {
       uint32_t u[32], ug[32];
@@ -506,23 +508,45 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float gl = gate_mma ? gate_sigmoid(__uint_as_float(ug[v + e])) : gs;
-            o8[e] = gl * gg[e] * (__uint_as_float(u[v + e]) * f_row);
+            o8[e] = gl * gg[e] * (__uint_as_float(u[v + e]) * f_out);
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o8[e] = __uint_as_float(u[v + e]) * f_row;
+          for (int e = 0; e < 8; ++e) o8[e] = __uint_as_float(u[v + e]) * f_out;
         }
-        *reinterpret_cast<uint4 *>(srow + (c + v) * 2) = pack8(o8);
+        if (out8) {
+          uint32_t w2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(o8[4 * e], o8[4 * e + 1]), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi =
+                __nv_cvt_float2_to_fp8x2(make_float2(o8[4 * e + 2], o8[4 * e + 3]), __NV_SATFINITE, __NV_E4M3);
+            w2[e] = (lo & 0xffffu) | (hi << 16);
+          }
+          *reinterpret_cast<uint2 *>(srow + c + v) = make_uint2(w2[0], w2[1]);
+        } else {
+          *reinterpret_cast<uint4 *>(srow + (c + v) * 2) = pack8(o8);
+        }
       }
     }
   }
   __syncthreads();
   if (ok) {
-    // two rows per warp instruction: lanes 0-15 one row, 16-31 the next (256 bytes each)
     const int nrows = min(BM, row_end - row0);
-    for (int rr = warp * 2 + (lane >> 4); rr < nrows; rr += 2 * (THREADS / 32)) {
-      const uint4 val = *reinterpret_cast<const uint4 *>(stage + rr * OUT_PITCH + (lane & 15) * 16);
-      *reinterpret_cast<uint4 *>(out + (int64_t)(row0 + rr) * out_stride + (int64_t)h * D + (lane & 15) * 8) = val;
+    if (fused && a8_scale != nullptr) {
+      // four rows per warp instruction: eight lanes per 128-byte row
+      for (int rr = warp * 4 + (lane >> 3); rr < nrows; rr += 4 * (THREADS / 32)) {
+        const uint4 val = *reinterpret_cast<const uint4 *>(stage + rr * OUT_PITCH8 + (lane & 7) * 16);
+        *reinterpret_cast<uint4 *>((uint8_t *)out + (int64_t)(row0 + rr) * out_stride + (int64_t)h * D +
+                                   (lane & 7) * 16) = val;
+      }
+    } else {
+      // two rows per warp instruction: lanes 0-15 one row, 16-31 the next (256 bytes each)
+      for (int rr = warp * 2 + (lane >> 4); rr < nrows; rr += 2 * (THREADS / 32)) {
+        const uint4 val = *reinterpret_cast<const uint4 *>(stage + rr * OUT_PITCH + (lane & 15) * 16);
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)out + (int64_t)(row0 + rr) * out_stride + (int64_t)h * D +
+                                   (lane & 15) * 8) = val;
+      }
     }
   }
   // ---- drain: no copy or MMA of this block may be in flight when it exits
@@ -585,7 +609,8 @@ cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf,
 }
 
 cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void *out, const float *wgl, int G_l,
-                           const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st) {
+                           const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st,
+                           const float *a8_scale) {
   using namespace rd;
   const uint64_t HD = (uint64_t)d.H * D;
   const int G = host_group_count(d);
@@ -610,7 +635,9 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
       return cudaErrorInvalidValue;
   }
   const int64_t stride = fused ? 2 * (int64_t)HD : (int64_t)HD;
-  __nv_bfloat16 *o = (__nv_bfloat16 *)out + (fused ? HD : 0);  // fused: the linear half of A
+  // fused: the linear half of A (bf16, or e4m3 codes with a8_scale)
+  void *o = (a8_scale != nullptr) ? (void *)((uint8_t *)out + HD) : (void *)((__nv_bfloat16 *)out + (fused ? HD : 0));
+  if (a8_scale != nullptr && !fused) return cudaErrorInvalidValue;
   const unsigned grid = (unsigned)(2 * host_tile_count(d) * d.H);
   const float *zs = (const float *)(ws + p.zsum);
   const int32_t *tl = (const int32_t *)(ws + p.tiles);
@@ -619,7 +646,8 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<grid, THREADS, SMEM, st>>>(mq, ms, mw, d, zs, fused ? wgl : nullptr, G_l, gamma, eps, o, stride, tl, sp);
+    kern<<<grid, THREADS, SMEM, st>>>(mq, ms, mw, d, zs, fused ? wgl : nullptr, G_l, gamma, eps, o, stride, tl,
+                                      a8_scale, sp);
     return cudaGetLastError();
   };
   if (delta) {

@@ -514,7 +514,14 @@ __global__ void __launch_bounds__(256) scan_delta_small_kernel(Dims d, const flo
 // S_fwd = S_txt/2 + prefix[ie_g], S_bwd = S_txt/2 + suffix[ib_g].  With SUM the block
 // stores S_fwd + S_bwd in bf16 and z_fwd + z_bwd in float, the operands of the
 // tensor-core read, instead of the four float memories.
-constexpr int SCAN_THREADS = 256;
+#ifndef VDN_SCAN_THREADS
+#define VDN_SCAN_THREADS 256
+#endif
+#ifndef VDN_SCAN_INFLIGHT
+#define VDN_SCAN_INFLIGHT 8
+#endif
+constexpr int SCAN_THREADS = VDN_SCAN_THREADS;
+constexpr int SCAN_INFLIGHT = VDN_SCAN_INFLIGHT;  // frames a lane loads per round trip
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -553,15 +560,19 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_seg_kernel(Dims d, const fl
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     if (valid) {
       const int hi = bnd[j + 1];
-      // eight frames per round trip: a segment of up to eight frames costs one memory latency
-      for (int f = bnd[j]; f < hi; f += 8) {
-        float4 x[8];
+      // SCAN_INFLIGHT frames per round trip: a segment of up to that many frames costs one
+      // memory latency
+      for (int f = bnd[j]; f < hi; f += SCAN_INFLIGHT) {
+        float4 x[SCAN_INFLIGHT];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int k = 0; k < SCAN_INFLIGHT; ++k)
           x[k] = f + k < hi ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(f + k) * fstride))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        a = f4add(a, f4add(f4add(x[0], x[1]), f4add(x[2], x[3])));
-        b = f4add(b, f4add(f4add(x[4], x[5]), f4add(x[6], x[7])));
+#pragma unroll
+        for (int k = 0; k < SCAN_INFLIGHT; k += 2) {
+          a = f4add(a, x[k]);
+          b = f4add(b, x[k + 1]);
+        }
       }
     }
     seg[j * 32 + lane] = f4add(a, b);

@@ -174,9 +174,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     softmax_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
                       const __grid_constant__ CUtensorMap tmVt, Dims d, float sl2, const float *__restrict__ scales,
-                      __nv_bfloat16 *__restrict__ out, int64_t out_row_stride, const float *__restrict__ w_gate_s,
+                      void *__restrict__ out, int64_t out_row_stride, const float *__restrict__ w_gate_s,
                       float *__restrict__ lse, const int32_t *__restrict__ gtab, const int32_t *__restrict__ tiles,
-                      DevStatus *st) {
+                      int out8, DevStatus *st) {
   using C = Cfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -545,22 +545,51 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (FP8) dot *= scales[h];  // s_q
         inv *= 1.f / (1.f + expf(-dot));
       }
-      __nv_bfloat16 *orow = out + (int64_t)row * out_row_stride + (int64_t)h * D;
+      if (out8) {
+        // e4m3 codes of g_s O / l in units of the V scale, which is then A_s's dequantisation
+        // scale: |g_s O| <= amax(V), so the codes stay within e4m3's 448
+        const float inv8 = inv / out_scale;
+        uint8_t *orow = (uint8_t *)out + (int64_t)row * out_row_stride + (int64_t)h * D;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(o_addr + c, u);
-        tmem_wait_ld();
-        if (valid) {
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
+        for (int c = 0; c < D; c += 32) {
+          uint32_t u[32];
+          tmem_ld32(o_addr + c, u);
+          tmem_wait_ld();
+          if (valid) {
+            uint32_t w4[8];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 o;
-            o.x = pack_bf16(__uint_as_float(u[8 * v + 0]) * inv, __uint_as_float(u[8 * v + 1]) * inv);
-            o.y = pack_bf16(__uint_as_float(u[8 * v + 2]) * inv, __uint_as_float(u[8 * v + 3]) * inv);
-            o.z = pack_bf16(__uint_as_float(u[8 * v + 4]) * inv, __uint_as_float(u[8 * v + 5]) * inv);
-            o.w = pack_bf16(__uint_as_float(u[8 * v + 6]) * inv, __uint_as_float(u[8 * v + 7]) * inv);
-            dst[v] = o;
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+                  make_float2(__uint_as_float(u[4 * i]) * inv8, __uint_as_float(u[4 * i + 1]) * inv8), __NV_SATFINITE,
+                  __NV_E4M3);
+              const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+                  make_float2(__uint_as_float(u[4 * i + 2]) * inv8, __uint_as_float(u[4 * i + 3]) * inv8),
+                  __NV_SATFINITE, __NV_E4M3);
+              w4[i] = (lo & 0xffffu) | (hi << 16);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
+            dst[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            dst[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
+          }
+        }
+      } else {
+        __nv_bfloat16 *orow = (__nv_bfloat16 *)out + (int64_t)row * out_row_stride + (int64_t)h * D;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t u[32];
+          tmem_ld32(o_addr + c, u);
+          tmem_wait_ld();
+          if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 o;
+              o.x = pack_bf16(__uint_as_float(u[8 * v + 0]) * inv, __uint_as_float(u[8 * v + 1]) * inv);
+              o.y = pack_bf16(__uint_as_float(u[8 * v + 2]) * inv, __uint_as_float(u[8 * v + 3]) * inv);
+              o.z = pack_bf16(__uint_as_float(u[8 * v + 4]) * inv, __uint_as_float(u[8 * v + 5]) * inv);
+              o.w = pack_bf16(__uint_as_float(u[8 * v + 6]) * inv, __uint_as_float(u[8 * v + 7]) * inv);
+              dst[v] = o;
+            }
           }
         }
       }
@@ -576,7 +605,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 template <int D, bool FP8>
 cudaError_t launch_t(const Dims &d, const void *q, const void *k, const void *v, const void *kt, const void *vt,
                      const float *scales, float sl2, void *o, int64_t o_row_stride, const float *w_gate_s,
-                     float *lse, char *ws, const WsPlan &p, cudaStream_t st) {
+                     float *lse, char *ws, const WsPlan &p, cudaStream_t st, bool out8 = false) {
   using C = Cfg<D, FP8>;
   const uint64_t HD = (uint64_t)d.H * D;
   const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -592,13 +621,13 @@ cudaError_t launch_t(const Dims &d, const void *q, const void *k, const void *v,
       !encode_tmap(&mkt, dt, 2, kt_base, dims_t, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap(&mvt, dt, 2, vt_base, dims_t, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  const int ntiles = host_tile_count(d);
   cudaError_t e = cudaFuncSetAttribute(softmax_tc_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::SMEM);
   if (e != cudaSuccess) return e;
-  const int ntiles = host_tile_count(d);
   softmax_tc_kernel<D, FP8><<<ntiles * d.H, THREADS, C::SMEM, st>>>(
-      mq, mk, mv, mkt, mvt, d, sl2, scales, (__nv_bfloat16 *)o, o_row_stride, w_gate_s, lse,
-      (const int32_t *)(ws + p.gtab), (const int32_t *)(ws + p.tiles), (DevStatus *)(ws + p.status));
+      mq, mk, mv, mkt, mvt, d, sl2, scales, o, o_row_stride, w_gate_s, lse, (const int32_t *)(ws + p.gtab),
+      (const int32_t *)(ws + p.tiles), out8 ? 1 : 0, (DevStatus *)(ws + p.status));
   return cudaGetLastError();
 }
 
@@ -622,10 +651,11 @@ cudaError_t launch_softmax_tc(const Dims &d, vdn_dtype dt, const void *q, const 
 
 cudaError_t launch_softmax_tc_gated(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
                                     const void *kt, const void *vt, const float *scales, const float *w_gate_s,
-                                    float sl2, void *a, char *ws, const WsPlan &p, cudaStream_t st) {
+                                    float sl2, void *a, char *ws, const WsPlan &p, cudaStream_t st, bool a8) {
   const int64_t stride = 2 * (int64_t)d.H * d.D;  // A = [A_s | A_l]: the softmax half of each row
   if (dt == VDN_E4M3 && d.D == 128)
-    return launch_t<128, true>(d, q, k, v, kt, vt, scales, sl2, a, stride, w_gate_s, nullptr, ws, p, st);
+    return launch_t<128, true>(d, q, k, v, kt, vt, scales, sl2, a, stride, w_gate_s, nullptr, ws, p, st, a8);
+  if (a8) return cudaErrorInvalidValue;
   if (dt != VDN_BF16) return cudaErrorInvalidValue;
   if (d.D == 128) return launch_t<128, false>(d, q, k, v, kt, vt, nullptr, sl2, a, stride, w_gate_s, nullptr, ws, p, st);
   if (d.D == 64) return launch_t<64, false>(d, q, k, v, kt, vt, nullptr, sl2, a, stride, w_gate_s, nullptr, ws, p, st);

@@ -372,14 +372,20 @@ vdn_status vdn_out_proj(const vdn_shape *shape, vdn_dtype dtype, const void *a, 
   return ok();
 }
 
-vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *q,
-                               const void *k, const void *v, const void *kt, const void *vt, const float *beta,
-                               const float *w_gate_s, const float *w_gate_l, int32_t G_l, const float *gamma,
-                               float eps, const void *w_os, const void *w_ol, void *y, void *ws, size_t ws_bytes,
-                               vdn_stream stream) {
+}  // extern "C"
+
+namespace {
+// The layer for this call's heads.  n_out = 0: y [N_v][HD] in the activation dtype (the
+// whole layer).  n_out > 0: W_os, W_ol [n_out][HD] are these heads' input columns of a
+// projection with n_out outputs, and y [N_v][n_out] receives float partial sums (the
+// head-sharded layer; tensor-core path only).
+vdn_status layer_impl(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *q, const void *k,
+                      const void *v, const void *kt, const void *vt, const float *beta, const float *w_gate_s,
+                      const float *w_gate_l, int32_t G_l, const float *gamma, float eps, const void *w_os,
+                      const void *w_ol, void *y, void *ws, size_t ws_bytes, vdn_stream stream, int32_t n_out) {
   VDN_TRY(check_shape(shape));
   VDN_TRY(check_kind(kind));
-  if (dtype != VDN_F32 && dtype != VDN_BF16 && dtype != VDN_E4M3)
+  if (dtype != VDN_F32 && dtype != VDN_BF16 && !dtype_e4m3_softmax(dtype))
     return fail(VDN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   VDN_TRY(need(q, "q")); VDN_TRY(need(k, "k")); VDN_TRY(need(v, "v")); VDN_TRY(need(y, "y"));
   if (shape->text_tokens > 0) { VDN_TRY(need(kt, "kt")); VDN_TRY(need(vt, "vt")); }
@@ -389,15 +395,24 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
   else if (beta != nullptr) return fail(VDN_ERR_INVALID_ARG, "beta must be NULL for VDN_LIN_ELU1");
   if (G_l != 1 && G_l != shape->head_dim) return fail(VDN_ERR_INVALID_ARG, "G_l must be 1 or D");
   if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(VDN_ERR_INVALID_ARG, "eps must be finite and >= 0");
-  if (dtype == VDN_E4M3 && (shape->head_dim != 128 || (int64_t)shape->heads * shape->head_dim > FP8_MAX_HD))
+  if (dtype_e4m3_softmax(dtype) && (shape->head_dim != 128 || (int64_t)shape->heads * shape->head_dim > FP8_MAX_HD))
     return fail(VDN_ERR_UNSUPPORTED, "the e4m3 layer needs head_dim 128 and H*D <= %d", FP8_MAX_HD);
+  if (dtype_e4m3_proj(dtype) && !out_proj_e4m3_supported(dims_of(*shape)))
+    return fail(VDN_ERR_UNSUPPORTED, "the e4m3 projection needs H*D a multiple of 256");
+  if (n_out > 0) {
+    if (dtype_e4m3_proj(dtype) || !layer_fused(*shape, dtype) || !out_proj_tc_supported(dims_of(*shape)))
+      return fail(VDN_ERR_UNSUPPORTED, "the partial layer runs bf16 or e4m3-softmax layers with head_dim 128");
+    if (n_out % 32 != 0) return fail(VDN_ERR_INVALID_ARG, "out_features must be a multiple of 32");
+  }
   const WsPlan p = plan_workspace(*shape, kind, dtype);
   VDN_TRY(check_ws(ws, ws_bytes, p.total));
   VDN_TRY(check_device());
   const Dims d = dims_of(*shape);
   cudaStream_t st = (cudaStream_t)stream;
   char *w = (char *)ws;
-  const vdn_dtype act = dtype == VDN_E4M3 ? VDN_BF16 : dtype;
+  const vdn_dtype act = dtype_e4m3_softmax(dtype) ? VDN_BF16 : dtype;
+  const bool a8 = dtype_e4m3_proj(dtype);  // A in e4m3 for the e4m3 projection
+  float *ascale = a8 ? (float *)(w + p.ascale) : nullptr;
   float *S = (float *)(w + p.S), *z = (float *)(w + p.z), *St = (float *)(w + p.St), *zt = (float *)(w + p.zt);
   float *Sf = (float *)(w + p.Sf), *Sb = (float *)(w + p.Sb), *zf = (float *)(w + p.zf), *zb = (float *)(w + p.zb);
   void *Os = w + p.Os, *Ol = w + p.Ol, *A = w + p.A;
@@ -422,17 +437,21 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
       ProfScope ps(K_READ_STAGE, st);
       VDN_CUDA(launch_read_stage(d, kind, seg ? nullptr : Sf, Sb, zf, zb, w_gate_l, G_l, w, p, st), "read staging");
     }
-    if (dtype == VDN_E4M3) {
+    if (dtype_e4m3_softmax(dtype)) {
       // per-head e4m3 Q/K/V for the softmax branch; the linear branch keeps the bf16 inputs
       {
         ProfScope ps(K_QUANT, st);
         VDN_CUDA(launch_fp8_quant(d, q, k, v, kt, vt, w + p.q8, w + p.k8, w + p.v8, w + p.kt8, w + p.vt8,
                                   (float *)(w + p.scales), (uint32_t *)(w + p.amax), st),
                  "fp8 quantisation launch");
+        if (a8)
+          VDN_CUDA(launch_a8_scales(d, (const float *)(w + p.scales) + 2 * d.H, gamma, ascale, st),
+                   "A scale launch");
       }
       ProfScope ps(K_SOFTMAX_TC, st);
       VDN_CUDA(launch_softmax_tc_gated(d, VDN_E4M3, w + p.q8, w + p.k8, w + p.v8, w + p.kt8, w + p.vt8,
-                                       (const float *)(w + p.scales), w_gate_s, scale_log2_of(0.f, d.D), A, w, p, st),
+                                       (const float *)(w + p.scales), w_gate_s, scale_log2_of(0.f, d.D), A, w, p, st,
+                                       a8),
                "softmax branch (tensor cores, e4m3) launch");
     } else {
       ProfScope ps(K_SOFTMAX_TC, st);
@@ -442,7 +461,8 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
     }
     {
       ProfScope ps(K_READ_TC, st);
-      VDN_CUDA(launch_read_tc(d, kind, q, A, w_gate_l, G_l, gamma, eps, w, p, st), "read launch");
+      VDN_CUDA(launch_read_tc(d, kind, q, A, w_gate_l, G_l, gamma, eps, w, p, st, a8 ? ascale + d.H : nullptr),
+               "read launch");
     }
   } else {
     VDN_TRY(softmax_dispatch(d, dtype, q, k, v, kt, vt, nullptr, scale_log2_of(0.f, d.D), Os, nullptr, w, p, st));
@@ -461,7 +481,82 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dt
       VDN_CUDA(launch_fuse(d, act, q, Os, Ol, w_gate_s, w_gate_l, G_l, gamma, eps, A, st), "fuse launch");
     }
   }
-  VDN_TRY(out_proj_dispatch(d, act, A, w_os, w_ol, y, w, p, st));
+  if (a8) {
+    ProfScope ps(K_GEMM_TC, st);
+    VDN_CUDA(launch_out_proj_e4m3(d, A, ascale, w_os, w_ol, y, (uint8_t *)(w + p.w8), (float *)(w + p.wsc),
+                                  (DevStatus *)(w + p.status), st),
+             "out-proj (tensor cores, e4m3) launch");
+  } else if (n_out > 0) {
+    ProfScope ps(K_GEMM_TC, st);
+    VDN_CUDA(launch_out_proj_tc(d, A, w_os, w_ol, y, w, p, st, n_out, true), "out-proj (tensor cores) launch");
+  } else {
+    VDN_TRY(out_proj_dispatch(d, act, A, w_os, w_ol, y, w, p, st));
+  }
+  return ok();
+}
+}  // namespace
+
+extern "C" {
+
+vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *q,
+                               const void *k, const void *v, const void *kt, const void *vt, const float *beta,
+                               const float *w_gate_s, const float *w_gate_l, int32_t G_l, const float *gamma,
+                               float eps, const void *w_os, const void *w_ol, void *y, void *ws, size_t ws_bytes,
+                               vdn_stream stream) {
+  return layer_impl(shape, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma, eps, w_os, w_ol, y,
+                    ws, ws_bytes, stream, 0);
+}
+
+vdn_status vdn_hybrid_attn_fwd_partial(const vdn_shape *shape, int32_t out_features, vdn_lin_kind kind,
+                                       vdn_dtype dtype, const void *q, const void *k, const void *v, const void *kt,
+                                       const void *vt, const float *beta, const float *w_gate_s,
+                                       const float *w_gate_l, int32_t G_l, const float *gamma, float eps,
+                                       const void *w_os, const void *w_ol, float *y_partial, void *ws,
+                                       size_t ws_bytes, vdn_stream stream) {
+  if (out_features < 1) return fail(VDN_ERR_INVALID_ARG, "out_features must be >= 1");
+  return layer_impl(shape, kind, dtype, q, k, v, kt, vt, beta, w_gate_s, w_gate_l, G_l, gamma, eps, w_os, w_ol,
+                    y_partial, ws, ws_bytes, stream, out_features);
+}
+
+namespace {
+// workspace of vdn_out_proj_e4m3: status word, the e4m3 weight copy, its column scales
+struct ProjE4m3Plan {
+  size_t status, w8, wsc, total;
+};
+ProjE4m3Plan plan_proj_e4m3(const vdn_shape &s) {
+  ProjE4m3Plan pp{};
+  const size_t hd = (size_t)s.heads * s.head_dim;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+  pp.status = take(256);
+  pp.w8 = take(hd * 2 * hd);
+  pp.wsc = take(hd * 4);
+  pp.total = off;
+  return pp;
+}
+}  // namespace
+
+size_t vdn_out_proj_e4m3_workspace_size(const vdn_shape *shape) {
+  if (check_shape(shape) != VDN_OK) return 0;
+  return plan_proj_e4m3(*shape).total;
+}
+
+vdn_status vdn_out_proj_e4m3(const vdn_shape *shape, const void *a8, const float *a_scales, const void *w_os,
+                             const void *w_ol, void *y, void *ws, size_t ws_bytes, vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  VDN_TRY(need(a8, "a8")); VDN_TRY(need(a_scales, "a_scales")); VDN_TRY(need(w_os, "w_os"));
+  VDN_TRY(need(w_ol, "w_ol")); VDN_TRY(need(y, "y"));
+  const Dims d = dims_of(*shape);
+  if (!out_proj_e4m3_supported(d)) return fail(VDN_ERR_UNSUPPORTED, "the e4m3 projection needs H*D a multiple of 256");
+  const ProjE4m3Plan pp = plan_proj_e4m3(*shape);
+  VDN_TRY(check_ws(ws, ws_bytes, pp.total));
+  VDN_TRY(check_device());
+  char *w = (char *)ws;
+  cudaStream_t st = (cudaStream_t)stream;
+  ProfScope ps(K_GEMM_TC, st);
+  VDN_CUDA(launch_out_proj_e4m3(d, a8, a_scales, w_os, w_ol, y, (uint8_t *)(w + pp.w8), (float *)(w + pp.wsc),
+                                (DevStatus *)(w + pp.status), st),
+           "out-proj (tensor cores, e4m3) launch");
   return ok();
 }
 
@@ -501,7 +596,7 @@ vdn_status vdn_hybrid_attn_fwd_host(const vdn_shape *shape, vdn_lin_kind kind, v
                                     vdn_stream stream) {
   VDN_TRY(check_shape(shape));
   VDN_TRY(check_kind(kind));
-  if (dtype != VDN_F32 && dtype != VDN_BF16 && dtype != VDN_E4M3)
+  if (dtype != VDN_F32 && dtype != VDN_BF16 && !dtype_e4m3_softmax(dtype))
     return fail(VDN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   const bool text = shape->text_tokens > 0;
   if (q_host == nullptr || k_host == nullptr || v_host == nullptr || y_host == nullptr ||

@@ -152,13 +152,17 @@ struct WsPlan {
   // normaliser, linear-gate weights in bf16
   size_t ssum, zsum, wl, stage_end;
   // layer part
-  size_t S, z, St, zt, Sf, Sb, zf, zb, Os, Ol, A, q8, k8, v8, kt8, vt8, scales, amax, total;
+  size_t S, z, St, zt, Sf, Sb, zf, zb, Os, Ol, A, q8, k8, v8, kt8, vt8, scales, amax, ascale, w8, wsc, total;
 };
+
+// e4m3 softmax branch (VDN_E4M3 and VDN_E4M3_PROJ); e4m3 output projection as well
+inline bool dtype_e4m3_softmax(vdn_dtype dt) { return dt == VDN_E4M3 || dt == VDN_E4M3_PROJ; }
+inline bool dtype_e4m3_proj(vdn_dtype dt) { return dt == VDN_E4M3_PROJ; }
 
 // The whole layer runs on the tensor-core path (softmax and linear read write A
 // directly; O_s and O_l are never stored) for bf16 activations with D = 128.
 inline bool layer_fused(const vdn_shape &s, vdn_dtype dtype) {
-  return (dtype == VDN_BF16 || dtype == VDN_E4M3) && s.head_dim == 128;
+  return (dtype == VDN_BF16 || dtype_e4m3_softmax(dtype)) && s.head_dim == 128;
 }
 
 // Number of scan segments of a layout (the same rule the tables kernel applies).
@@ -221,8 +225,9 @@ inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dt
   p.zb = take(Gm * H * D * 4);
   p.Os = take(fused ? 0 : Nv * H * D * act);
   p.Ol = take(fused ? 0 : Nv * H * D * act);
-  p.A = take(Nv * 2 * H * D * act);
-  if (dtype == VDN_E4M3) {
+  // A: bf16 (or float), or e4m3 codes when the projection runs in e4m3
+  p.A = take(Nv * 2 * H * D * (dtype_e4m3_proj(dtype) ? 1 : act));
+  if (dtype_e4m3_softmax(dtype)) {
     p.q8 = take(Nv * H * D);
     p.k8 = take(Nv * H * D);
     p.v8 = take(Nv * H * D);
@@ -230,6 +235,11 @@ inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dt
     p.vt8 = take(L * H * D + 16);
     p.scales = take(3 * H * 4);
     p.amax = take(3 * H * 4);
+  }
+  if (dtype_e4m3_proj(dtype)) {
+    p.ascale = take(2 * H * 4);          // A's dequantisation scales per (branch half, head)
+    p.w8 = take(H * D * 2 * H * D);      // e4m3 [W_os | W_ol] with A's scales folded in
+    p.wsc = take(H * D * 4);             // its per-output-column scales
   }
   p.total = off;
   return p;
@@ -344,11 +354,14 @@ cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf,
                               const float *zb, const float *wgl, int G_l, char *ws, const WsPlan &p,
                               cudaStream_t st);
 // o_l (plain) or, with gate weights, A_l = g_l * gamma * RMSNorm(o_l) into the linear half of A
+// a8_scale (fused only): A_l written as e4m3 codes in units of a8_scale[h]
 cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void *out, const float *wgl, int G_l,
-                           const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st);
+                           const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st,
+                           const float *a8_scale = nullptr);
+// a8: A_s written as e4m3 codes in units of the V scale (e4m3 softmax only)
 cudaError_t launch_softmax_tc_gated(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
                                     const void *kt, const void *vt, const float *scales, const float *w_gate_s,
-                                    float sl2, void *a, char *ws, const WsPlan &p, cudaStream_t st);
+                                    float sl2, void *a, char *ws, const WsPlan &p, cudaStream_t st, bool a8 = false);
 // per-head e4m3 quantisation of q, k (+ text), v (+ text); scales float[3][H]
 cudaError_t launch_fp8_quant(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
                              const void *vt, void *q8, void *k8, void *v8, void *kt8, void *vt8, float *scales,
@@ -360,9 +373,17 @@ cudaError_t launch_fuse(const Dims &d, vdn_dtype dt, const void *q, const void *
                         cudaStream_t st);
 cudaError_t launch_out_proj_simt(const Dims &d, vdn_dtype dt, const void *a, const void *wos, const void *wol,
                                  void *y, cudaStream_t st);
+// n_out > 0: W_os, W_ol [n_out][H D] (this call's heads' input columns of a wider
+// projection) and y [N_v][n_out]; y_f32: float output (partial sums of the head split)
 cudaError_t launch_out_proj_tc(const Dims &d, const void *a, const void *wos, const void *wol, void *y,
-                               char *ws, const WsPlan &p, cudaStream_t st);
+                               char *ws, const WsPlan &p, cudaStream_t st, int n_out = 0, bool y_f32 = false);
 bool out_proj_tc_supported(const Dims &d);
+// e4m3 projection: A8 [N_v][2HD] codes with dequantisation scales ascale[2][H] (per branch
+// half and head), bf16 W_os, W_ol; w8 (HD x 2HD bytes) and wsc (HD floats) are scratch
+bool out_proj_e4m3_supported(const Dims &d);
+cudaError_t launch_a8_scales(const Dims &d, const float *vscale, const float *gamma, float *ascale, cudaStream_t st);
+cudaError_t launch_out_proj_e4m3(const Dims &d, const void *a8, const float *ascale, const void *wos, const void *wol,
+                                 void *y, uint8_t *w8, float *wsc, DevStatus *status, cudaStream_t st);
 cudaError_t launch_debug_wait(char *ws, uint32_t max_polls, cudaStream_t st);
 
 }  // namespace vdn

@@ -57,7 +57,9 @@ typedef int vdn_status;
 #define VDN_ERR_TIMEOUT 5       /* a device wait hit its bound (vdn_check_device_status) */
 #define VDN_ERR_DEVICE 6        /* a device-side check failed (vdn_check_device_status) */
 
-typedef enum { VDN_F32 = 0, VDN_BF16 = 1, VDN_E4M3 = 2 } vdn_dtype;
+/* VDN_E4M3: bf16 tensors, softmax branch in e4m3.  VDN_E4M3_PROJ: the same, and the
+ * output projections in e4m3 too (whole layer and vdn_out_proj_e4m3 only). */
+typedef enum { VDN_F32 = 0, VDN_BF16 = 1, VDN_E4M3 = 2, VDN_E4M3_PROJ = 3 } vdn_dtype;
 
 /* Linear branch kind.  ELU1: phi = elu+1 linear attention with a normaliser ([ART]
  * 局部精确计算 para. 1-3).  DELTA: delta-rule state over frame-mean keys/values
@@ -232,12 +234,33 @@ VDN_API vdn_status vdn_hybrid_fuse(const vdn_shape *shape, vdn_dtype dtype, cons
 VDN_API vdn_status vdn_out_proj(const vdn_shape *shape, vdn_dtype dtype, const void *a, const void *w_os,
                                 const void *w_ol, void *y, void *ws, size_t ws_bytes, vdn_stream stream);
 
+/* vdn_out_proj_e4m3 — the same projections with e4m3 operands on the tensor cores ([CARD]
+ * "Inference with Diffusers": every wide Linear in fp8 e4m3).
+ *   a8 [N_v][2*H*D] e4m3 codes; column c's value is a8 * a_scales[c / D], so a_scales
+ *   float[2][H] holds one dequantisation scale per (branch half, head): softmax half
+ *   first.  w_os, w_ol bf16 [HD][HD]; y bf16 [N_v][HD].
+ *   Each call folds a_scales into an e4m3 copy of [W_os | W_ol] quantised with one scale
+ *   per output column (its amax / 448, round to nearest, saturating), then runs one GEMM
+ *   with K = 2HD, fp32 accumulation, the column scale applied to y.  Needs H*D a multiple
+ *   of 256 (VDN_ERR_UNSUPPORTED otherwise).
+ * ws: vdn_out_proj_e4m3_workspace_size(shape) bytes (status word and the weight copy). */
+VDN_API size_t vdn_out_proj_e4m3_workspace_size(const vdn_shape *shape);
+VDN_API vdn_status vdn_out_proj_e4m3(const vdn_shape *shape, const void *a8, const float *a_scales,
+                                     const void *w_os, const void *w_ol, void *y, void *ws, size_t ws_bytes,
+                                     vdn_stream stream);
+
 /* ------------------------------------------------------------------ whole layer
  * vdn_hybrid_attn_fwd — the layer: both branches, fuse and projections, in one call.
  *   dtype VDN_F32:  every tensor float.
  *   dtype VDN_BF16: q,k,v,kt,vt,w_os,w_ol,y bf16.
  *   dtype VDN_E4M3: inputs as for VDN_BF16; the softmax branch quantises Q/K/V to e4m3
  *                   with per-head scales amax/448 ([CARD] "Inference with Diffusers").
+ *   dtype VDN_E4M3_PROJ: as VDN_E4M3, and the output projections run in e4m3 as in
+ *                   vdn_out_proj_e4m3: the branch epilogues write A as e4m3 codes with
+ *                   per-head scales from static bounds (softmax half: the V scale, since
+ *                   g_s O_s is a gated convex combination of V rows; linear half:
+ *                   max|gamma_h| sqrt(D) / 448, since g_l gamma O_l / rms(O_l) is bounded
+ *                   by it).  head_dim 128 and H*D a multiple of 256.
  *   kind selects the linear branch; beta float[F][H] for DELTA, else NULL.
  *   w_gate_s, w_gate_l (G_l columns), gamma as for vdn_hybrid_fuse; eps of RMSNorm.
  * ws: vdn_hybrid_attn_workspace_size(shape, kind, dtype) bytes. */
@@ -246,6 +269,27 @@ VDN_API vdn_status vdn_hybrid_attn_fwd(const vdn_shape *shape, vdn_lin_kind kind
                                const float *w_gate_s, const float *w_gate_l, int32_t G_l, const float *gamma,
                                float eps, const void *w_os, const void *w_ol, void *y, void *ws,
                                size_t ws_bytes, vdn_stream stream);
+
+/* vdn_hybrid_attn_fwd_partial — one rank's share of the layer split by heads across
+ * GPUs ([CARD] "Set up" and "Inference with SGLang" run the model on 8 GPUs; heads are
+ * independent through both branches and the fuse, so the split needs one exchange, a sum
+ * of the projections' partial outputs).
+ *   shape.heads is this rank's head count H_r; q, k, v, kt, vt, w_gate_s, w_gate_l,
+ *   gamma are those heads' slices (layouts as for vdn_hybrid_attn_fwd with H = H_r);
+ *   beta float[F][H_r] for DELTA.  w_os, w_ol are bf16 [out_features][H_r*D]: the
+ *   columns of the full projections that multiply these heads' A columns.
+ *   y_partial float [N_v][out_features] = A_r[:, :H_r D] w_os^T + A_r[:, H_r D:] w_ol^T.
+ *   Summed over the ranks (for example an all-reduce or reduce-scatter), the partials
+ *   give the layer's y in float.
+ *   dtype VDN_BF16 or VDN_E4M3, head_dim 128, out_features a multiple of 32
+ *   (VDN_ERR_UNSUPPORTED / VDN_ERR_INVALID_ARG otherwise).
+ * ws: vdn_hybrid_attn_workspace_size(shape, kind, dtype) bytes with shape.heads = H_r. */
+VDN_API vdn_status vdn_hybrid_attn_fwd_partial(const vdn_shape *shape, int32_t out_features, vdn_lin_kind kind,
+                                               vdn_dtype dtype, const void *q, const void *k, const void *v,
+                                               const void *kt, const void *vt, const float *beta,
+                                               const float *w_gate_s, const float *w_gate_l, int32_t G_l,
+                                               const float *gamma, float eps, const void *w_os, const void *w_ol,
+                                               float *y_partial, void *ws, size_t ws_bytes, vdn_stream stream);
 
 /* vdn_hybrid_attn_fwd_host — the layer with its per-call tensors in HOST memory.  No
  * counterpart in the pages: it is the streaming form of vdn_hybrid_attn_fwd.

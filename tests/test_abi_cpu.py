@@ -150,6 +150,24 @@ def test_noalloc_checks_match_the_workspace_entry_point():
     assert st == 3 and b"256 KiB" in L.vdn_last_error()
 
 
+def test_partial_layer_checks():
+    """vdn_hybrid_attn_fwd_partial (one rank's share of the head split) rejects what it
+    cannot run before touching the device: head_dim other than 128, an out_features that
+    is not a multiple of 32, and the e4m3 projection."""
+    L = vdn.lib()
+    p = [16] * 5
+
+    def call(shape, n_out, dtype):
+        s = vdn.Shape(*shape)
+        return L.vdn_hybrid_attn_fwd_partial(ctypes.byref(s), n_out, vdn.ELU1, dtype, *p, None, 16, 16, shape[5], 16,
+                                             1e-6, 16, 16, 16, 256, 1 << 40, None)
+    assert call((4, 64, 5, 0, 2, 64), 128, vdn.BF16) == 2
+    assert call((4, 64, 5, 0, 2, 128), 100, vdn.BF16) == 1
+    assert call((4, 64, 5, 0, 2, 128), 0, vdn.BF16) == 1
+    assert call((4, 64, 5, 0, 2, 128), 256, vdn.E4M3_PROJ) == 2
+    assert call((4, 64, 5, 0, 2, 128), 256, vdn.BF16) not in (1, 2)   # valid; fails only for want of a GPU
+
+
 def test_host_entry_point_checks_and_sizes():
     """The host-buffer layer: its workspace adds the staging area; missing host tensors and a
     short workspace are reported before any device work."""

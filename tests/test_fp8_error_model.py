@@ -8,8 +8,9 @@ query block with the key count and head size of the full-size workload (17,648 k
 D = 128), and checks that the GPU bound of 7e-2 sits above it with margin.  The kernel
 itself is held to 3e-2 against the oracle evaluated on its own e4m3 inputs.
 
-The second test fixes, ahead of its kernel, the model error of an e4m3 output projection
-with per-row and per-column scales."""
+The next tests fix the model error of the e4m3 output projection (per-column weight
+scales; static per-head A scales from the branches' bounds) and of the whole e4m3 layer,
+which set the bounds its GPU tests use (tests/test_e4m3_projection_gpu.py)."""
 import numpy as np
 import torch
 
@@ -87,3 +88,50 @@ def test_e4m3_projection_static_bounds_cost_nothing():
     err_static = ((a8_static @ w8.T - ref).norm() / ref.norm()).item()
     err_row = ((a8_row @ w8.T - ref).norm() / ref.norm()).item()
     assert err_static < 0.8 * PROJ_GPU_BOUND and abs(err_static - err_row) < 0.05 * err_row, (err_static, err_row)
+
+
+LAYER_E4M3_BOUND = 6e-2
+
+
+def test_e4m3_layer_model_error():
+    """The whole e4m3 layer's model error on y: the e4m3 softmax (per-head Q/K/V scales,
+    e4m3 P) feeds A_s, A is written as e4m3 codes with the static per-head scales (the V
+    scale for A_s, max|gamma| sqrt(D) / 448 for A_l) and [W_os | W_ol] is rounded per output
+    column.  Simulated here with torch's CPU e4m3 conversion on layer-shaped data (2 heads
+    of 128, 17,648 keys per query, gates and RMSNorm as in the layer); y's error against
+    the exact float64 layer must sit well inside the GPU bound LAYER_E4M3_BOUND."""
+    g = torch.Generator().manual_seed(3)
+    n, nk, d, H = 128, 17648, 128, 2
+    hd = H * d
+    q = torch.randn(H, n, d, generator=g, dtype=torch.float64)
+    k = torch.randn(H, nk, d, generator=g, dtype=torch.float64)
+    v = torch.randn(H, nk, d, generator=g, dtype=torch.float64)
+    w_s = torch.randn(H, d, generator=g, dtype=torch.float64) * 0.02
+    w_l = torch.randn(H, d, d, generator=g, dtype=torch.float64) * 0.02
+    o_l = torch.randn(H, n, d, generator=g, dtype=torch.float64)          # any linear-branch output
+    w = torch.randn(hd, 2 * hd, generator=g, dtype=torch.float64) * 0.02
+
+    def layer_y(o_s, a8):
+        gs = torch.sigmoid((q * w_s[:, None, :]).sum(-1, keepdim=True))
+        gl = torch.sigmoid(torch.einsum("hnd,hde->hne", q, w_l))
+        nrm = o_l / torch.sqrt((o_l ** 2).mean(-1, keepdim=True) + 1e-6)
+        a_s, a_l = gs * o_s, gl * nrm                                        # gamma = 1
+        if a8:
+            vs = v.abs().amax((1, 2)) / 448.0                                # the V scale per head
+            ls = torch.full((H,), d ** 0.5 / 448.0, dtype=torch.float64)     # max|gamma| sqrt(D) / 448
+            a_s = (a_s / vs[:, None, None]).float().to(torch.float8_e4m3fn).double() * vs[:, None, None]
+            a_l = (a_l / ls[:, None, None]).float().to(torch.float8_e4m3fn).double() * ls[:, None, None]
+        a = torch.cat([a_s.permute(1, 0, 2).reshape(n, hd), a_l.permute(1, 0, 2).reshape(n, hd)], 1)
+        ww = torch.cat([_e4m3(c, c.abs().max()).unsqueeze(0) for c in w]) if a8 else w
+        return a @ ww.T
+
+    exact_o = torch.softmax(q @ k.transpose(1, 2) / d ** 0.5, -1) @ v
+    q8 = torch.stack([_e4m3(x, x.abs().max()) for x in q])
+    k8 = torch.stack([_e4m3(x, x.abs().max()) for x in k])
+    v8 = torch.stack([_e4m3(x, x.abs().max()) for x in v])
+    s = q8 @ k8.transpose(1, 2) / d ** 0.5
+    p = torch.exp(s - s.amax(-1, keepdim=True))
+    o8 = (p.float().to(torch.float8_e4m3fn).double() @ v8) / p.sum(-1, keepdim=True)
+    ref = layer_y(exact_o, False)
+    err = ((layer_y(o8, True) - ref).norm() / ref.norm()).item()
+    assert 0.02 < err < 0.8 * LAYER_E4M3_BOUND, err
