@@ -96,7 +96,8 @@ def kernel_work(shape: synth.Shape, linear: str, fp8: bool) -> dict:
     return work
 
 
-def kernel_rooflines(prof: dict, steps: int, shape, linear: str, fp8: bool, peaks: dict, fp8_ratio: float) -> dict:
+def kernel_rooflines(prof: dict, steps: int, shape, linear: str, fp8: bool, peaks: dict, fp8_ratio: float,
+                     fp8_proj: bool = False) -> dict:
     """Per kernel: live ms per call, achieved TFLOP/s or GB/s, and its fractions of the
     measured burst and sustained tensor peaks (the e4m3 softmax: times the e4m3/bf16 ratio)
     or of the measured HBM bandwidth."""
@@ -109,7 +110,8 @@ def kernel_rooflines(prof: dict, steps: int, shape, linear: str, fp8: bool, peak
         kind, amount = work[name]
         if kind == "tensor":
             tf = amount / (ms / 1e3) / 1e12
-            scale = fp8_ratio if (fp8 and name == "softmax_tc") else 1.0
+            e4m3 = (fp8 and name == "softmax_tc") or (fp8_proj and name == "out_proj_tc")
+            scale = fp8_ratio if e4m3 else 1.0
             out[name] = {"ms": round(ms, 4), "tflops": round(tf, 1),
                          "frac_of_burst": round(tf / (peaks["bf16_tflops"] * scale), 3),
                          "frac_of_sustained": round(tf / (peaks["bf16_tflops_sustained"] * scale), 3)}
@@ -433,7 +435,7 @@ PARITY_BOUNDS = {
 }
 
 
-def extra_layer_timing(s, kind, cdt, d, beta, G_l, steps, warmup, dev, local_rank, peaks, fp8_ratio):
+def extra_layer_timing(s, kind, cdt, d, beta, G_l, steps, warmup, dev, local_rank, peaks, fp8_ratio):  # noqa: PLR0913
     """Times one more configuration of the layer in this process (inputs already on the
     device): ms per step, video tokens/s, per-kernel rooflines and the clocks seen."""
     import torch
@@ -466,7 +468,9 @@ def extra_layer_timing(s, kind, cdt, d, beta, G_l, steps, warmup, dev, local_ran
     ms = e0.elapsed_time(e1) / max(steps, 1)
     linear = "delta" if kind == vdn.DELTA else "elu1"
     out = {"ms_per_step": ms, "value": s.n_video / (ms / 1e3), "unit": UNIT, "steps": steps, "warmup": warmup,
-           "kernels": kernel_rooflines(prof, steps, s, linear, True, dict(FALLBACK_PEAKS) | peaks, fp8_ratio),
+           "kernels": kernel_rooflines(prof, steps, s, linear, True, dict(FALLBACK_PEAKS) | peaks, fp8_ratio,
+                                       fp8_proj=(cdt == vdn.E4M3_PROJ)),
+           "peak_note": "e4m3 contractions against the measured bf16 peaks times the measured e4m3/bf16 ratio",
            "per_kernel_ms_per_step": {k: round(v[0] / max(steps, 1), 4) for k, v in prof.items()},
            "clocks": clk}
     del ws, y

@@ -330,6 +330,12 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
   const int g = tr[0];
   const int row0 = tr[1] + (int)(half_tile & 1) * BM, row_end = tr[2];
   if (row0 >= row_end) return;  // the second half of a short tile (block-uniform)
+  // range-check build: the tile, its group (memories, normaliser) and its rows
+  if (!(in_range(st, (int64_t)(half_tile >> 1), max_tiles(d.F, d.T, d.C), K_READ_TC, 1) &&
+        in_range(st, g, max_groups(d.F, d.C), K_READ_TC, 2) && in_range(st, row0, d.Nv(), K_READ_TC, 3) &&
+        in_range(st, row_end - 1, d.Nv(), K_READ_TC, 4) &&
+        in_range(st, (int64_t)h * D + D - 1, out_stride, K_READ_TC, 5)))
+    return;  // (block-uniform: every thread evaluates the same indices)
 
   const int quad = warp & 3, hf = warp >> 2;  // lane quarter (tensor-memory rule), column half
   const int r = quad * 32 + lane;             // row within the tile

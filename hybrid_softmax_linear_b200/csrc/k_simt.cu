@@ -514,14 +514,7 @@ __global__ void __launch_bounds__(256) scan_delta_small_kernel(Dims d, const flo
 // S_fwd = S_txt/2 + prefix[ie_g], S_bwd = S_txt/2 + suffix[ib_g].  With SUM the block
 // stores S_fwd + S_bwd in bf16 and z_fwd + z_bwd in float, the operands of the
 // tensor-core read, instead of the four float memories.
-#ifndef VDN_SCAN_THREADS
-#define VDN_SCAN_THREADS 256
-#endif
-#ifndef VDN_SCAN_INFLIGHT
-#define VDN_SCAN_INFLIGHT 8
-#endif
-constexpr int SCAN_THREADS = VDN_SCAN_THREADS;
-constexpr int SCAN_INFLIGHT = VDN_SCAN_INFLIGHT;  // frames a lane loads per round trip
+constexpr int SCAN_THREADS = 256;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -541,7 +534,8 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_seg_kernel(Dims d, const fl
                                                                 float *__restrict__ zb,
                                                                 __nv_bfloat16 *__restrict__ ssum,
                                                                 float *__restrict__ zsum,
-                                                                const int32_t *__restrict__ splan, int gcap) {
+                                                                const int32_t *__restrict__ splan, int gcap,
+                                                                DevStatus *stat) {
   extern __shared__ float4 sm4[];
   const int nseg = splan[0], G = splan[1];
   float4 *seg = sm4, *pre = sm4 + nseg * 32, *suf = pre + (nseg + 1) * 32;
@@ -558,21 +552,18 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_seg_kernel(Dims d, const fl
   const int32_t *bnd = splan + 4;
   for (int j = warp; j < nseg; j += SCAN_THREADS / 32) {
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    if (valid) {
+    // range-check build: segment bounds inside the frames the memories may hold
+    if (valid && in_range(stat, bnd[j] - 1, d.F - 2, K_SCAN, 1) && in_range(stat, bnd[j + 1] - 2, d.F - 2, K_SCAN, 2)) {
       const int hi = bnd[j + 1];
-      // SCAN_INFLIGHT frames per round trip: a segment of up to that many frames costs one
-      // memory latency
-      for (int f = bnd[j]; f < hi; f += SCAN_INFLIGHT) {
-        float4 x[SCAN_INFLIGHT];
+      // eight frames per round trip: a segment of up to eight frames costs one memory latency
+      for (int f = bnd[j]; f < hi; f += 8) {
+        float4 x[8];
 #pragma unroll
-        for (int k = 0; k < SCAN_INFLIGHT; ++k)
+        for (int k = 0; k < 8; ++k)
           x[k] = f + k < hi ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(f + k) * fstride))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < SCAN_INFLIGHT; k += 2) {
-          a = f4add(a, x[k]);
-          b = f4add(b, x[k + 1]);
-        }
+        a = f4add(a, f4add(f4add(x[0], x[1]), f4add(x[2], x[3])));
+        b = f4add(b, f4add(f4add(x[4], x[5]), f4add(x[6], x[7])));
       }
     }
     seg[j * 32 + lane] = f4add(a, b);
@@ -592,6 +583,9 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_seg_kernel(Dims d, const fl
   const float4 t = *reinterpret_cast<const float4 *>((isz ? zt : St) + h * per + off);
   const int32_t *ie = splan + splan_ie(d.F), *ib = splan + splan_ib(d.F, gcap);
   for (int g = warp; g < G; g += SCAN_THREADS / 32) {
+    if (!(in_range(stat, g, gcap, K_SCAN, 3) && in_range(stat, ie[g], nseg + 1, K_SCAN, 4) &&
+          in_range(stat, ib[g], nseg + 1, K_SCAN, 5)))
+      continue;
     const float4 pf = pre[ie[g] * 32 + lane], sb = suf[ib[g] * 32 + lane];
     const int64_t o = ((int64_t)g * d.H + h) * per + off;
     if (SUM) {
@@ -622,7 +616,8 @@ cudaError_t launch_scan_seg(const Dims &d, const float *S, const float *z, const
   const int64_t DD = (int64_t)d.D * d.D;
   dim3 grid((unsigned)(DD / 128 + (d.D + 127) / 128), d.H);
   scan_seg_kernel<SUM><<<grid, SCAN_THREADS, smem, st>>>(d, S, z, St, zt, Sf, Sb, zf, zb, ssum, zsum,
-                                                          (const int32_t *)(ws + p.splan), max_groups(d.F, d.C));
+                                                          (const int32_t *)(ws + p.splan), max_groups(d.F, d.C),
+                                                          (DevStatus *)(ws + p.status));
   return cudaGetLastError();
 }
 

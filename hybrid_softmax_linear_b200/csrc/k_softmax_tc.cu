@@ -195,12 +195,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int32_t *t0 = tiles + (int64_t)(blockIdx.x / d.H) * TILE_REC;
     const int first = t0[4], count = t0[5];
     const int rel = (int)(blockIdx.x - (unsigned)first * d.H);
-    const int32_t *tr = tiles + (int64_t)(first + rel % count) * TILE_REC;
+    const int64_t ti = first + rel % count;
+    const int32_t *tr = tiles + ti * TILE_REC;
     bars->h = rel / count;
     bars->row0 = tr[1];
     bars->row_end = tr[2];
     kv_parts(gtab + tr[0] * 16, d.L, bars->parts);
     bars->nkv = kv_tiles(bars->parts);
+    // range-check build: the tile, its group, its rows, its head and every key part must lie
+    // inside their tensors; a block that fails does no work
+    bool in = in_range(st, ti, max_tiles(d.F, d.T, d.C), K_SOFTMAX_TC, 1) &&
+              in_range(st, tr[0], max_groups(d.F, d.C), K_SOFTMAX_TC, 2) &&
+              in_range(st, bars->row0, d.Nv(), K_SOFTMAX_TC, 3) &&
+              in_range(st, bars->row_end - 1, d.Nv(), K_SOFTMAX_TC, 4) &&
+              in_range(st, bars->h, d.H, K_SOFTMAX_TC, 5) &&
+              in_range(st, (int64_t)bars->h * D + D - 1, out_row_stride, K_SOFTMAX_TC, 6);
+    for (int i = 0; in && i < bars->parts.n; ++i)
+      in = in_range(st, bars->parts.lo[i], bars->parts.text[i] ? d.L : d.Nv(), K_SOFTMAX_TC, 7) &&
+           in_range(st, bars->parts.hi[i] - 1, bars->parts.text[i] ? d.L : d.Nv(), K_SOFTMAX_TC, 8);
+    if (!in) { bars->nkv = 0; bars->row_end = bars->row0; }
   }
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);

@@ -267,6 +267,26 @@ __device__ __forceinline__ void report(DevStatus *st, uint32_t code, uint32_t wh
   }
 }
 
+// ---------------------------------------------------------------- range-check build
+// Built with VDN_BOUNDS_CHECK=1 (libvdn_checked.so, a test build standing in for a memory
+// checker), the tensor-core kernels check every global index they derive from the layout
+// tables against its tensor's extent before use; the first violation goes to the status
+// word as VDN_ERR_DEVICE with detail 0x10000 | site, and the access is skipped.  The
+// normal build compiles the checks away.
+#ifndef VDN_BOUNDS_CHECK
+#define VDN_BOUNDS_CHECK 0
+#endif
+__device__ __forceinline__ bool in_range(DevStatus *st, int64_t i, int64_t n, uint32_t kid, uint32_t site) {
+#if VDN_BOUNDS_CHECK
+  if (i >= 0 && i < n) return true;
+  report(st, VDN_ERR_DEVICE, kid, 0x10000u | site);
+  return false;
+#else
+  (void)st; (void)i; (void)n; (void)kid; (void)site;
+  return true;
+#endif
+}
+
 // Bound on device polls of an mbarrier or flag before a kernel gives up (about a
 // second at the polling rates involved).  Settable per call for the wait test.
 constexpr uint32_t DEFAULT_MAX_POLLS = 1u << 26;
