@@ -58,7 +58,6 @@ struct Cfg {
   static constexpr int K_OFF = Q_OFF + NQ * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + KST * TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + VST * TILE_BYTES;
-  static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
   static constexpr uint32_t IDESC_S = FP8 ? idesc_e4m3(BM, BN, false, false) : idesc_bf16(BM, BN, false, false);
   static constexpr uint32_t IDESC_O = FP8 ? idesc_e4m3(BM, D, false, true) : idesc_bf16(BM, D, false, true);
   // e4m3: P goes to the tensor cores in two pieces of 64 keys, so the P.V MMA of the first
@@ -89,6 +88,13 @@ struct alignas(8) Bars {
   int h, row0, row_end, nkv;
   KvParts parts;
 };
+
+// dynamic shared memory of a block: the 1024-byte alignment pad, the Q, K and V tiles, and
+// the barriers
+template <int D, bool FP8>
+constexpr size_t smem_bytes() { return 1024 + Cfg<D, FP8>::BAR_OFF + sizeof(Bars); }
+static_assert(smem_bytes<128, false>() <= 227 * 1024 && smem_bytes<128, true>() <= 227 * 1024,
+              "shared memory of a block");
 
 __device__ __forceinline__ void kv_parts(const int32_t *g, int L, KvParts &p) {
   p.n = 0;
@@ -636,9 +642,9 @@ cudaError_t launch_t(const Dims &d, const void *q, const void *k, const void *v,
     return cudaErrorInvalidValue;
   const int ntiles = host_tile_count(d);
   cudaError_t e = cudaFuncSetAttribute(softmax_tc_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)C::SMEM);
+                                       (int)smem_bytes<D, FP8>());
   if (e != cudaSuccess) return e;
-  softmax_tc_kernel<D, FP8><<<ntiles * d.H, THREADS, C::SMEM, st>>>(
+  softmax_tc_kernel<D, FP8><<<ntiles * d.H, THREADS, smem_bytes<D, FP8>(), st>>>(
       mq, mk, mv, mkt, mvt, d, sl2, scales, o, o_row_stride, w_gate_s, lse, (const int32_t *)(ws + p.gtab),
       (const int32_t *)(ws + p.tiles), out8 ? 1 : 0, (DevStatus *)(ws + p.status));
   return cudaGetLastError();
