@@ -51,19 +51,42 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
 }
 
 // ============================================================================ state build
+// Persistent: every CTA walks the (frame or text, head) items blockIdx.x, blockIdx.x +
+// gridDim.x, ... (heads vary fastest, so the CTAs in flight read whole token rows of K and
+// V), two CTAs per SM.  The TMA ring of 64-token chunks runs on across items, so no CTA
+// waits for its first loads after the first item; the accumulator alternates between two
+// 128-column halves of tensor memory, so the MMAs of an item start while the previous
+// item's S is still being read out.
 namespace sb {
 constexpr int D = 128, TK = 64, NS = 3, THREADS = 320, PHI_WARPS = 8;
 constexpr int BOX_BYTES = TK * 128;        // 64 tokens x 64 bf16
 constexpr int TILE_BYTES = 2 * BOX_BYTES;  // 64 tokens x 128 features
 constexpr int STAGE_BYTES = 2 * TILE_BYTES;
 constexpr uint32_t IDESC = idesc_bf16(128, 128, true, true);
+constexpr uint32_t TMEM_COLS = 256;        // two accumulators of 128 columns
 struct alignas(8) Bars {
-  uint64_t full[NS], phi[NS], empty[NS], acc, drain;
+  uint64_t full[NS], phi[NS], empty[NS], acc_full[2], acc_empty[2], drain;
   uint32_t tmem;
   int abort;
   float zpart[PHI_WARPS][D];  // z of each phi warp, summed in a fixed order (repeatable bits)
 };
 constexpr size_t SMEM = 1024 + NS * STAGE_BYTES + sizeof(Bars);
+
+// item x: frame fr = x / H (fr == F: the text), head h = x % H; its rows and token count
+struct Item {
+  int h, fr, row_base, ntok, nch;
+  bool text;
+};
+__device__ __forceinline__ Item item_of(const Dims &d, int x) {
+  Item it;
+  it.h = x % d.H;
+  it.fr = x / d.H;
+  it.text = it.fr == d.F;
+  it.ntok = it.text ? d.L : d.T;
+  it.row_base = it.text ? 0 : it.fr * d.T;
+  it.nch = (it.ntok + TK - 1) / TK;
+  return it;
+}
 }  // namespace sb
 
 __global__ void __launch_bounds__(sb::THREADS, 2)
@@ -81,14 +104,7 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
   if (threadIdx.x == 0) skip = *(volatile uint32_t *)&st->code != 0u;
   __syncthreads();
   if (skip) return;
-
-  // heads vary fastest across the grid, so the CTAs in flight read whole token rows of K and V
-  const int h = (int)(blockIdx.x % (unsigned)d.H);
-  const int fr = (int)(blockIdx.x / (unsigned)d.H);
-  const bool text = fr == d.F;
-  const int ntok = text ? d.L : d.T;
-  const int row_base = text ? 0 : fr * d.T;
-  const int nch = (ntok + TK - 1) / TK;
+  const int n_items = (d.F + 1) * d.H;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -96,134 +112,182 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
       mbar_init(smem_u32(&bars->phi[s]), PHI_WARPS);
       mbar_init(smem_u32(&bars->empty[s]), 1);
     }
-    mbar_init(smem_u32(&bars->acc), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bars->acc_full[b]), 1);
+      mbar_init(smem_u32(&bars->acc_empty[b]), PHI_WARPS);
+    }
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) { tmem_alloc(smem_u32(&bars->tmem), 128); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(smem_u32(&bars->tmem), TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
-  const CUtensorMap *mk = text ? &tmKt : &tmK;
-  const CUtensorMap *mv = text ? &tmVt : &tmV;
 
+  // Every role walks the same items and chunks in the same order: the ring slot of global
+  // chunk gc is gc % NS with phase (gc / NS) & 1, and the accumulator of the n-th item that
+  // has chunks is n & 1 with phase (n >> 1) & 1.
   if (warp == 0) {
     if (lane == 0) {
       uint32_t armed = 0, armed_ph = 0;
-      for (int c = 0; c < nch; ++c) {
-        const int s = c % NS;
-        if (!mbar_wait(smem_u32(&bars->empty[s]), ((c / NS) & 1) ^ 1, abort_flag, st, K_STATE, 1)) break;
-        const uint32_t fb = smem_u32(&bars->full[s]);
-        mbar_arrive_expect_tx(fb, STAGE_BYTES);
-        uint8_t *stg = base + s * STAGE_BYTES;
-        for (int b = 0; b < 2; ++b) {
-          tma_load_2d(smem_u32(stg + b * BOX_BYTES), mk, fb, h * D + b * 64, row_base + c * TK);
-          tma_load_2d(smem_u32(stg + TILE_BYTES + b * BOX_BYTES), mv, fb, h * D + b * 64, row_base + c * TK);
+      int gc = 0;
+      bool go = true;
+      for (int x = blockIdx.x; go && x < n_items; x += gridDim.x) {
+        const Item it = item_of(d, x);
+        const CUtensorMap *mk = it.text ? &tmKt : &tmK;
+        const CUtensorMap *mv = it.text ? &tmVt : &tmV;
+        for (int c = 0; c < it.nch; ++c, ++gc) {
+          const int s = gc % NS;
+          if (!mbar_wait(smem_u32(&bars->empty[s]), ((gc / NS) & 1) ^ 1, abort_flag, st, K_STATE_TC, 1)) {
+            go = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&bars->full[s]);
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          uint8_t *stg = base + s * STAGE_BYTES;
+          for (int bx = 0; bx < 2; ++bx) {
+            tma_load_2d(smem_u32(stg + bx * BOX_BYTES), mk, fb, it.h * D + bx * 64, it.row_base + c * TK);
+            tma_load_2d(smem_u32(stg + TILE_BYTES + bx * BOX_BYTES), mv, fb, it.h * D + bx * 64,
+                        it.row_base + c * TK);
+          }
+          armed |= 1u << s;
+          armed_ph = (armed_ph & ~(1u << s)) | (((gc / NS) & 1u) << s);
         }
-        armed |= 1u << s;
-        armed_ph = (armed_ph & ~(1u << s)) | (((c / NS) & 1u) << s);
       }
       int no_abort = 0;
       for (int s = 0; s < NS; ++s)
-        if (armed & (1u << s)) mbar_wait(smem_u32(&bars->full[s]), (armed_ph >> s) & 1u, &no_abort, st, K_STATE, 2);
+        if (armed & (1u << s)) mbar_wait(smem_u32(&bars->full[s]), (armed_ph >> s) & 1u, &no_abort, st, K_STATE_TC, 2);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      for (int c = 0; c < nch; ++c) {
-        const int s = c % NS;
-        if (!mbar_wait(smem_u32(&bars->phi[s]), (c / NS) & 1, abort_flag, st, K_STATE, 3)) break;
+      int gc = 0, na = 0;
+      bool ok = true;
+      for (int x = blockIdx.x; ok && x < n_items; x += gridDim.x) {
+        const Item it = item_of(d, x);
+        if (it.nch == 0) continue;
+        const int b = na & 1;
+        // the accumulator's previous item has been read out
+        if (!mbar_wait(smem_u32(&bars->acc_empty[b]), ((na >> 1) & 1) ^ 1, abort_flag, st, K_STATE_TC, 3)) break;
         tc_fence_after();
-        const uint32_t kb = smem_u32(base + s * STAGE_BYTES), vb = kb + TILE_BYTES;
+        const uint32_t acc = tmem + (uint32_t)(b * 128);
+        for (int c = 0; c < it.nch; ++c, ++gc) {
+          const int s = gc % NS;
+          if (!mbar_wait(smem_u32(&bars->phi[s]), (gc / NS) & 1, abort_flag, st, K_STATE_TC, 4)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kb = smem_u32(base + s * STAGE_BYTES), vb = kb + TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < TK / 16; ++kk)
-          mma_ss(tmem, sdesc(kb + kk * 2048, BOX_BYTES, 1024), sdesc(vb + kk * 2048, BOX_BYTES, 1024), IDESC,
-                 (c | kk) != 0);
-        mma_commit(smem_u32(&bars->empty[s]));
+          for (int kk = 0; kk < TK / 16; ++kk)
+            mma_ss(acc, sdesc(kb + kk * 2048, BOX_BYTES, 1024), sdesc(vb + kk * 2048, BOX_BYTES, 1024), IDESC,
+                   (c | kk) != 0);
+          mma_commit(smem_u32(&bars->empty[s]));
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&bars->acc_full[b]));
+        ++na;
       }
-      mma_commit(smem_u32(&bars->acc));
       mma_commit(smem_u32(&bars->drain));
       int no_abort = 0;
-      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_STATE, 4);
+      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_STATE_TC, 5);
     }
   } else {
-    // ---------------- phi pass (in place, masked) and z; then the epilogue
+    // ---------------- phi pass (in place, masked) and z; then each item's epilogue
     const int tid = threadIdx.x - 64;
     const int cl = tid & 15, rg = tid >> 4;  // column chunk 8cl..8cl+7; rows rg + 16i
-    float zacc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
-    bool ok = true;
-    for (int c = 0; c < nch; ++c) {
-      const int s = c % NS;
-      const bool got = mbar_wait(smem_u32(&bars->full[s]), (c / NS) & 1, abort_flag, st, K_STATE, 5);
-      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      uint8_t *kt = base + s * STAGE_BYTES;
-#pragma unroll
-      for (int i = 0; i < TK / 16; ++i) {
-        const int r = rg + 16 * i;
-        uint4 *p = reinterpret_cast<uint4 *>(kt + swz_off(r, cl, TK));
-        float f[8];
-        unpack8(*p, f);
-        const bool valid = c * TK + r < ntok;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          // phi enters the MMA in bf16, so the fast exponential is accurate enough
-          const float ph = valid ? phi_fast(f[e]) : 0.f;
-          zacc[e] += ph;
-          f[e] = ph;
-        }
-        *p = pack8(f);
-      }
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->phi[s]));
-    }
-    // lanes l and l ^ 16 hold the same columns: pair them, then one row per warp
-#pragma unroll
-    for (int e = 0; e < 8; ++e) zacc[e] += __shfl_xor_sync(0xffffffffu, zacc[e], 16);
-    if (lane < 16) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) bars->zpart[warp - 2][cl * 8 + e] = zacc[e];
-    }
     const int quad = warp & 3, c_lo = ((warp - 2) >> 2) * (D / 2);  // lane quarter; column half
-    const int i = quad * 32 + lane;  // key feature = accumulator row = tensor-memory lane
-    float *So = text ? St + (int64_t)h * D * D : S + ((int64_t)fr * d.H + h) * D * D;
-    if (nch > 0) {
-      const bool done = ok && mbar_wait(smem_u32(&bars->acc), 0, abort_flag, st, K_STATE, 6);
-      if (__all_sync(0xffffffffu, done)) {
-        tc_fence_after();
-        uint32_t u0[32], u1[32];
-        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c_lo, u0);
-        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c_lo + 32, u1);
-        tmem_wait_ld();
-        float4 *dst = reinterpret_cast<float4 *>(So + i * D + c_lo);
+    const int i_row = quad * 32 + lane;  // key feature = accumulator row = tensor-memory lane
+    int gc = 0, na = 0;
+    bool ok = true;
+    for (int x = blockIdx.x; x < n_items; x += gridDim.x) {
+      const Item it = item_of(d, x);
+      float zacc[8];
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = make_float4(__uint_as_float(u0[4 * v]), __uint_as_float(u0[4 * v + 1]),
-                               __uint_as_float(u0[4 * v + 2]), __uint_as_float(u0[4 * v + 3]));
+      for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+      for (int c = 0; c < it.nch; ++c, ++gc) {
+        const int s = gc % NS;
+        if (ok) ok = mbar_wait(smem_u32(&bars->full[s]), (gc / NS) & 1, abort_flag, st, K_STATE_TC, 6);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        uint8_t *kt = base + s * STAGE_BYTES;
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[8 + v] = make_float4(__uint_as_float(u1[4 * v]), __uint_as_float(u1[4 * v + 1]),
-                                   __uint_as_float(u1[4 * v + 2]), __uint_as_float(u1[4 * v + 3]));
+        for (int i = 0; i < TK / 16; ++i) {
+          const int r = rg + 16 * i;
+          uint4 *p = reinterpret_cast<uint4 *>(kt + swz_off(r, cl, TK));
+          float f[8];
+          unpack8(*p, f);
+          const bool valid = c * TK + r < it.ntok;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            // phi enters the MMA in bf16, so the fast exponential is accurate enough
+            const float ph = valid ? phi_fast(f[e]) : 0.f;
+            zacc[e] += ph;
+            f[e] = ph;
+          }
+          *p = pack8(f);
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->phi[s]));
       }
-    } else {
-      for (int cc = 0; cc < D / 2; ++cc) So[i * D + c_lo + cc] = 0.f;
-    }
-    named_bar_sync(1, 32 * PHI_WARPS);  // every phi warp has written its share of z
-    float *zo = text ? zt : z;
-    if (zo != nullptr && tid < D) {
-      float zs = 0.f;
+      // lanes l and l ^ 16 hold the same columns: pair them, then one row per warp
 #pragma unroll
-      for (int pw = 0; pw < PHI_WARPS; ++pw) zs += bars->zpart[pw][tid];
-      zo[(text ? (int64_t)h * D : ((int64_t)fr * d.H + h) * D) + tid] = zs;
+      for (int e = 0; e < 8; ++e) zacc[e] += __shfl_xor_sync(0xffffffffu, zacc[e], 16);
+      named_bar_sync(1, 32 * PHI_WARPS);  // the previous item's z sums are read
+      if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) bars->zpart[warp - 2][cl * 8 + e] = zacc[e];
+      }
+      float *So = it.text ? St + (int64_t)it.h * D * D : S + ((int64_t)it.fr * d.H + it.h) * D * D;
+      if (it.nch > 0) {
+        const int b = na & 1;
+        const bool done = ok && mbar_wait(smem_u32(&bars->acc_full[b]), (na >> 1) & 1, abort_flag, st, K_STATE_TC, 7);
+        ok = __all_sync(0xffffffffu, done);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t acc = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * 128) + c_lo;
+          uint32_t u0[32], u1[32];
+          tmem_ld32(acc, u0);
+          tmem_ld32(acc + 32, u1);
+          tmem_wait_ld();
+          // this accumulator may take the next item's MMAs once every phi warp has read it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty[b]));
+          float4 *dst = reinterpret_cast<float4 *>(So + i_row * D + c_lo);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(u0[4 * v]), __uint_as_float(u0[4 * v + 1]),
+                                 __uint_as_float(u0[4 * v + 2]), __uint_as_float(u0[4 * v + 3]));
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[8 + v] = make_float4(__uint_as_float(u1[4 * v]), __uint_as_float(u1[4 * v + 1]),
+                                     __uint_as_float(u1[4 * v + 2]), __uint_as_float(u1[4 * v + 3]));
+        }
+        ++na;
+      } else {
+        for (int cc = 0; cc < D / 2; ++cc) So[i_row * D + c_lo + cc] = 0.f;
+      }
+      // every phi warp has written its share of z; their states are ANDed, so that all eight
+      // leave the item loop together and their named barriers always pair up
+      ok = named_bar_and(1, 32 * PHI_WARPS, ok);
+      float *zo = it.text ? zt : z;
+      if (zo != nullptr && tid < D) {
+        float zs = 0.f;
+#pragma unroll
+        for (int pw = 0; pw < PHI_WARPS; ++pw) zs += bars->zpart[pw][tid];
+        zo[(it.text ? (int64_t)it.h * D : ((int64_t)it.fr * d.H + it.h) * D) + tid] = zs;
+      }
+      if (!ok) break;
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 128);
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 // ============================================================================ read staging
@@ -295,6 +359,16 @@ __device__ __forceinline__ float fast_sigmoid(float x) { return __fdividef(1.f, 
 // approximation (relative error below 2^-10.9): within 2.5e-4 of sigmoid(x), about half a
 // bf16 step of a gate of 1/8 and a tenth of one at 1/2, at one exponential-unit operation
 // per element instead of two
+__device__ __forceinline__ float tanh_fast(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(x));
+  return t;
+}
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ float gate_sigmoid(float x) {
   float t;
   asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
@@ -413,33 +487,33 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
   }
   if (ok) {
     const bool scalar_gate = fused && !gate_mma;
+    // pairs of values through the packed fp32 instructions; the normaliser in two chains
+    float2 den2 = make_float2(0.f, 0.f);
+    const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
 #pragma unroll
     for (int i = 0; i < HC / 8; ++i) {
       const int cl = c0 / 8 + i;
-      float f[8];
-      unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
-      if (scalar_gate) {
+      const uint4 raw = *reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM));
+      const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) gate1 = fmaf(f[e], bars->wg1[cl * 8 + e], gate1);
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (delta) {
-          f[e] *= inv_norm;
-        } else {
-          f[e] = phi_fast(f[e]);
+      for (int e = 0; e < 4; ++e) {
+        float2 x = __bfloat1622float2(hp[e]);
+        if (scalar_gate) {
+          gate1 = fmaf(x.x, bars->wg1[cl * 8 + 2 * e], gate1);
+          gate1 = fmaf(x.y, bars->wg1[cl * 8 + 2 * e + 1], gate1);
         }
+        if (delta) {
+          x = __fmul2_rn(x, make_float2(inv_norm, inv_norm));
+        } else {
+          // elu + 1 as max(x, 0) + 2^(min(x, 0) log2 e): no branch
+          const float2 e2 = __fmul2_rn(make_float2(fminf(x.x, 0.f), fminf(x.y, 0.f)), l2e);
+          x = __fadd2_rn(make_float2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)), make_float2(ex2f(e2.x), ex2f(e2.y)));
+          den2 = __ffma2_rn(x, *reinterpret_cast<const float2 *>(&bars->z[cl * 8 + 2 * e]), den2);
+        }
+        fr[i * 4 + e] = pack_bf16(x.x, x.y);
       }
-      if (!delta) {
-        const float4 za = *reinterpret_cast<const float4 *>(&bars->z[cl * 8]);
-        const float4 zb = *reinterpret_cast<const float4 *>(&bars->z[cl * 8 + 4]);
-        den = fmaf(f[0], za.x, den); den = fmaf(f[1], za.y, den); den = fmaf(f[2], za.z, den);
-        den = fmaf(f[3], za.w, den); den = fmaf(f[4], zb.x, den); den = fmaf(f[5], zb.y, den);
-        den = fmaf(f[6], zb.z, den); den = fmaf(f[7], zb.w, den);
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) fr[i * 4 + e] = pack_bf16(f[2 * e], f[2 * e + 1]);
     }
+    den = den2.x + den2.y;
   }
   // ---- 3. features over Q once the gate MMA has read it; then num
   ok = __syncthreads_and(ok && mbar_wait(smem_u32(&bars->gate_done), 0, abort_flag, st, K_READ, 2)) != 0;
@@ -477,13 +551,13 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
       tmem_ld32(acc, u0);
       tmem_ld32(acc + 32, u1);
       tmem_wait_ld();
+      float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float a = __uint_as_float(u0[i]), b = __uint_as_float(u1[i]);
-        ss = fmaf(a, a, ss);
-        ss = fmaf(b, b, ss);
+        const float2 ab = make_float2(__uint_as_float(u0[i]), __uint_as_float(u1[i]));
+        ss2 = __ffma2_rn(ab, ab, ss2);
       }
-      ss *= scale * scale;
+      ss = (ss2.x + ss2.y) * (scale * scale);
     }
   }
   __syncthreads();  // part[2] held the |q|^2 halves of the delta rule: all read before reuse
@@ -508,13 +582,24 @@ __global__ void __launch_bounds__(rd::THREADS, 2)
       for (int v = 0; v < 32; v += 8) {
         float o8[8];
         if (fused) {
-          const float4 ga = *reinterpret_cast<const float4 *>(&bars->gamma[c0 + c + v]);
-          const float4 gb = *reinterpret_cast<const float4 *>(&bars->gamma[c0 + c + v + 4]);
-          const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+          // pairs: gl * gamma * (num * f) with the packed fp32 instructions
+          const float2 fo = make_float2(f_out, f_out);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float gl = gate_mma ? gate_sigmoid(__uint_as_float(ug[v + e])) : gs;
-            o8[e] = gl * gg[e] * (__uint_as_float(u[v + e]) * f_out);
+          for (int e = 0; e < 8; e += 2) {
+            const float2 gg = *reinterpret_cast<const float2 *>(&bars->gamma[c0 + c + v + e]);
+            float2 gl;
+            if (gate_mma) {
+              const float2 t = __fmul2_rn(make_float2(__uint_as_float(ug[v + e]), __uint_as_float(ug[v + e + 1])),
+                                          make_float2(0.5f, 0.5f));
+              gl = __ffma2_rn(make_float2(0.5f, 0.5f), make_float2(tanh_fast(t.x), tanh_fast(t.y)),
+                              make_float2(0.5f, 0.5f));
+            } else {
+              gl = make_float2(gs, gs);
+            }
+            const float2 o = __fmul2_rn(__fmul2_rn(gl, gg),
+                                        __fmul2_rn(make_float2(__uint_as_float(u[v + e]), __uint_as_float(u[v + e + 1])), fo));
+            o8[e] = o.x;
+            o8[e + 1] = o.y;
           }
         } else {
 #pragma unroll
@@ -594,8 +679,10 @@ cudaError_t launch_state_build_tc(const Dims &d, const void *k, const void *v, c
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(state_build_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
   if (e != cudaSuccess) return e;
-  state_build_tc_kernel<<<(unsigned)((d.F + 1) * d.H), THREADS, SMEM, st>>>(mk, mv, mkt, mvt, d, S, z, St, zt,
-                                                                   (DevStatus *)(ws + p.status));
+  const int n_items = (d.F + 1) * d.H;
+  const int grid = n_items < 2 * sm_count() ? n_items : 2 * sm_count();  // persistent: two CTAs per SM
+  state_build_tc_kernel<<<(unsigned)grid, THREADS, SMEM, st>>>(mk, mv, mkt, mvt, d, S, z, St, zt,
+                                                               (DevStatus *)(ws + p.status));
   return cudaGetLastError();
 }
 

@@ -568,19 +568,39 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_seg_kernel(Dims d, const fl
     }
     seg[j * 32 + lane] = f4add(a, b);
   }
+  // the text state's entries, loaded while the segments are summed
+  const float4 t = valid ? *reinterpret_cast<const float4 *>((isz ? zt : St) + h * per + off)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
+  // prefix (warp 0) and suffix (warp 1) sums over the segments, in segment order; eight
+  // segments' loads are issued ahead of their chain of adds
   if (warp == 0) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < nseg; ++j) { pre[j * 32 + lane] = acc; acc = f4add(acc, seg[j * 32 + lane]); }
+    int j = 0;
+    for (; j + 8 <= nseg; j += 8) {
+      float4 x[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = seg[(j + k) * 32 + lane];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) { pre[(j + k) * 32 + lane] = acc; acc = f4add(acc, x[k]); }
+    }
+    for (; j < nseg; ++j) { pre[j * 32 + lane] = acc; acc = f4add(acc, seg[j * 32 + lane]); }
     pre[nseg * 32 + lane] = acc;
   } else if (warp == 1) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     suf[nseg * 32 + lane] = acc;
-    for (int j = nseg - 1; j >= 0; --j) { acc = f4add(acc, seg[j * 32 + lane]); suf[j * 32 + lane] = acc; }
+    int j = nseg - 1;
+    for (; j - 8 >= -1; j -= 8) {
+      float4 x[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = seg[(j - k) * 32 + lane];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) { acc = f4add(acc, x[k]); suf[(j - k) * 32 + lane] = acc; }
+    }
+    for (; j >= 0; --j) { acc = f4add(acc, seg[j * 32 + lane]); suf[j * 32 + lane] = acc; }
   }
   __syncthreads();
   if (!valid) return;
-  const float4 t = *reinterpret_cast<const float4 *>((isz ? zt : St) + h * per + off);
   const int32_t *ie = splan + splan_ie(d.F), *ib = splan + splan_ib(d.F, gcap);
   for (int g = warp; g < G; g += SCAN_THREADS / 32) {
     if (!(in_range(stat, g, gcap, K_SCAN, 3) && in_range(stat, ie[g], nseg + 1, K_SCAN, 4) &&
