@@ -316,39 +316,54 @@ __global__ void __launch_bounds__(256) read_stage_kernel(int64_t n_s8, int64_t n
 }
 
 // ============================================================================ read (+ gate, RMSNorm)
-// One CTA per 128 query rows (half of a 256-row tile) and head; two CTAs fit on an SM.
-// Eight warps; each query row belongs to two threads (one per column half), and thread 0
-// also drives the copy engine and the tensor cores:
-//   1. thread 0 loads Q, S_sum and W_l with TMA; everyone waits for them;
-//   2. thread 0 issues the gate logits Q W_l (G_l = D) while every thread builds its half of
-//      the feature row phi(q) (or q/|q|), its part of the normaliser phi(q).z and, with
-//      G_l = 1, of the scalar gate logit;
-//   3. once the gate MMA has read Q the features go over it; thread 0 issues
-//      num = feature * S_sum;
-//   4. every thread forms its half of o = num / den and stores o, or
-//      A_l = g_l * gamma * o / rms(o) with the sum of squares shared between the halves.
-// The halves meet through shared memory at block barriers that every thread reaches
-// whatever happened before (a failed wait only turns the remaining work off).
+// Persistent, one CTA per SM; CTA c takes a contiguous range of the work list.  An item is
+// the 128-row half of a query tile for one head, listed head by head (a CTA keeps one
+// head's gate weights W_l for long runs) and, inside a head, tile by tile in row order (so
+// consecutive items of one group share the group memory S_sum).  Roles:
+//   warp 0      TMA: Q tiles into a 3-stage ring, then W_l and S_sum into one slot each
+//               when the item's head or group changes (each slot is a one-stage ring whose
+//               refill waits for the release of the previous fill)
+//   warp 1      one thread issues the MMAs: the gate logits Q W_l into tensor memory as
+//               soon as the Q tile has landed, then num = feature * S_sum once the feature
+//               rows are written; two accumulator sets of 256 columns
+//   warps 4-11  two threads per query row, one per column half: that half of the feature
+//               row phi(q) (or q/|q|), written over the Q tile once the gate MMA has read
+//               it, and its share of the normaliser phi(q).z and (G_l = 1) the scalar gate
+//               logit
+//   warps 12-19 epilogue, two threads per row: o = num / den from tensor memory, then o or
+//               A_l = g_l * gamma * o / rms(o) (the halves' sums of squares meet in shared
+//               memory), staged in shared memory and written by a TMA store that runs on
+//               while the next item is computed (a short last tile of a group, whose box
+//               would reach the next group's rows, with plain stores instead)
+// (warps 2 and 3 have no role.)  Eight warps per role keep two of them on each scheduler,
+// so that one covers the exponential-unit and memory latencies of the other.  The TMA loads of later tiles, the tensor cores, the feature
+// rows of one item and the epilogue of the previous one overlap.  Every wait names the fill
+// or use it expects with a phase parity that cannot be two phases behind: a slot is refilled
+// only after its previous contents are released, and no release is issued before a use.
 namespace rd {
-constexpr int D = 128, BM = 128, THREADS = 256, HC = D / 2;
+constexpr int D = 128, BM = 128, HC = D / 2, NQ = 3, THREADS = 640;
+constexpr int FEAT_WARP0 = 4, EPI_WARP0 = 12, ROLE_WARPS = 8;  // two threads per row: one per column half
 constexpr int TILE_BYTES = BM * D * 2;  // 32 KB: one 128-row bf16 tile (two 64-column boxes)
-constexpr int Q_OFF = 0, S_OFF = TILE_BYTES, W_OFF = 2 * TILE_BYTES;
-constexpr int BAR_OFF = 3 * TILE_BYTES;
+// staged output tile: the TMA store's boxes with the 128-byte swizzle (bf16: two boxes of 64
+// columns, 16 KB each; e4m3: one box of 128 columns)
+constexpr int Q_OFF = 0, S_OFF = NQ * TILE_BYTES, W_OFF = S_OFF + TILE_BYTES, O_OFF = W_OFF + TILE_BYTES;
+constexpr int BAR_OFF = O_OFF + TILE_BYTES;
 constexpr uint32_t IDESC_NUM = idesc_bf16(BM, D, false, true);   // A K-major, B MN-major
-constexpr uint32_t TMEM_COLS = 256;                               // num at 0, gate logits at 128
+constexpr uint32_t TMEM_COLS = 512;                               // set a: num at 256a, gate logits at 256a + 128
 struct alignas(16) Bars {
-  float z[D], gamma[D], wg1[D];
-  float part[3][2][BM];  // per column half: normaliser, scalar-gate logit, sum of squares
-  uint64_t q_full, w_full, s_full, gate_done, acc, drain;
+  // with S_sum (one fill per group and head): the normaliser z and the scalar-gate weights
+  float zs[D], wg1[D];
+  float gam[D];                 // gamma of the epilogue's current head (staged by the epilogue)
+  float den[2][2][BM], g1[2][2][BM];  // per accumulator set and column half: normaliser and scalar-gate logit
+  float ssq[2][BM];                   // the epilogue's sums of squares per column half
+  uint64_t q_full[NQ], q_empty[NQ], gate_done[NQ], feat_full[NQ], den_full[2], acc_full[2], acc_empty[2];
+  uint64_t s_full, s_empty, w_full, w_empty, drain;
   uint32_t tmem;
   int abort;
 };
 constexpr size_t SMEM = 1024 + BAR_OFF + sizeof(Bars);
-// Output rows are staged in shared memory (over Q and S, free once num is complete) with a
-// 16-byte pad per row, then written out two whole rows per warp instruction.
-constexpr int OUT_PITCH = D * 2 + 16;
-constexpr int OUT_PITCH8 = D + 16;  // e4m3 output rows
-static_assert(BM * OUT_PITCH <= 2 * TILE_BYTES, "output staging must fit over Q and S");
+static_assert(SMEM <= 227 * 1024, "shared memory of a block");
+static_assert(BAR_OFF % 16 == 0, "barrier alignment");
 }  // namespace rd
 
 // 1 / (1 + 2^(-x log2 e)) with the hardware exp2 and reciprocal approximations (relative
@@ -369,287 +384,409 @@ __device__ __forceinline__ float ex2f(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ float gate_sigmoid(float x) {
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
-  return fmaf(0.5f, t, 0.5f);
+
+struct ReadItem {
+  int g, h, row0, row_end;
+};
+
+// Item x of the work list: head x / (2 n_tiles), then the tiles in row order, two halves
+// each.  False for the empty second half of a short tile, and (range-check build) for an
+// item whose group or rows fall outside their tensors; every role decodes the same list,
+// so all of them skip the same items.
+__device__ __forceinline__ bool read_item(const int32_t *__restrict__ tiles, int n_tiles, const Dims &d,
+                                          DevStatus *st, int64_t x, ReadItem &it) {
+  const int64_t per_head = 2 * (int64_t)n_tiles;
+  it.h = (int)(x / per_head);
+  const int rem = (int)(x - (int64_t)it.h * per_head);
+  const int32_t *tr = tiles + (int64_t)(rem >> 1) * TILE_REC;
+  it.g = tr[0];
+  it.row0 = tr[1] + (rem & 1) * rd::BM;
+  it.row_end = tr[2];
+  return it.row0 < it.row_end && in_range(st, it.g, max_groups(d.F, d.C), K_READ_TC, 2) &&
+         in_range(st, it.row0, d.Nv(), K_READ_TC, 3) && in_range(st, it.row_end - 1, d.Nv(), K_READ_TC, 4);
 }
 
 // DELTA: q/|q| features and no normaliser; FUSED: RMSNorm and the linear gate (GATE_MMA:
 // element-wise, G_l = D, on the tensor cores; otherwise the scalar gate, G_l = 1)
 template <bool DELTA, bool FUSED, bool GATE_MMA>
-__global__ void __launch_bounds__(rd::THREADS, 2)
+__global__ void __launch_bounds__(rd::THREADS, 1)
     read_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
-                   const __grid_constant__ CUtensorMap tmW, Dims d, const float *__restrict__ zsum,
-                   const float *__restrict__ wgl, int G_l, const float *__restrict__ gamma, float eps,
-                   void *__restrict__ out, int64_t out_stride, const int32_t *__restrict__ tiles,
-                   const float *__restrict__ a8_scale,
-                   DevStatus *st) {
+                   const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmO, Dims d,
+                   const float *__restrict__ zsum, const float *__restrict__ wgl, int G_l,
+                   const float *__restrict__ gamma, float eps, void *__restrict__ out, int64_t out_stride,
+                   const int32_t *__restrict__ tiles, int n_tiles,
+                   int64_t n_items, const float *__restrict__ a8_scale, DevStatus *st) {
   using namespace rd;
-  constexpr bool delta = DELTA, fused = FUSED, gate_mma = FUSED && GATE_MMA;
+  constexpr bool delta = DELTA, fused = FUSED, gate_mma = FUSED && GATE_MMA, scalar_gate = FUSED && !GATE_MMA;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   Bars *bars = reinterpret_cast<Bars *>(base + BAR_OFF);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int *abort_flag = &bars->abort;
   __shared__ int skip;
-  if (tid == 0) skip = *(volatile uint32_t *)&st->code != 0u;
+  if (threadIdx.x == 0) skip = *(volatile uint32_t *)&st->code != 0u;
   __syncthreads();
   if (skip) return;
+  const int64_t per = (n_items + gridDim.x - 1) / gridDim.x;
+  const int64_t x0 = (int64_t)blockIdx.x * per;
+  const int64_t x1 = x0 + per < n_items ? x0 + per : n_items;
+  if (x0 >= x1) return;  // block-uniform
+  // range-check build: the last head's columns lie inside an output row (block-uniform)
+  if (!in_range(st, (int64_t)d.H * D - 1, out_stride, K_READ_TC, 5)) return;
 
-  // heads vary fastest across the grid: the CTAs in flight read and write whole rows
-  const int h = (int)(blockIdx.x % (unsigned)d.H);
-  const unsigned half_tile = blockIdx.x / (unsigned)d.H;
-  const int32_t *tr = tiles + (int64_t)(half_tile >> 1) * TILE_REC;
-  const int g = tr[0];
-  const int row0 = tr[1] + (int)(half_tile & 1) * BM, row_end = tr[2];
-  if (row0 >= row_end) return;  // the second half of a short tile (block-uniform)
-  // range-check build: the tile, its group (memories, normaliser) and its rows
-  if (!(in_range(st, (int64_t)(half_tile >> 1), max_tiles(d.F, d.T, d.C), K_READ_TC, 1) &&
-        in_range(st, g, max_groups(d.F, d.C), K_READ_TC, 2) && in_range(st, row0, d.Nv(), K_READ_TC, 3) &&
-        in_range(st, row_end - 1, d.Nv(), K_READ_TC, 4) &&
-        in_range(st, (int64_t)h * D + D - 1, out_stride, K_READ_TC, 5)))
-    return;  // (block-uniform: every thread evaluates the same indices)
-
-  const int quad = warp & 3, hf = warp >> 2;  // lane quarter (tensor-memory rule), column half
-  const int r = quad * 32 + lane;             // row within the tile
-  const int c0 = hf * HC;                     // first column of this thread's half
-  const uint32_t qf = smem_u32(&bars->q_full), wf = smem_u32(&bars->w_full), sf = smem_u32(&bars->s_full);
-  if (tid == 0) {
-    mbar_init(qf, 1);
-    mbar_init(wf, 1);
-    mbar_init(sf, 1);
-    mbar_init(smem_u32(&bars->gate_done), 1);
-    mbar_init(smem_u32(&bars->acc), 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(smem_u32(&bars->q_full[s]), 1);
+      mbar_init(smem_u32(&bars->q_empty[s]), 1);
+      mbar_init(smem_u32(&bars->gate_done[s]), 1);
+      mbar_init(smem_u32(&bars->feat_full[s]), ROLE_WARPS);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&bars->den_full[a]), ROLE_WARPS);
+      mbar_init(smem_u32(&bars->acc_full[a]), 1);
+      mbar_init(smem_u32(&bars->acc_empty[a]), ROLE_WARPS);
+    }
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->s_empty), 1);
+    mbar_init(smem_u32(&bars->w_full), 1);
+    mbar_init(smem_u32(&bars->w_empty), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
     fence_mbar_init();
-    // ---- 1. operands, each on its own barrier: the features need only Q, the gate MMA
-    // Q and W, the num MMA S; issued before the per-head vectors are fetched
-    mbar_arrive_expect_tx(qf, TILE_BYTES);
-    if (gate_mma) mbar_arrive_expect_tx(wf, TILE_BYTES);
-    mbar_arrive_expect_tx(sf, TILE_BYTES);
-    for (int b = 0; b < 2; ++b) {
-      tma_load_2d(smem_u32(base + Q_OFF + b * BM * 128), &tmQ, qf, h * D + b * 64, row0);
-      if (gate_mma) tma_load_2d(smem_u32(base + W_OFF + b * BM * 128), &tmW, wf, b * 64, h * D);
-      tma_load_2d(smem_u32(base + S_OFF + b * BM * 128), &tmS, sf, b * 64, (g * d.H + h) * D);
-    }
-  }
-  if (tid < D) {
-    bars->z[tid] = delta ? 0.f : zsum[((int64_t)g * d.H + h) * D + tid];
-    bars->gamma[tid] = fused ? gamma[(int64_t)h * D + tid] : 0.f;
-    bars->wg1[tid] = (fused && !gate_mma) ? wgl[((int64_t)h * D + tid) * G_l] : 0.f;
+    tma_prefetch(&tmQ);
+    tma_prefetch(&tmS);
+    if (gate_mma) tma_prefetch(&tmW);
+    tma_prefetch(&tmO);
   }
   if (warp == 0) { tmem_alloc(smem_u32(&bars->tmem), TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
-  const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-  const uint32_t qa = smem_u32(base + Q_OFF), sb_ = smem_u32(base + S_OFF), wb = smem_u32(base + W_OFF);
-  bool issued = false;  // thread 0: MMAs in flight that must drain before the block exits
-  bool ok = __syncthreads_and(mbar_wait(qf, 0, abort_flag, st, K_READ, 1)) != 0;
 
-  // ---- 2. gate logits on the tensor cores; the feature half-row in registers
-  if (ok && tid == 0 && (!gate_mma || mbar_wait(wf, 0, abort_flag, st, K_READ, 6))) {
-    tc_fence_after();
-    if (gate_mma) {
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + 128, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
-               sdesc(wb + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
-    }
-    mma_commit(smem_u32(&bars->gate_done));  // Q may be overwritten once this arrives
-    issued = true;
-  }
-  __syncwarp();
-  uint8_t *qt = base + Q_OFF;
-  uint32_t fr[HC / 2];
-  float den = 0.f, gate1 = 0.f, ssq = 0.f;
-  if (ok) {
-    if (delta) {
-      // |q|^2 over the whole row: this half's share now, the other's through part[2]
-#pragma unroll
-      for (int cl = c0 / 8; cl < (c0 + HC) / 8; ++cl) {
-        float f[8];
-        unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM)), f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ssq = fmaf(f[e], f[e], ssq);
-      }
-    }
-    bars->part[2][hf][r] = ssq;
-  }
-  if (delta) __syncthreads();  // block-uniform: the |q|^2 halves meet (delta rule only)
-  float inv_norm = 1.f;
-  if (ok && delta) {
-    const float qq = bars->part[2][0][r] + bars->part[2][1][r];
-    inv_norm = qq > 0.f ? rsqrtf(qq) : 0.f;
-  }
-  if (ok) {
-    const bool scalar_gate = fused && !gate_mma;
-    // pairs of values through the packed fp32 instructions; the normaliser in two chains
-    float2 den2 = make_float2(0.f, 0.f);
-    const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
-#pragma unroll
-    for (int i = 0; i < HC / 8; ++i) {
-      const int cl = c0 / 8 + i;
-      const uint4 raw = *reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM));
-      const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float2 x = __bfloat1622float2(hp[e]);
-        if (scalar_gate) {
-          gate1 = fmaf(x.x, bars->wg1[cl * 8 + 2 * e], gate1);
-          gate1 = fmaf(x.y, bars->wg1[cl * 8 + 2 * e + 1], gate1);
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      // Per item: its Q tile first, then a refill of W_l / S_sum if the head / group
+      // changed.  The MMA thread releases a slot at the first item of the next head or
+      // group, before it waits for anything of that item, so these waits never wait on a
+      // load that comes after them.
+      int k = 0, ns = 0, nw = 0, cur_s = -1, cur_w = -1;
+      for (int64_t x = x0; x < x1; ++x) {
+        ReadItem it;
+        if (!read_item(tiles, n_tiles, d, st, x, it)) continue;
+        const int s = k % NQ;
+        if (!mbar_wait(smem_u32(&bars->q_empty[s]), ((k / NQ) & 1) ^ 1, abort_flag, st, K_READ, 1)) break;
+        const uint32_t qb = smem_u32(&bars->q_full[s]);
+        mbar_arrive_expect_tx(qb, TILE_BYTES);
+        for (int b = 0; b < 2; ++b)
+          tma_load_2d(smem_u32(base + Q_OFF + s * TILE_BYTES + b * BM * 128), &tmQ, qb, it.h * D + b * 64, it.row0);
+        ++k;
+        if (gate_mma && it.h != cur_w) {
+          if (!mbar_wait(smem_u32(&bars->w_empty), (nw & 1) ^ 1, abort_flag, st, K_READ, 2)) break;
+          const uint32_t wb = smem_u32(&bars->w_full);
+          mbar_arrive_expect_tx(wb, TILE_BYTES);
+          for (int b = 0; b < 2; ++b) tma_load_2d(smem_u32(base + W_OFF + b * BM * 128), &tmW, wb, b * 64, it.h * D);
+          ++nw;
+          cur_w = it.h;
         }
-        if (delta) {
-          x = __fmul2_rn(x, make_float2(inv_norm, inv_norm));
-        } else {
-          // elu + 1 as max(x, 0) + 2^(min(x, 0) log2 e): no branch
-          const float2 e2 = __fmul2_rn(make_float2(fminf(x.x, 0.f), fminf(x.y, 0.f)), l2e);
-          x = __fadd2_rn(make_float2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)), make_float2(ex2f(e2.x), ex2f(e2.y)));
-          den2 = __ffma2_rn(x, *reinterpret_cast<const float2 *>(&bars->z[cl * 8 + 2 * e]), den2);
-        }
-        fr[i * 4 + e] = pack_bf16(x.x, x.y);
-      }
-    }
-    den = den2.x + den2.y;
-  }
-  // ---- 3. features over Q once the gate MMA has read it; then num
-  ok = __syncthreads_and(ok && mbar_wait(smem_u32(&bars->gate_done), 0, abort_flag, st, K_READ, 2)) != 0;
-  if (ok) {
-#pragma unroll
-    for (int i = 0; i < HC / 8; ++i)
-      *reinterpret_cast<uint4 *>(qt + swz_off(r, c0 / 8 + i, BM)) =
-          make_uint4(fr[i * 4], fr[i * 4 + 1], fr[i * 4 + 2], fr[i * 4 + 3]);
-    fence_proxy_async();
-  }
-  bars->part[0][hf][r] = den;
-  bars->part[1][hf][r] = gate1;
-  __syncthreads();
-  if (ok && tid == 0 && mbar_wait(sf, 0, abort_flag, st, K_READ, 7)) {
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk)
-      mma_ss(tmem, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
-             sdesc(sb_ + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
-    mma_commit(smem_u32(&bars->acc));
-  }
-  __syncwarp();
-  ok = __syncthreads_and(ok && mbar_wait(smem_u32(&bars->acc), 0, abort_flag, st, K_READ, 3)) != 0;
-
-  // ---- 4. epilogue on this thread's half of the row
-  const float den_row = bars->part[0][0][r] + bars->part[0][1][r];
-  const float g1_row = bars->part[1][0][r] + bars->part[1][1][r];
-  const float scale = delta ? 1.f : (den_row > 0.f ? 1.f / den_row : 0.f);
-  const uint32_t acc = tmem + lane_off + (uint32_t)c0;
-  float ss = 0.f;
-  if (ok) {
-    tc_fence_after();
-    if (fused) {
-      uint32_t u0[32], u1[32];
-      tmem_ld32(acc, u0);
-      tmem_ld32(acc + 32, u1);
-      tmem_wait_ld();
-      float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float2 ab = make_float2(__uint_as_float(u0[i]), __uint_as_float(u1[i]));
-        ss2 = __ffma2_rn(ab, ab, ss2);
-      }
-      ss = (ss2.x + ss2.y) * (scale * scale);
-    }
-  }
-  __syncthreads();  // part[2] held the |q|^2 halves of the delta rule: all read before reuse
-  bars->part[2][hf][r] = ss;
-  __syncthreads();
-  uint8_t *stage = base + Q_OFF;  // Q, F and S are no longer read once num is complete
-  if (ok) {
-    const float rinv = fused ? rsqrtf((bars->part[2][0][r] + bars->part[2][1][r]) / (float)D + eps) : 1.f;
-    const float f_row = scale * rinv;  // o / rms(o) = num * scale * rinv
-    const float gs = fast_sigmoid(g1_row);
-    // e4m3 output (fused only): codes of A_l in units of its per-head scale a8_scale[h]
-    const bool out8 = fused && a8_scale != nullptr;
-    const float f_out = out8 ? f_row / a8_scale[h] : f_row;
-    uint8_t *srow = stage + (out8 ? r * OUT_PITCH8 + c0 : r * OUT_PITCH + c0 * 2);
-#pragma unroll
-    for (int c = 0; c < HC; c += 32) {
-      uint32_t u[32], ug[32];
-      tmem_ld32(acc + c, u);
-      if (fused && gate_mma) tmem_ld32(acc + 128 + c, ug);
-      tmem_wait_ld();
-#pragma unroll
-      for (int v = 0; v < 32; v += 8) {
-        float o8[8];
-        if (fused) {
-          // pairs: gl * gamma * (num * f) with the packed fp32 instructions
-          const float2 fo = make_float2(f_out, f_out);
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const float2 gg = *reinterpret_cast<const float2 *>(&bars->gamma[c0 + c + v + e]);
-            float2 gl;
-            if (gate_mma) {
-              const float2 t = __fmul2_rn(make_float2(__uint_as_float(ug[v + e]), __uint_as_float(ug[v + e + 1])),
-                                          make_float2(0.5f, 0.5f));
-              gl = __ffma2_rn(make_float2(0.5f, 0.5f), make_float2(tanh_fast(t.x), tanh_fast(t.y)),
-                              make_float2(0.5f, 0.5f));
-            } else {
-              gl = make_float2(gs, gs);
-            }
-            const float2 o = __fmul2_rn(__fmul2_rn(gl, gg),
-                                        __fmul2_rn(make_float2(__uint_as_float(u[v + e]), __uint_as_float(u[v + e + 1])), fo));
-            o8[e] = o.x;
-            o8[e + 1] = o.y;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o8[e] = __uint_as_float(u[v + e]) * f_out;
-        }
-        if (out8) {
-          uint32_t w2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(o8[4 * e], o8[4 * e + 1]), __NV_SATFINITE, __NV_E4M3);
-            const uint32_t hi =
-                __nv_cvt_float2_to_fp8x2(make_float2(o8[4 * e + 2], o8[4 * e + 3]), __NV_SATFINITE, __NV_E4M3);
-            w2[e] = (lo & 0xffffu) | (hi << 16);
-          }
-          *reinterpret_cast<uint2 *>(srow + c + v) = make_uint2(w2[0], w2[1]);
-        } else {
-          *reinterpret_cast<uint4 *>(srow + (c + v) * 2) = pack8(o8);
+        const int key = it.g * d.H + it.h;
+        if (key != cur_s) {
+          if (!mbar_wait(smem_u32(&bars->s_empty), (ns & 1) ^ 1, abort_flag, st, K_READ, 3)) break;
+          const uint32_t sb = smem_u32(&bars->s_full);
+          mbar_arrive_expect_tx(sb, TILE_BYTES + (delta ? 0u : D * 4u) + (scalar_gate ? D * 4u : 0u));
+          for (int b = 0; b < 2; ++b) tma_load_2d(smem_u32(base + S_OFF + b * BM * 128), &tmS, sb, b * 64, key * D);
+          if (!delta) bulk_load(smem_u32(bars->zs), zsum + (int64_t)key * D, D * 4u, sb);
+          if (scalar_gate) bulk_load(smem_u32(bars->wg1), wgl + (int64_t)it.h * D, D * 4u, sb);
+          ++ns;
+          cur_s = key;
         }
       }
-    }
-  }
-  __syncthreads();
-  if (ok) {
-    const int nrows = min(BM, row_end - row0);
-    if (fused && a8_scale != nullptr) {
-      // four rows per warp instruction: eight lanes per 128-byte row
-      for (int rr = warp * 4 + (lane >> 3); rr < nrows; rr += 4 * (THREADS / 32)) {
-        const uint4 val = *reinterpret_cast<const uint4 *>(stage + rr * OUT_PITCH8 + (lane & 7) * 16);
-        *reinterpret_cast<uint4 *>((uint8_t *)out + (int64_t)(row0 + rr) * out_stride + (int64_t)h * D +
-                                   (lane & 7) * 16) = val;
+      // every copy issued here lands before the block may exit (bounded waits)
+      int no_abort = 0;
+      for (int s = 0; s < NQ && s < k; ++s) {
+        const int fills = (k - s + NQ - 1) / NQ;
+        mbar_wait(smem_u32(&bars->q_full[s]), (fills - 1) & 1, &no_abort, st, K_READ, 4);
       }
-    } else {
-      // two rows per warp instruction: lanes 0-15 one row, 16-31 the next (256 bytes each)
-      for (int rr = warp * 2 + (lane >> 4); rr < nrows; rr += 2 * (THREADS / 32)) {
-        const uint4 val = *reinterpret_cast<const uint4 *>(stage + rr * OUT_PITCH + (lane & 15) * 16);
-        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)out + (int64_t)(row0 + rr) * out_stride + (int64_t)h * D +
-                                   (lane & 15) * 8) = val;
-      }
+      if (ns > 0) mbar_wait(smem_u32(&bars->s_full), (ns - 1) & 1, &no_abort, st, K_READ, 4);
+      if (nw > 0) mbar_wait(smem_u32(&bars->w_full), (nw - 1) & 1, &no_abort, st, K_READ, 4);
     }
-  }
-  // ---- drain: no copy or MMA of this block may be in flight when it exits
-  if (tid == 0) {
-    int no_abort = 0;
-    mbar_wait(qf, 0, &no_abort, st, K_READ, 4);
-    if (gate_mma) mbar_wait(wf, 0, &no_abort, st, K_READ, 4);
-    mbar_wait(sf, 0, &no_abort, st, K_READ, 4);
-    if (issued) {
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      int k = 0, ns = 0, nw = 0, cur_s = -1, cur_w = -1;
+      const uint32_t sb_ = smem_u32(base + S_OFF), wb = smem_u32(base + W_OFF);
+      for (int64_t x = x0; x < x1; ++x) {
+        ReadItem it;
+        if (!read_item(tiles, n_tiles, d, st, x, it)) continue;
+        const int s = k % NQ, a = k & 1;
+        const int key = it.g * d.H + it.h;
+        const bool new_w = gate_mma && it.h != cur_w, new_s = key != cur_s;
+        // releases first: every MMA on the previous W_l / S_sum has been issued
+        if (new_w && nw > 0) mma_commit(smem_u32(&bars->w_empty));
+        if (new_s && ns > 0) mma_commit(smem_u32(&bars->s_empty));
+        if (new_w) {
+          if (!mbar_wait(smem_u32(&bars->w_full), nw & 1, abort_flag, st, K_READ, 5)) break;
+          ++nw;
+          cur_w = it.h;
+        }
+        if (!mbar_wait(smem_u32(&bars->q_full[s]), (k / NQ) & 1, abort_flag, st, K_READ, 6)) break;
+        if (!mbar_wait(smem_u32(&bars->acc_empty[a]), ((k >> 1) & 1) ^ 1, abort_flag, st, K_READ, 7)) break;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(base + Q_OFF + s * TILE_BYTES);
+        const uint32_t acc = tmem + (uint32_t)a * 256;
+        if (gate_mma) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(acc + 128, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc(wb + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
+        }
+        // Q may be overwritten by the features, and den/g1 of set a reused, once this arrives
+        mma_commit(smem_u32(&bars->gate_done[s]));
+        if (new_s) {
+          if (!mbar_wait(smem_u32(&bars->s_full), ns & 1, abort_flag, st, K_READ, 8)) break;
+          ++ns;
+          cur_s = key;
+        }
+        if (!mbar_wait(smem_u32(&bars->feat_full[s]), (k / NQ) & 1, abort_flag, st, K_READ, 9)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(acc, sdesc(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
+                 sdesc(sb_ + kk * 2048, BM * 128, 1024), IDESC_NUM, kk > 0);
+        mma_commit(smem_u32(&bars->acc_full[a]));
+        mma_commit(smem_u32(&bars->q_empty[s]));
+        ++k;
+      }
+      // no MMA of this block may be in flight when it exits
       mma_commit(smem_u32(&bars->drain));
-      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_READ, 5);
+      int no_abort = 0;
+      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, st, K_READ, 10);
     }
+  } else if (warp >= FEAT_WARP0 && warp < FEAT_WARP0 + ROLE_WARPS) {
+    // ---------------------------------------------------------------- feature rows
+    const int r = (warp & 3) * 32 + lane, hf = (warp - FEAT_WARP0) >> 2, c0 = hf * HC;
+    int k = 0, ns = 0, cur_s = -1;
+    for (int64_t x = x0; x < x1; ++x) {
+      ReadItem it;
+      if (!read_item(tiles, n_tiles, d, st, x, it)) continue;
+      const int s = k % NQ, a = k & 1;
+      // z (and the scalar-gate weights) of a new group come with its S_sum; the slot is
+      // refilled only after the last item of the previous group has been handed over
+      const int key = it.g * d.H + it.h;
+      if (key != cur_s && (!delta || scalar_gate)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full), ns & 1, abort_flag, st, K_READ, 15))) break;
+        ++ns;
+        cur_s = key;
+      }
+      // the warp proceeds (or gives up) as a whole
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->q_full[s]), (k / NQ) & 1, abort_flag, st, K_READ, 11)))
+        break;
+      uint8_t *qt = base + Q_OFF + s * TILE_BYTES;
+      float inv_norm = 1.f;
+      if (delta) {
+        // |q|^2 over the whole row, by each of its two threads
+        float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int cl = 0; cl < D / 8; ++cl) {
+          const uint4 raw = *reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM));
+          const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 x2 = __bfloat1622float2(hp[e]);
+            ss2 = __ffma2_rn(x2, x2, ss2);
+          }
+        }
+        const float qq = ss2.x + ss2.y;
+        inv_norm = qq > 0.f ? rsqrtf(qq) : 0.f;
+      }
+      uint32_t fr[HC / 2];
+      float2 den2 = make_float2(0.f, 0.f);
+      float gate1 = 0.f;
+      const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
+#pragma unroll
+      for (int i = 0; i < HC / 8; ++i) {
+        const int cl = c0 / 8 + i;
+        const uint4 raw = *reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM));
+        const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2 xv = __bfloat1622float2(hp[e]);
+          if (scalar_gate) {
+            const float2 wv = *reinterpret_cast<const float2 *>(&bars->wg1[cl * 8 + 2 * e]);
+            gate1 = fmaf(xv.x, wv.x, fmaf(xv.y, wv.y, gate1));
+          }
+          if (delta) {
+            xv = __fmul2_rn(xv, make_float2(inv_norm, inv_norm));
+          } else {
+            // elu + 1 as max(x, 0) + 2^(min(x, 0) log2 e): no branch
+            const float2 e2 = __fmul2_rn(make_float2(fminf(xv.x, 0.f), fminf(xv.y, 0.f)), l2e);
+            xv = __fadd2_rn(make_float2(fmaxf(xv.x, 0.f), fmaxf(xv.y, 0.f)), make_float2(ex2f(e2.x), ex2f(e2.y)));
+            den2 = __ffma2_rn(xv, *reinterpret_cast<const float2 *>(&bars->zs[cl * 8 + 2 * e]), den2);
+          }
+          fr[i * 4 + e] = pack_bf16(xv.x, xv.y);
+        }
+      }
+      // Q is the A operand of the gate MMA: the features go over it only afterwards.
+      // gate_done also means the epilogue has released accumulator set a, and with it den[a]
+      // and g1[a].
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(smem_u32(&bars->gate_done[s]), (k / NQ) & 1, abort_flag, st, K_READ, 12)))
+        break;
+#pragma unroll
+      for (int i = 0; i < HC / 8; ++i)
+        *reinterpret_cast<uint4 *>(qt + swz_off(r, c0 / 8 + i, BM)) =
+            make_uint4(fr[i * 4], fr[i * 4 + 1], fr[i * 4 + 2], fr[i * 4 + 3]);
+      bars->den[a][hf][r] = den2.x + den2.y;
+      bars->g1[a][hf][r] = gate1;
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&bars->feat_full[s]));
+        mbar_arrive(smem_u32(&bars->den_full[a]));
+      }
+      ++k;
+    }
+  } else if (warp >= EPI_WARP0) {
+    // ---------------------------------------------------------------- epilogue
+    const int quad = warp & 3, r = quad * 32 + lane, hf = (warp - EPI_WARP0) >> 2, c0 = hf * HC;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    uint8_t *stage = base + O_OFF;
+    const bool out8 = fused && a8_scale != nullptr;  // e4m3 codes of A_l in units of a8_scale[h]
+    const int et = threadIdx.x - EPI_WARP0 * 32;     // 0 .. 255
+    constexpr int NT = ROLE_WARPS * 32;
+    int k = 0, cur_h = -1;
+    for (int64_t x = x0; x < x1; ++x) {
+      ReadItem it;
+      if (!read_item(tiles, n_tiles, d, st, x, it)) continue;
+      const int a = k & 1;
+      // gamma of a new head: every epilogue thread has passed the previous item's last
+      // barrier, so nobody reads the old values any more; the next barrier publishes these
+      if (fused && it.h != cur_h) {
+        if (et < D) bars->gam[et] = gamma[(int64_t)it.h * D + et];
+        cur_h = it.h;
+      }
+      // the previous item's TMA store has read the staged tile once this returns; the
+      // barrier below tells the others
+      if (et == 0) bulk_wait_read_all();
+      const bool got = mbar_wait(smem_u32(&bars->acc_full[a]), (k >> 1) & 1, abort_flag, st, K_READ, 13) &&
+                       mbar_wait(smem_u32(&bars->den_full[a]), (k >> 1) & 1, abort_flag, st, K_READ, 14);
+      // the epilogue warps go on (or give up) together: they share the staging buffer, which
+      // the previous item's stores have finished reading once all of them are here
+      if (!named_bar_and(1, NT, got)) break;
+      tc_fence_after();
+      const float den = bars->den[a][0][r] + bars->den[a][1][r];
+      const float gate1 = bars->g1[a][0][r] + bars->g1[a][1][r];
+      const float scale = delta ? 1.f : (den > 0.f ? 1.f / den : 0.f);
+      const uint32_t acc = tmem + lane_off + (uint32_t)a * 256 + (uint32_t)c0;
+      float rinv = 1.f;
+      if (fused) {
+        uint32_t u0[32], u1[32];
+        tmem_ld32(acc, u0);
+        tmem_ld32(acc + 32, u1);
+        tmem_wait_ld();
+        float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 ab = make_float2(__uint_as_float(u0[i]), __uint_as_float(u1[i]));
+          ss2 = __ffma2_rn(ab, ab, ss2);
+        }
+        bars->ssq[hf][r] = ss2.x + ss2.y;
+        named_bar_sync(1, NT);  // both halves' sums of squares are in
+        rinv = rsqrtf((bars->ssq[0][r] + bars->ssq[1][r]) * (scale * scale) / (float)D + eps);
+      }
+      const float f_row = scale * rinv;  // o / rms(o) = num * scale * rinv
+      const float f_out = out8 ? f_row / a8_scale[it.h] : f_row;
+      const float gs = fast_sigmoid(gate1);
+      // this thread's 64 columns: bf16, box hf, chunks 0-7 of row r; e4m3, chunks 4hf .. 4hf+3
+      uint8_t *srow = stage + (out8 ? 0 : hf * (BM * 128)) + r * 128;
+#pragma unroll
+      for (int c = 0; c < HC; c += 32) {
+        uint32_t u[32], ug[32];
+        tmem_ld32(acc + c, u);
+        if (gate_mma) tmem_ld32(acc + 128 + c, ug);
+        tmem_wait_ld();
+#pragma unroll
+        for (int v = 0; v < 32; v += 8) {
+          float o8[8];
+          if (fused) {
+            const float2 *gg = reinterpret_cast<const float2 *>(&bars->gam[c0 + c + v]);
+            const float2 fo = make_float2(f_out, f_out);
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              float2 gl;
+              if (gate_mma) {
+                const float2 t = __fmul2_rn(make_float2(__uint_as_float(ug[v + e]), __uint_as_float(ug[v + e + 1])),
+                                            make_float2(0.5f, 0.5f));
+                gl = __ffma2_rn(make_float2(0.5f, 0.5f), make_float2(tanh_fast(t.x), tanh_fast(t.y)),
+                                make_float2(0.5f, 0.5f));
+              } else {
+                gl = make_float2(gs, gs);
+              }
+              const float2 o = __fmul2_rn(__fmul2_rn(gl, gg[e >> 1]),
+                                          __fmul2_rn(make_float2(__uint_as_float(u[v + e]), __uint_as_float(u[v + e + 1])), fo));
+              o8[e] = o.x;
+              o8[e + 1] = o.y;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o8[e] = __uint_as_float(u[v + e]) * f_out;
+          }
+          if (out8) {
+            uint32_t w2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(o8[4 * e], o8[4 * e + 1]), __NV_SATFINITE, __NV_E4M3);
+              const uint32_t hi =
+                  __nv_cvt_float2_to_fp8x2(make_float2(o8[4 * e + 2], o8[4 * e + 3]), __NV_SATFINITE, __NV_E4M3);
+              w2[e] = (lo & 0xffffu) | (hi << 16);
+            }
+            const int byte = c0 + c + v;  // 8 bytes inside 16-byte chunk byte / 16
+            *reinterpret_cast<uint2 *>(srow + ((((byte >> 4) ^ (r & 7))) << 4) + (byte & 15)) =
+                make_uint2(w2[0], w2[1]);
+          } else {
+            *reinterpret_cast<uint4 *>(srow + ((((c + v) >> 3) ^ (r & 7)) << 4)) = pack8(o8);
+          }
+        }
+      }
+      // accumulator set a is free once every warp's tensor-memory reads are done
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty[a]));
+      fence_proxy_async();    // the staged values, for the TMA store
+      named_bar_sync(1, NT);  // the staged rows are complete
+      const int nrows = min(BM, it.row_end - it.row0);
+      if (nrows == BM) {
+        if (et == 0) {
+          if (out8) {
+            tma_store_2d(&tmO, smem_u32(stage), it.h * D, it.row0);
+          } else {
+            tma_store_2d(&tmO, smem_u32(stage), it.h * D, it.row0);
+            tma_store_2d(&tmO, smem_u32(stage + BM * 128), it.h * D + 64, it.row0);
+          }
+          bulk_commit_group();
+        }
+      } else if (out8) {
+        // four rows per warp instruction: eight lanes per 128-byte row
+        for (int rr = (et >> 5) * 4 + (lane >> 3); rr < nrows; rr += 4 * ROLE_WARPS) {
+          const int j = lane & 7;
+          const uint4 val = *reinterpret_cast<const uint4 *>(stage + rr * 128 + ((j ^ (rr & 7)) << 4));
+          *reinterpret_cast<uint4 *>((uint8_t *)out + (int64_t)(it.row0 + rr) * out_stride + (int64_t)it.h * D +
+                                     j * 16) = val;
+        }
+      } else {
+        // two rows per warp instruction: lanes 0-15 one row, 16-31 the next (256 bytes each)
+        for (int rr = (et >> 5) * 2 + (lane >> 4); rr < nrows; rr += 2 * ROLE_WARPS) {
+          const int j = lane & 15;
+          const uint4 val =
+              *reinterpret_cast<const uint4 *>(stage + (j >> 3) * (BM * 128) + rr * 128 + (((j & 7) ^ (rr & 7)) << 4));
+          *reinterpret_cast<uint4 *>((__nv_bfloat16 *)out + (int64_t)(it.row0 + rr) * out_stride + (int64_t)it.h * D +
+                                     j * 8) = val;
+        }
+      }
+      ++k;
+    }
+    if (et == 0) bulk_wait_all();  // every TMA store of this block has completed
   }
   tc_fence_before();
   __syncthreads();
@@ -709,6 +846,7 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
   const int G = host_group_count(d);
   const bool fused = wgl != nullptr;
   const bool gate_mma = fused && G_l == D;
+  if (a8_scale != nullptr && !fused) return cudaErrorInvalidValue;
   CUtensorMap mq, ms, mw;
   {
     uint64_t dims[2] = {HD, (uint64_t)d.Nv()}, strides[1] = {HD * 2};
@@ -730,8 +868,18 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
   const int64_t stride = fused ? 2 * (int64_t)HD : (int64_t)HD;
   // fused: the linear half of A (bf16, or e4m3 codes with a8_scale)
   void *o = (a8_scale != nullptr) ? (void *)((uint8_t *)out + HD) : (void *)((__nv_bfloat16 *)out + (fused ? HD : 0));
-  if (a8_scale != nullptr && !fused) return cudaErrorInvalidValue;
-  const unsigned grid = (unsigned)(2 * host_tile_count(d) * d.H);
+  CUtensorMap mo;  // the output rows' H*D columns (the linear half of A when fused)
+  {
+    uint64_t dims[2] = {HD, (uint64_t)d.Nv()};
+    uint64_t strides[1] = {(uint64_t)stride * (a8_scale != nullptr ? 1 : 2)};
+    uint32_t box[2] = {a8_scale != nullptr ? 128u : 64u, (uint32_t)BM};
+    if (!encode_tmap(&mo, a8_scale != nullptr ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, o,
+                     dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  const int n_tiles = host_tile_count(d);
+  const int64_t n_items = (int64_t)2 * n_tiles * d.H;
+  const int grid = (int)(n_items < sm_count() ? n_items : sm_count());  // persistent: one CTA per SM
   const float *zs = (const float *)(ws + p.zsum);
   const int32_t *tl = (const int32_t *)(ws + p.tiles);
   DevStatus *sp = (DevStatus *)(ws + p.status);
@@ -739,8 +887,8 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<grid, THREADS, SMEM, st>>>(mq, ms, mw, d, zs, fused ? wgl : nullptr, G_l, gamma, eps, o, stride, tl,
-                                      a8_scale, sp);
+    kern<<<grid, THREADS, SMEM, st>>>(mq, ms, mw, mo, d, zs, fused ? wgl : nullptr, G_l, gamma, eps, o, stride, tl,
+                                      n_tiles, n_items, a8_scale, sp);
     return cudaGetLastError();
   };
   if (delta) {
