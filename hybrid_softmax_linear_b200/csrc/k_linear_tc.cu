@@ -327,9 +327,11 @@ __global__ void __launch_bounds__(256) read_stage_kernel(int64_t n_s8, int64_t n
 //               soon as the Q tile has landed, then num = feature * S_sum once the feature
 //               rows are written; two accumulator sets of 256 columns
 //   warps 4-11  two threads per query row, one per column half: that half of the feature
-//               row phi(q) (or q/|q|), written over the Q tile once the gate MMA has read
-//               it, and its share of the normaliser phi(q).z and (G_l = 1) the scalar gate
-//               logit
+//               row phi(q), written over the Q tile once the gate MMA has read it, and its
+//               share of the normaliser phi(q).z (delta rule: of |q|^2; the MMAs read q and
+//               the epilogue divides by |q|) and (G_l = 1) of the scalar gate logit; then
+//               (G_l = D) that half of the gate sigmoid(Q W_l), in place over its logits
+//               in tensor memory
 //   warps 12-19 epilogue, two threads per row: o = num / den from tensor memory, then o or
 //               A_l = g_l * gamma * o / rms(o) (the halves' sums of squares meet in shared
 //               memory), staged in shared memory and written by a TMA store that runs on
@@ -583,23 +585,11 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->q_full[s]), (k / NQ) & 1, abort_flag, st, K_READ, 11)))
         break;
       uint8_t *qt = base + Q_OFF + s * TILE_BYTES;
-      float inv_norm = 1.f;
-      if (delta) {
-        // |q|^2 over the whole row, by each of its two threads
-        float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int cl = 0; cl < D / 8; ++cl) {
-          const uint4 raw = *reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM));
-          const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 x2 = __bfloat1622float2(hp[e]);
-            ss2 = __ffma2_rn(x2, x2, ss2);
-          }
-        }
-        const float qq = ss2.x + ss2.y;
-        inv_norm = qq > 0.f ? rsqrtf(qq) : 0.f;
-      }
+      // ELU1: this half of phi(q) and of the normaliser phi(q).z.  Delta rule: no feature
+      // rows at all; the MMAs take q itself (q/|q| . S = (q . S) / |q|), and this half's
+      // share of |q|^2 goes where the normaliser would, for the epilogue to apply 1/|q|.
+      // (Each half reads only its own columns of the tile: the other half's thread may
+      // already be writing its features over the rest.)
       uint32_t fr[HC / 2];
       float2 den2 = make_float2(0.f, 0.f);
       float gate1 = 0.f;
@@ -617,14 +607,14 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
             gate1 = fmaf(xv.x, wv.x, fmaf(xv.y, wv.y, gate1));
           }
           if (delta) {
-            xv = __fmul2_rn(xv, make_float2(inv_norm, inv_norm));
+            den2 = __ffma2_rn(xv, xv, den2);
           } else {
             // elu + 1 as max(x, 0) + 2^(min(x, 0) log2 e): no branch
             const float2 e2 = __fmul2_rn(make_float2(fminf(xv.x, 0.f), fminf(xv.y, 0.f)), l2e);
             xv = __fadd2_rn(make_float2(fmaxf(xv.x, 0.f), fmaxf(xv.y, 0.f)), make_float2(ex2f(e2.x), ex2f(e2.y)));
             den2 = __ffma2_rn(xv, *reinterpret_cast<const float2 *>(&bars->zs[cl * 8 + 2 * e]), den2);
+            fr[i * 4 + e] = pack_bf16(xv.x, xv.y);
           }
-          fr[i * 4 + e] = pack_bf16(xv.x, xv.y);
         }
       }
       // Q is the A operand of the gate MMA: the features go over it only afterwards.
@@ -633,18 +623,43 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
       if (!__all_sync(0xffffffffu,
                       mbar_wait(smem_u32(&bars->gate_done[s]), (k / NQ) & 1, abort_flag, st, K_READ, 12)))
         break;
+      if (!delta) {
 #pragma unroll
-      for (int i = 0; i < HC / 8; ++i)
-        *reinterpret_cast<uint4 *>(qt + swz_off(r, c0 / 8 + i, BM)) =
-            make_uint4(fr[i * 4], fr[i * 4 + 1], fr[i * 4 + 2], fr[i * 4 + 3]);
+        for (int i = 0; i < HC / 8; ++i)
+          *reinterpret_cast<uint4 *>(qt + swz_off(r, c0 / 8 + i, BM)) =
+              make_uint4(fr[i * 4], fr[i * 4 + 1], fr[i * 4 + 2], fr[i * 4 + 3]);
+      }
       bars->den[a][hf][r] = den2.x + den2.y;
       bars->g1[a][hf][r] = gate1;
       fence_proxy_async();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(&bars->feat_full[s]));
-        mbar_arrive(smem_u32(&bars->den_full[a]));
+      if (lane == 0) mbar_arrive(smem_u32(&bars->feat_full[s]));
+      if (gate_mma) {
+        // the element-wise gate sigmoid(Q W_l) in place over its logits in tensor memory (the
+        // gate MMA has completed: gate_done), so the epilogue only multiplies
+        const uint32_t ga = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)a * 256 + 128 + (uint32_t)c0;
+        tc_fence_after();  // the logits were written by the gate MMA that gate_done saw complete
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) {
+          uint32_t ug[32];
+          tmem_ld32(ga + c, ug);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float2 t = __fmul2_rn(make_float2(__uint_as_float(ug[i]), __uint_as_float(ug[i + 1])),
+                                        make_float2(0.5f, 0.5f));
+            const float2 g = __ffma2_rn(make_float2(0.5f, 0.5f), make_float2(tanh_fast(t.x), tanh_fast(t.y)),
+                                        make_float2(0.5f, 0.5f));
+            ug[i] = __float_as_uint(g.x);
+            ug[i + 1] = __float_as_uint(g.y);
+          }
+          tmem_st32(ga + c, ug);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
       }
+      if (lane == 0) mbar_arrive(smem_u32(&bars->den_full[a]));
       ++k;
     }
   } else if (warp >= EPI_WARP0) {
@@ -675,9 +690,10 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
       // the previous item's stores have finished reading once all of them are here
       if (!named_bar_and(1, NT, got)) break;
       tc_fence_after();
+      // ELU1: the normaliser phi(q).z; delta rule: |q|^2 (o = (q . S) / |q|)
       const float den = bars->den[a][0][r] + bars->den[a][1][r];
       const float gate1 = bars->g1[a][0][r] + bars->g1[a][1][r];
-      const float scale = delta ? 1.f : (den > 0.f ? 1.f / den : 0.f);
+      const float scale = delta ? (den > 0.f ? rsqrtf(den) : 0.f) : (den > 0.f ? 1.f / den : 0.f);
       const uint32_t acc = tmem + lane_off + (uint32_t)a * 256 + (uint32_t)c0;
       float rinv = 1.f;
       if (fused) {
@@ -716,10 +732,7 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
             for (int e = 0; e < 8; e += 2) {
               float2 gl;
               if (gate_mma) {
-                const float2 t = __fmul2_rn(make_float2(__uint_as_float(ug[v + e]), __uint_as_float(ug[v + e + 1])),
-                                            make_float2(0.5f, 0.5f));
-                gl = __ffma2_rn(make_float2(0.5f, 0.5f), make_float2(tanh_fast(t.x), tanh_fast(t.y)),
-                                make_float2(0.5f, 0.5f));
+                gl = make_float2(__uint_as_float(ug[v + e]), __uint_as_float(ug[v + e + 1]));  // sigmoid, in place
               } else {
                 gl = make_float2(gs, gs);
               }
