@@ -6,7 +6,10 @@
 // round-to-nearest-even, saturating e4m3 of x / s; the softmax kernel multiplies the
 // scales back in.  Two passes: an amax reduction (per-block maxima in shared memory,
 // then one atomicMax per head and block on the float bit pattern, which orders like
-// the value for non-negative floats) and the cast.
+// the value for non-negative floats) and the cast.  Where the layer's linear branch
+// reads every value of Q, K and V anyway (the delta rule's frame statistics, text init
+// and read), those kernels leave the per-head maxima behind and only the cast runs here
+// (launch_fp8_cast): one pass over the bf16 inputs.
 #include "vdn_internal.cuh"
 
 namespace vdn {
@@ -118,6 +121,21 @@ cudaError_t launch_fp8_quant(const Dims &d, const void *q, const void *k, const 
   if (e != cudaSuccess) return e;
   fp8_scale_kernel<<<(3 * d.H + 255) / 256, 256, 0, st>>>(3 * d.H, amax_bits, scales);
   e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  fp8_cast_kernel<<<dim3(4096, 3), 256, 0, st>>>(d, s, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_cast(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
+                            const void *vt, void *q8, void *k8, void *v8, void *kt8, void *vt8, float *scales,
+                            const uint32_t *amax_bits, cudaStream_t st) {
+  Src s;
+  s.video[0] = (const __nv_bfloat16 *)q; s.video[1] = (const __nv_bfloat16 *)k; s.video[2] = (const __nv_bfloat16 *)v;
+  s.text[0] = nullptr; s.text[1] = (const __nv_bfloat16 *)kt; s.text[2] = (const __nv_bfloat16 *)vt;
+  s.video8[0] = (uint8_t *)q8; s.video8[1] = (uint8_t *)k8; s.video8[2] = (uint8_t *)v8;
+  s.text8[0] = nullptr; s.text8[1] = (uint8_t *)kt8; s.text8[2] = (uint8_t *)vt8;
+  fp8_scale_kernel<<<(3 * d.H + 255) / 256, 256, 0, st>>>(3 * d.H, amax_bits, scales);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   fp8_cast_kernel<<<dim3(4096, 3), 256, 0, st>>>(d, s, scales);
   return cudaGetLastError();

@@ -409,17 +409,20 @@ __device__ __forceinline__ bool read_item(const int32_t *__restrict__ tiles, int
 }
 
 // DELTA: q/|q| features and no normaliser; FUSED: RMSNorm and the linear gate (GATE_MMA:
-// element-wise, G_l = D, on the tensor cores; otherwise the scalar gate, G_l = 1)
-template <bool DELTA, bool FUSED, bool GATE_MMA>
+// element-wise, G_l = D, on the tensor cores; otherwise the scalar gate, G_l = 1); AMAX:
+// also the per-head max |q| into amax_q (for the e4m3 quantisation that follows)
+template <bool DELTA, bool FUSED, bool GATE_MMA, bool AMAX>
 __global__ void __launch_bounds__(rd::THREADS, 1)
     read_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                    const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmO, Dims d,
                    const float *__restrict__ zsum, const float *__restrict__ wgl, int G_l,
                    const float *__restrict__ gamma, float eps, void *__restrict__ out, int64_t out_stride,
                    const int32_t *__restrict__ tiles, int n_tiles,
-                   int64_t n_items, const float *__restrict__ a8_scale, DevStatus *st) {
+                   int64_t n_items, const float *__restrict__ a8_scale, uint32_t *__restrict__ amax_q,
+                   DevStatus *st) {
   using namespace rd;
   constexpr bool delta = DELTA, fused = FUSED, gate_mma = FUSED && GATE_MMA, scalar_gate = FUSED && !GATE_MMA;
+  constexpr bool amax = AMAX;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   Bars *bars = reinterpret_cast<Bars *>(base + BAR_OFF);
@@ -569,6 +572,17 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
     // ---------------------------------------------------------------- feature rows
     const int r = (warp & 3) * 32 + lane, hf = (warp - FEAT_WARP0) >> 2, c0 = hf * HC;
     int k = 0, ns = 0, cur_s = -1;
+    // amax_q: this warp's max |q| over the items of head qh, flushed (one atomicMax per warp)
+    // when the head changes and at the end
+    float qmax = 0.f;
+    int qh = -1;
+    auto flush_qmax = [&]() {
+      float m = qmax;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0 && qh >= 0) atomicMax(&amax_q[qh], __float_as_uint(m));
+      qmax = 0.f;
+    };
     for (int64_t x = x0; x < x1; ++x) {
       ReadItem it;
       if (!read_item(tiles, n_tiles, d, st, x, it)) continue;
@@ -580,6 +594,10 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full), ns & 1, abort_flag, st, K_READ, 15))) break;
         ++ns;
         cur_s = key;
+      }
+      if (amax && it.h != qh) {  // warp-uniform
+        flush_qmax();
+        qh = it.h;
       }
       // the warp proceeds (or gives up) as a whole
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->q_full[s]), (k / NQ) & 1, abort_flag, st, K_READ, 11)))
@@ -602,6 +620,7 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float2 xv = __bfloat1622float2(hp[e]);
+          if (amax) qmax = fmaxf(qmax, fmaxf(fabsf(xv.x), fabsf(xv.y)));
           if (scalar_gate) {
             const float2 wv = *reinterpret_cast<const float2 *>(&bars->wg1[cl * 8 + 2 * e]);
             gate1 = fmaf(xv.x, wv.x, fmaf(xv.y, wv.y, gate1));
@@ -662,6 +681,7 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
       if (lane == 0) mbar_arrive(smem_u32(&bars->den_full[a]));
       ++k;
     }
+    if (amax) flush_qmax();
   } else if (warp >= EPI_WARP0) {
     // ---------------------------------------------------------------- epilogue
     const int quad = warp & 3, r = quad * 32 + lane, hf = (warp - EPI_WARP0) >> 2, c0 = hf * HC;
@@ -853,7 +873,7 @@ cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf,
 
 cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void *out, const float *wgl, int G_l,
                            const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st,
-                           const float *a8_scale) {
+                           const float *a8_scale, uint32_t *amax_q) {
   using namespace rd;
   const uint64_t HD = (uint64_t)d.H * D;
   const int G = host_group_count(d);
@@ -901,15 +921,19 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
     if (e != cudaSuccess) return e;
     kern<<<grid, THREADS, SMEM, st>>>(mq, ms, mw, mo, d, zs, fused ? wgl : nullptr, G_l, gamma, eps, o, stride, tl,
-                                      n_tiles, n_items, a8_scale, sp);
+                                      n_tiles, n_items, a8_scale, amax_q, sp);
     return cudaGetLastError();
   };
-  if (delta) {
-    if (!fused) return go(read_tc_kernel<true, false, false>);
-    return gate_mma ? go(read_tc_kernel<true, true, true>) : go(read_tc_kernel<true, true, false>);
+  if (amax_q != nullptr) {  // the max |q| by-product: the delta rule's gated layer only
+    if (!(delta && gate_mma)) return cudaErrorInvalidValue;
+    return go(read_tc_kernel<true, true, true, true>);
   }
-  if (!fused) return go(read_tc_kernel<false, false, false>);
-  return gate_mma ? go(read_tc_kernel<false, true, true>) : go(read_tc_kernel<false, true, false>);
+  if (delta) {
+    if (!fused) return go(read_tc_kernel<true, false, false, false>);
+    return gate_mma ? go(read_tc_kernel<true, true, true, false>) : go(read_tc_kernel<true, true, false, false>);
+  }
+  if (!fused) return go(read_tc_kernel<false, false, false, false>);
+  return gate_mma ? go(read_tc_kernel<false, true, true, false>) : go(read_tc_kernel<false, true, false, false>);
 }
 
 }  // namespace vdn

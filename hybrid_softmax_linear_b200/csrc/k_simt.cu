@@ -125,6 +125,23 @@ cudaError_t launch_softmax_simt(const Dims &d, vdn_dtype dt, const void *q, cons
   return cudaErrorInvalidValue;
 }
 
+// Block-wide maximum of a non-negative float (every thread passes its own), then one
+// atomicMax on the float's bit pattern (which orders like the value for non-negative
+// floats) by thread 0.  red: shared scratch of blockDim.x / 32 floats.  Every thread of the
+// block must call it.
+__device__ __forceinline__ void block_amax_to(float m, float *red, uint32_t *dst) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t = fmaxf(t, red[w]);
+    atomicMax(dst, __float_as_uint(t));
+  }
+}
+
 // ------------------------------------------------------------------ per-frame states
 // Block per (frame or text, head).  Tokens are staged 32 at a time in shared memory as
 // float (phi(k) or the L2-normalised key for the delta text init, and v); thread t owns
@@ -134,7 +151,7 @@ __global__ void __launch_bounds__(256) state_build_kernel(Dims d, const T *__res
                                                           const T *__restrict__ kt, const T *__restrict__ vt,
                                                           float *__restrict__ S, float *__restrict__ z,
                                                           float *__restrict__ St, float *__restrict__ zt,
-                                                          int nframes, int normalise_rows) {
+                                                          int nframes, int normalise_rows, uint32_t *__restrict__ amax) {
   constexpr int R = D / 16, TK = 32;
   __shared__ float ks[TK][D], vs[TK][D];
   const int h = blockIdx.y, tid = threadIdx.x;
@@ -148,7 +165,7 @@ __global__ void __launch_bounds__(256) state_build_kernel(Dims d, const T *__res
   for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int c = 0; c < R; ++c) acc[r][c] = 0.f;
-  float zacc = 0.f;
+  float zacc = 0.f, ak = 0.f, av = 0.f;  // ak, av: max |k|, |v| of the rows read (amax)
   const int i0 = tid >> 4, j0 = tid & 15;
   for (int t0 = 0; t0 < ntok; t0 += TK) {
     const int nt = min(TK, ntok - t0);
@@ -158,6 +175,8 @@ __global__ void __launch_bounds__(256) state_build_kernel(Dims d, const T *__res
       if (t < nt) {
         kx = to_f(kb[(int64_t)(t0 + t) * HD + h * D + i]);
         vx = to_f(vb[(int64_t)(t0 + t) * HD + h * D + i]);
+        ak = fmaxf(ak, fabsf(kx));
+        av = fmaxf(av, fabsf(vx));
         if (!normalise_rows) kx = phi_elu1(kx);
       }
       ks[t][i] = kx; vs[t][i] = vx;
@@ -195,6 +214,11 @@ __global__ void __launch_bounds__(256) state_build_kernel(Dims d, const T *__res
     for (int c = 0; c < R; ++c) So[(i0 + 16 * r) * D + j0 + 16 * c] = acc[r][c];
   float *zo = text ? zt : z;
   if (zo != nullptr && tid < D) zo[(text ? (int64_t)h * D : ((int64_t)blockIdx.x * d.H + h) * D) + tid] = zacc;
+  if (amax != nullptr && text) {  // block-uniform: the delta text init's max |k|, |v| per head
+    __shared__ float red[256 / 32];
+    block_amax_to(ak, red, amax + d.H + h);
+    block_amax_to(av, red, amax + 2 * d.H + h);
+  }
 }
 
 // Delta-rule frame statistics: kbar = mean key (L2-normalised), vbar = mean value.
@@ -224,10 +248,13 @@ __global__ void __launch_bounds__(D) delta_stats_kernel(Dims d, const T *__restr
 // head with 16-byte loads (8 values each) and the block's 16 token slices are summed
 // through shared memory; then kbar is L2-normalised.
 constexpr int DS_THREADS = 256, DS_SLICES = DS_THREADS / 16;
+// amax (optional): the per-head max |k| and |v| of these rows go into amax[H + h] and
+// amax[2H + h] (float bits), as a by-product of reading them
 __global__ void __launch_bounds__(DS_THREADS) delta_stats_bf16_kernel(Dims d, const __nv_bfloat16 *__restrict__ k,
                                                                       const __nv_bfloat16 *__restrict__ v,
                                                                       float *__restrict__ kbar,
-                                                                      float *__restrict__ vbar) {
+                                                                      float *__restrict__ vbar,
+                                                                      uint32_t *__restrict__ amax) {
   constexpr int D = 128;
   __shared__ float acc[2][DS_SLICES][D];
   __shared__ float nrm;
@@ -236,7 +263,7 @@ __global__ void __launch_bounds__(DS_THREADS) delta_stats_bf16_kernel(Dims d, co
   const int64_t HD = (int64_t)d.H * D;
   const __nv_bfloat16 *kb = k + (int64_t)f * d.T * HD + h * D + c8;
   const __nv_bfloat16 *vb = v + (int64_t)f * d.T * HD + h * D + c8;
-  float sk[8], sv[8];
+  float sk[8], sv[8], ak = 0.f, av = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) sk[e] = sv[e] = 0.f;
 #pragma unroll 4
@@ -246,6 +273,15 @@ __global__ void __launch_bounds__(DS_THREADS) delta_stats_bf16_kernel(Dims d, co
     load8(vb + (int64_t)t * HD, b);
 #pragma unroll
     for (int e = 0; e < 8; ++e) { sk[e] += a[e]; sv[e] += b[e]; }
+    if (amax != nullptr) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { ak = fmaxf(ak, fabsf(a[e])); av = fmaxf(av, fabsf(b[e])); }
+    }
+  }
+  if (amax != nullptr) {  // block-uniform
+    __shared__ float red[DS_THREADS / 32];
+    block_amax_to(ak, red, amax + d.H + h);
+    block_amax_to(av, red, amax + 2 * d.H + h);
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) { acc[0][sl][c8 + e] = sk[e]; acc[1][sl][c8 + e] = sv[e]; }
@@ -275,28 +311,31 @@ __global__ void __launch_bounds__(DS_THREADS) delta_stats_bf16_kernel(Dims d, co
 
 template <typename T, int D>
 static cudaError_t state_build_t(const Dims &d, vdn_lin_kind kind, const void *k, const void *v, const void *kt,
-                                 const void *vt, float *S, float *z, float *St, float *zt, cudaStream_t st) {
+                                 const void *vt, float *S, float *z, float *St, float *zt, cudaStream_t st,
+                                 uint32_t *amax) {
   if (kind == VDN_LIN_ELU1) {
     state_build_kernel<T, D><<<dim3(d.F + 1, d.H), 256, 0, st>>>(d, (const T *)k, (const T *)v, (const T *)kt,
-                                                                 (const T *)vt, S, z, St, zt, d.F, 0);
+                                                                 (const T *)vt, S, z, St, zt, d.F, 0, nullptr);
     return cudaGetLastError();
   }
   if constexpr (D == 128 && sizeof(T) == 2)
-    delta_stats_bf16_kernel<<<dim3(d.F, d.H), DS_THREADS, 0, st>>>(d, (const T *)k, (const T *)v, S, z);
+    delta_stats_bf16_kernel<<<dim3(d.F, d.H), DS_THREADS, 0, st>>>(d, (const T *)k, (const T *)v, S, z, amax);
   else
     delta_stats_kernel<T, D><<<dim3(d.F, d.H), D, 0, st>>>(d, (const T *)k, (const T *)v, S, z);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // text init only: one block per head, with L2-normalised text keys
   state_build_kernel<T, D><<<dim3(1, d.H), 256, 0, st>>>(d, (const T *)k, (const T *)v, (const T *)kt,
-                                                         (const T *)vt, nullptr, nullptr, St, nullptr, 0, 1);
+                                                         (const T *)vt, nullptr, nullptr, St, nullptr, 0, 1, amax);
   return cudaGetLastError();
 }
 
 cudaError_t launch_state_build(const Dims &d, vdn_lin_kind kind, vdn_dtype dt, const void *k, const void *v,
                                const void *kt, const void *vt, float *S, float *z, float *St, float *zt,
-                               cudaStream_t st) {
-#define VDN_SB(T, DD) return state_build_t<T, DD>(d, kind, k, v, kt, vt, S, z, St, zt, st)
+                               cudaStream_t st, uint32_t *amax) {
+  // the amax by-product exists on the delta rule's bf16, D = 128 path only
+  if (amax != nullptr && !(kind == VDN_LIN_DELTA && dt == VDN_BF16 && d.D == 128)) return cudaErrorInvalidValue;
+#define VDN_SB(T, DD) return state_build_t<T, DD>(d, kind, k, v, kt, vt, S, z, St, zt, st, amax)
   if (dt == VDN_F32) {
     if (d.D == 32) VDN_SB(float, 32);
     if (d.D == 64) VDN_SB(float, 64);

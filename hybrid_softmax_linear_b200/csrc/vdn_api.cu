@@ -151,13 +151,13 @@ vdn_status softmax_dispatch(const Dims &d, vdn_dtype dt, const void *q, const vo
 
 vdn_status state_build_dispatch(const Dims &d, vdn_lin_kind kind, vdn_dtype act, const void *k, const void *v,
                                 const void *kt, const void *vt, float *S, float *z, float *St, float *zt, char *ws,
-                                const WsPlan &p, cudaStream_t st) {
+                                const WsPlan &p, cudaStream_t st, uint32_t *amax = nullptr) {
   if (kind == VDN_LIN_ELU1 && linear_tc_supported(d, act)) {
     ProfScope ps(K_STATE_TC, st);
     VDN_CUDA(launch_state_build_tc(d, k, v, kt, vt, S, z, St, zt, ws, p, st), "state build (tensor cores) launch");
   } else {
     ProfScope ps(K_STATE, st);
-    VDN_CUDA(launch_state_build(d, kind, act, k, v, kt, vt, S, z, St, zt, st), "state build launch");
+    VDN_CUDA(launch_state_build(d, kind, act, k, v, kt, vt, S, z, St, zt, st, amax), "state build launch");
   }
   return VDN_OK;
 }
@@ -422,9 +422,16 @@ vdn_status layer_impl(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype
   }
   if (layer_fused(*shape, dtype)) {
     // tensor-core path: the softmax epilogue writes A_s = g_s * O_s and the linear read
-    // writes A_l = g_l * gamma * RMSNorm(O_l), both straight into A
+    // writes A_l = g_l * gamma * RMSNorm(O_l), both straight into A.
+    // e4m3 softmax with the delta rule: the frame statistics, the text init and the read
+    // read every value of Q, K and V anyway, so they leave the per-head maxima behind, the
+    // read runs before the softmax, and the quantisation is a single cast pass.
+    const bool fold_amax = dtype_e4m3_softmax(dtype) && !a8 && kind == VDN_LIN_DELTA && act == VDN_BF16 &&
+                           d.D == 128 && linear_tc_supported(d, act);
+    uint32_t *amax = (uint32_t *)(w + p.amax);
+    if (fold_amax) VDN_CUDA(cudaMemsetAsync(amax, 0, 3 * (size_t)d.H * sizeof(uint32_t), st), "amax clear");
     VDN_TRY(state_build_dispatch(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, w, p,
-                                 st));
+                                 st, fold_amax ? amax : nullptr));
     const bool seg = layer_seg_scan(*shape, kind);
     {
       ProfScope ps(K_SCAN, st);
@@ -437,7 +444,23 @@ vdn_status layer_impl(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype
       ProfScope ps(K_READ_STAGE, st);
       VDN_CUDA(launch_read_stage(d, kind, seg ? nullptr : Sf, Sb, zf, zb, w_gate_l, G_l, w, p, st), "read staging");
     }
-    if (dtype_e4m3_softmax(dtype)) {
+    if (fold_amax) {
+      {
+        ProfScope ps(K_READ_TC, st);
+        VDN_CUDA(launch_read_tc(d, kind, q, A, w_gate_l, G_l, gamma, eps, w, p, st, nullptr, amax), "read launch");
+      }
+      {
+        ProfScope ps(K_QUANT, st);
+        VDN_CUDA(launch_fp8_cast(d, q, k, v, kt, vt, w + p.q8, w + p.k8, w + p.v8, w + p.kt8, w + p.vt8,
+                                 (float *)(w + p.scales), amax, st),
+                 "fp8 cast launch");
+      }
+      ProfScope ps(K_SOFTMAX_TC, st);
+      VDN_CUDA(launch_softmax_tc_gated(d, VDN_E4M3, w + p.q8, w + p.k8, w + p.v8, w + p.kt8, w + p.vt8,
+                                       (const float *)(w + p.scales), w_gate_s, scale_log2_of(0.f, d.D), A, w, p, st,
+                                       false),
+               "softmax branch (tensor cores, e4m3) launch");
+    } else if (dtype_e4m3_softmax(dtype)) {
       // per-head e4m3 Q/K/V for the softmax branch; the linear branch keeps the bf16 inputs
       {
         ProfScope ps(K_QUANT, st);
@@ -459,7 +482,7 @@ vdn_status layer_impl(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype
                                        p, st),
                "softmax branch (tensor cores) launch");
     }
-    {
+    if (!fold_amax) {
       ProfScope ps(K_READ_TC, st);
       VDN_CUDA(launch_read_tc(d, kind, q, A, w_gate_l, G_l, gamma, eps, w, p, st, a8 ? ascale + d.H : nullptr),
                "read launch");

@@ -350,9 +350,11 @@ cudaError_t launch_softmax_tc(const Dims &d, vdn_dtype dt, const void *q, const 
                               float *lse, char *ws, const WsPlan &p, cudaStream_t st);
 bool softmax_tc_supported(const Dims &d, vdn_dtype dt);
 
+// amax (delta rule, bf16, D = 128 only): also the per-head max |k|, |v| of the video and text
+// rows, atomicMax'ed into amax[H + h], amax[2H + h] (float bits; zeroed by the caller)
 cudaError_t launch_state_build(const Dims &d, vdn_lin_kind kind, vdn_dtype dt, const void *k, const void *v,
                                const void *kt, const void *vt, float *S, float *z, float *St, float *zt,
-                               cudaStream_t st);
+                               cudaStream_t st, uint32_t *amax = nullptr);
 cudaError_t launch_state_scan(const Dims &d, vdn_lin_kind kind, const float *S, const float *z, const float *St,
                               const float *zt, const float *beta, float *Sf, float *Sb, float *zf, float *zb,
                               char *ws, const WsPlan &p, cudaStream_t st);
@@ -377,7 +379,7 @@ cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf,
 // a8_scale (fused only): A_l written as e4m3 codes in units of a8_scale[h]
 cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void *out, const float *wgl, int G_l,
                            const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st,
-                           const float *a8_scale = nullptr);
+                           const float *a8_scale = nullptr, uint32_t *amax_q = nullptr);  // amax_q: per-head max |q|
 // a8: A_s written as e4m3 codes in units of the V scale (e4m3 softmax only)
 cudaError_t launch_softmax_tc_gated(const Dims &d, vdn_dtype dt, const void *q, const void *k, const void *v,
                                     const void *kt, const void *vt, const float *scales, const float *w_gate_s,
@@ -386,6 +388,10 @@ cudaError_t launch_softmax_tc_gated(const Dims &d, vdn_dtype dt, const void *q, 
 cudaError_t launch_fp8_quant(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
                              const void *vt, void *q8, void *k8, void *v8, void *kt8, void *vt8, float *scales,
                              uint32_t *amax_bits, cudaStream_t st);
+// the cast alone, with amax_bits already holding every head's max |q|, |k|, |v|
+cudaError_t launch_fp8_cast(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
+                            const void *vt, void *q8, void *k8, void *v8, void *kt8, void *vt8, float *scales,
+                            const uint32_t *amax_bits, cudaStream_t st);
 constexpr int FP8_MAX_HD = 256 * 8 * 8;  // column chunks the amax pass keeps in registers
 
 cudaError_t launch_fuse(const Dims &d, vdn_dtype dt, const void *q, const void *os, const void *ol,
