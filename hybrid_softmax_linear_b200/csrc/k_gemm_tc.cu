@@ -300,15 +300,18 @@ __global__ void __launch_bounds__(256) w8_prep_kernel(const __nv_bfloat16 *__res
 // A_s = g_s O_s is a gated convex combination of V rows, so |A_s| <= amax(V_h), the e4m3
 // V scale's 448 (its scale is then that of V); A_l = g_l gamma O_l / rms(O_l) has
 // |A_l| <= max|gamma_h| sqrt(D), so its scale is that / 448.
+// halves: bit 0 the A_s scales (the V scales), bit 1 the A_l scales (from gamma alone)
 __global__ void a8_scale_kernel(int H, int D, const float *__restrict__ vscale, const float *__restrict__ gamma,
-                                float *__restrict__ ascale) {
+                                float *__restrict__ ascale, int halves) {
   const int h = blockIdx.x * blockDim.x + threadIdx.x;
   if (h >= H) return;
-  float g = 0.f;
-  for (int i = 0; i < D; ++i) g = fmaxf(g, fabsf(gamma[(int64_t)h * D + i]));
-  ascale[h] = vscale[h];
-  const float b = g * sqrtf((float)D) / 448.f;
-  ascale[H + h] = b > 0.f ? b : 1.f;
+  if (halves & 1) ascale[h] = vscale[h];
+  if (halves & 2) {
+    float g = 0.f;
+    for (int i = 0; i < D; ++i) g = fmaxf(g, fabsf(gamma[(int64_t)h * D + i]));
+    const float b = g * sqrtf((float)D) / 448.f;
+    ascale[H + h] = b > 0.f ? b : 1.f;
+  }
 }
 
 }  // namespace
@@ -355,8 +358,9 @@ bool out_proj_e4m3_supported(const Dims &d) {
   return HD % 256 == 0 && HD >= 256;
 }
 
-cudaError_t launch_a8_scales(const Dims &d, const float *vscale, const float *gamma, float *ascale, cudaStream_t st) {
-  a8_scale_kernel<<<(d.H + 127) / 128, 128, 0, st>>>(d.H, d.D, vscale, gamma, ascale);
+cudaError_t launch_a8_scales(const Dims &d, const float *vscale, const float *gamma, float *ascale, cudaStream_t st,
+                             int halves) {
+  a8_scale_kernel<<<(d.H + 127) / 128, 128, 0, st>>>(d.H, d.D, vscale, gamma, ascale, halves);
   return cudaGetLastError();
 }
 

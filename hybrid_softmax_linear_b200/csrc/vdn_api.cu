@@ -426,8 +426,8 @@ vdn_status layer_impl(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype
     // e4m3 softmax with the delta rule: the frame statistics, the text init and the read
     // read every value of Q, K and V anyway, so they leave the per-head maxima behind, the
     // read runs before the softmax, and the quantisation is a single cast pass.
-    const bool fold_amax = dtype_e4m3_softmax(dtype) && !a8 && kind == VDN_LIN_DELTA && act == VDN_BF16 &&
-                           d.D == 128 && linear_tc_supported(d, act);
+    const bool fold_amax = dtype_e4m3_softmax(dtype) && kind == VDN_LIN_DELTA && act == VDN_BF16 && d.D == 128 &&
+                           linear_tc_supported(d, act) && w_gate_l != nullptr && G_l == d.D;
     uint32_t *amax = (uint32_t *)(w + p.amax);
     if (fold_amax) VDN_CUDA(cudaMemsetAsync(amax, 0, 3 * (size_t)d.H * sizeof(uint32_t), st), "amax clear");
     VDN_TRY(state_build_dispatch(d, kind, act, k, v, kt, vt, S, z, St, kind == VDN_LIN_ELU1 ? zt : nullptr, w, p,
@@ -445,20 +445,27 @@ vdn_status layer_impl(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype
       VDN_CUDA(launch_read_stage(d, kind, seg ? nullptr : Sf, Sb, zf, zb, w_gate_l, G_l, w, p, st), "read staging");
     }
     if (fold_amax) {
+      // e4m3 projection: A_l's scales come from gamma alone (before the read); A_s's are
+      // the V scales (after the cast)
+      if (a8) VDN_CUDA(launch_a8_scales(d, nullptr, gamma, ascale, st, 2), "A scale launch");
       {
         ProfScope ps(K_READ_TC, st);
-        VDN_CUDA(launch_read_tc(d, kind, q, A, w_gate_l, G_l, gamma, eps, w, p, st, nullptr, amax), "read launch");
+        VDN_CUDA(launch_read_tc(d, kind, q, A, w_gate_l, G_l, gamma, eps, w, p, st, a8 ? ascale + d.H : nullptr, amax),
+                 "read launch");
       }
       {
         ProfScope ps(K_QUANT, st);
         VDN_CUDA(launch_fp8_cast(d, q, k, v, kt, vt, w + p.q8, w + p.k8, w + p.v8, w + p.kt8, w + p.vt8,
                                  (float *)(w + p.scales), amax, st),
                  "fp8 cast launch");
+        if (a8)
+          VDN_CUDA(launch_a8_scales(d, (const float *)(w + p.scales) + 2 * d.H, gamma, ascale, st, 1),
+                   "A scale launch");
       }
       ProfScope ps(K_SOFTMAX_TC, st);
       VDN_CUDA(launch_softmax_tc_gated(d, VDN_E4M3, w + p.q8, w + p.k8, w + p.v8, w + p.kt8, w + p.vt8,
                                        (const float *)(w + p.scales), w_gate_s, scale_log2_of(0.f, d.D), A, w, p, st,
-                                       false),
+                                       a8),
                "softmax branch (tensor cores, e4m3) launch");
     } else if (dtype_e4m3_softmax(dtype)) {
       // per-head e4m3 Q/K/V for the softmax branch; the linear branch keeps the bf16 inputs

@@ -407,7 +407,9 @@ bool out_proj_tc_supported(const Dims &d);
 // e4m3 projection: A8 [N_v][2HD] codes with dequantisation scales ascale[2][H] (per branch
 // half and head), bf16 W_os, W_ol; w8 (HD x 2HD bytes) and wsc (HD floats) are scratch
 bool out_proj_e4m3_supported(const Dims &d);
-cudaError_t launch_a8_scales(const Dims &d, const float *vscale, const float *gamma, float *ascale, cudaStream_t st);
+// halves: 1 the A_s scales (= the V scales), 2 the A_l scales (from gamma), 3 both
+cudaError_t launch_a8_scales(const Dims &d, const float *vscale, const float *gamma, float *ascale, cudaStream_t st,
+                             int halves = 3);
 cudaError_t launch_out_proj_e4m3(const Dims &d, const void *a8, const float *ascale, const void *wos, const void *wol,
                                  void *y, uint8_t *w8, float *wsc, DevStatus *status, cudaStream_t st);
 cudaError_t launch_debug_wait(char *ws, uint32_t max_polls, cudaStream_t st);
