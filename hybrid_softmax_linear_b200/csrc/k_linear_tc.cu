@@ -50,6 +50,13 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
   return u;
 }
 
+// 2^x with the hardware approximation (flushes subnormal results to zero)
+__device__ __forceinline__ float ex2_sb(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ============================================================================ state build
 // Persistent: every CTA walks the (frame or text, head) items blockIdx.x, blockIdx.x +
 // gridDim.x, ... (heads vary fastest, so the CTAs in flight read whole token rows of K and
@@ -213,21 +220,32 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         uint8_t *kt = base + s * STAGE_BYTES;
+        // all four rows' loads first, so their latencies overlap (the stores below go to the
+        // same tile, which the compiler would otherwise keep in order with the next load)
+        constexpr int RI = TK / 16;
+        uint4 raw[RI];
 #pragma unroll
-        for (int i = 0; i < TK / 16; ++i) {
+        for (int i = 0; i < RI; ++i) raw[i] = *reinterpret_cast<const uint4 *>(kt + swz_off(rg + 16 * i, cl, TK));
+#pragma unroll
+        for (int i = 0; i < RI; ++i) {
           const int r = rg + 16 * i;
-          uint4 *p = reinterpret_cast<uint4 *>(kt + swz_off(r, cl, TK));
-          float f[8];
-          unpack8(*p, f);
           const bool valid = c * TK + r < it.ntok;
+          const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw[i]);
+          uint32_t w4[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            // phi enters the MMA in bf16, so the fast exponential is accurate enough
-            const float ph = valid ? phi_fast(f[e]) : 0.f;
-            zacc[e] += ph;
-            f[e] = ph;
+          for (int e = 0; e < 4; ++e) {
+            // phi = max(x, 0) + 2^(min(x, 0) log2 e) on pairs; phi enters the MMA in bf16, so
+            // the hardware exponential is accurate enough
+            const float2 x = __bfloat1622float2(hp[e]);
+            const float2 t = __fmul2_rn(make_float2(fminf(x.x, 0.f), fminf(x.y, 0.f)),
+                                        make_float2(1.4426950408889634f, 1.4426950408889634f));
+            float2 ph = __fadd2_rn(make_float2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)), make_float2(ex2_sb(t.x), ex2_sb(t.y)));
+            if (!valid) ph = make_float2(0.f, 0.f);
+            zacc[2 * e] += ph.x;
+            zacc[2 * e + 1] += ph.y;
+            w4[e] = pack_bf16(ph.x, ph.y);
           }
-          *p = pack8(f);
+          *reinterpret_cast<uint4 *>(kt + swz_off(r, cl, TK)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
         fence_proxy_async();
         __syncwarp();
