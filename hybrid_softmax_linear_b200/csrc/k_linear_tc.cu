@@ -58,9 +58,12 @@ __device__ __forceinline__ float ex2_sb(float x) {
 }
 
 // ============================================================================ state build
-// Persistent: every CTA walks the (frame or text, head) items blockIdx.x, blockIdx.x +
-// gridDim.x, ... (heads vary fastest, so the CTAs in flight read whole token rows of K and
-// V), two CTAs per SM.  The TMA ring of 64-token chunks runs on across items, so no CTA
+// Persistent: every CTA walks the (frame or text, head group) items blockIdx.x, blockIdx.x +
+// gridDim.x, ... (head groups vary fastest, so the CTAs in flight read whole token rows of K
+// and V), two CTAs per SM.  A head group is 128 features: one head of D = 128, or 128 / D
+// heads of D = 64 or 32, whose states are the diagonal D x D blocks of the group's 128 x 128
+// product (the tensor cores compute the off-diagonal blocks too, for free: the kernel is
+// bound by HBM).  The TMA ring of 64-token chunks runs on across items, so no CTA
 // waits for its first loads after the first item; the accumulator alternates between two
 // 128-column halves of tensor memory, so the MMAs of an item start while the previous
 // item's S is still being read out.
@@ -79,15 +82,15 @@ struct alignas(8) Bars {
 };
 constexpr size_t SMEM = 1024 + NS * STAGE_BYTES + sizeof(Bars);
 
-// item x: frame fr = x / H (fr == F: the text), head h = x % H; its rows and token count
+// item x: frame fr = x / Hg (fr == F: the text), head group h = x % Hg; its rows and tokens
 struct Item {
   int h, fr, row_base, ntok, nch;
   bool text;
 };
-__device__ __forceinline__ Item item_of(const Dims &d, int x) {
+__device__ __forceinline__ Item item_of(const Dims &d, int Hg, int x) {
   Item it;
-  it.h = x % d.H;
-  it.fr = x / d.H;
+  it.h = x % Hg;
+  it.fr = x / Hg;
   it.text = it.fr == d.F;
   it.ntok = it.text ? d.L : d.T;
   it.row_base = it.text ? 0 : it.fr * d.T;
@@ -111,7 +114,8 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
   if (threadIdx.x == 0) skip = *(volatile uint32_t *)&st->code != 0u;
   __syncthreads();
   if (skip) return;
-  const int n_items = (d.F + 1) * d.H;
+  const int Hg = d.H * d.D / D;  // head groups of 128 features
+  const int n_items = (d.F + 1) * Hg;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
       int gc = 0;
       bool go = true;
       for (int x = blockIdx.x; go && x < n_items; x += gridDim.x) {
-        const Item it = item_of(d, x);
+        const Item it = item_of(d, Hg, x);
         const CUtensorMap *mk = it.text ? &tmKt : &tmK;
         const CUtensorMap *mv = it.text ? &tmVt : &tmV;
         for (int c = 0; c < it.nch; ++c, ++gc) {
@@ -172,7 +176,7 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
       int gc = 0, na = 0;
       bool ok = true;
       for (int x = blockIdx.x; ok && x < n_items; x += gridDim.x) {
-        const Item it = item_of(d, x);
+        const Item it = item_of(d, Hg, x);
         if (it.nch == 0) continue;
         const int b = na & 1;
         // the accumulator's previous item has been read out
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
     int gc = 0, na = 0;
     bool ok = true;
     for (int x = blockIdx.x; x < n_items; x += gridDim.x) {
-      const Item it = item_of(d, x);
+      const Item it = item_of(d, Hg, x);
       float zacc[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
@@ -259,7 +263,9 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
 #pragma unroll
         for (int e = 0; e < 8; ++e) bars->zpart[warp - 2][cl * 8 + e] = zacc[e];
       }
-      float *So = it.text ? St + (int64_t)it.h * D * D : S + ((int64_t)it.fr * d.H + it.h) * D * D;
+      // this thread's accumulator row is key feature ii of head ph of the group
+      const int dh = d.D, ph = i_row / dh, ii = i_row % dh, hh = it.h * (D / dh) + ph;
+      float *So = (it.text ? St + (int64_t)hh * dh * dh : S + ((int64_t)it.fr * d.H + hh) * dh * dh) + (int64_t)ii * dh;
       if (it.nch > 0) {
         const int b = na & 1;
         const bool done = ok && mbar_wait(smem_u32(&bars->acc_full[b]), (na >> 1) & 1, abort_flag, st, K_STATE_TC, 7);
@@ -275,19 +281,27 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty[b]));
-          float4 *dst = reinterpret_cast<float4 *>(So + i_row * D + c_lo);
+          // the 32-column chunks c_lo and c_lo + 32 that belong to head ph (the diagonal block)
+          if (c_lo / dh == ph) {
+            float4 *dst = reinterpret_cast<float4 *>(So + (c_lo - ph * dh));
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(__uint_as_float(u0[4 * v]), __uint_as_float(u0[4 * v + 1]),
-                                 __uint_as_float(u0[4 * v + 2]), __uint_as_float(u0[4 * v + 3]));
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(u0[4 * v]), __uint_as_float(u0[4 * v + 1]),
+                                   __uint_as_float(u0[4 * v + 2]), __uint_as_float(u0[4 * v + 3]));
+          }
+          if ((c_lo + 32) / dh == ph) {
+            float4 *dst = reinterpret_cast<float4 *>(So + (c_lo + 32 - ph * dh));
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[8 + v] = make_float4(__uint_as_float(u1[4 * v]), __uint_as_float(u1[4 * v + 1]),
-                                     __uint_as_float(u1[4 * v + 2]), __uint_as_float(u1[4 * v + 3]));
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(u1[4 * v]), __uint_as_float(u1[4 * v + 1]),
+                                   __uint_as_float(u1[4 * v + 2]), __uint_as_float(u1[4 * v + 3]));
+          }
         }
         ++na;
       } else {
-        for (int cc = 0; cc < D / 2; ++cc) So[i_row * D + c_lo + cc] = 0.f;
+        // no tokens (an empty text): the head's block is zero
+        for (int cc = 0; cc < D / 2; ++cc)
+          if ((c_lo + cc) / dh == ph) So[c_lo + cc - ph * dh] = 0.f;
       }
       // every phi warp has written its share of z; their states are ANDed, so that all eight
       // leave the item loop together and their named barriers always pair up
@@ -297,7 +311,8 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
         float zs = 0.f;
 #pragma unroll
         for (int pw = 0; pw < PHI_WARPS; ++pw) zs += bars->zpart[pw][tid];
-        zo[(it.text ? (int64_t)it.h * D : ((int64_t)it.fr * d.H + it.h) * D) + tid] = zs;
+        // the group's 128 features are its heads' z vectors back to back
+        zo[(it.text ? (int64_t)it.h * D : (int64_t)it.fr * d.H * d.D + (int64_t)it.h * D) + tid] = zs;
       }
       if (!ok) break;
     }
@@ -309,27 +324,39 @@ __global__ void __launch_bounds__(sb::THREADS, 2)
 }
 
 // ============================================================================ read staging
-__global__ void __launch_bounds__(256) read_stage_kernel(int64_t n_s8, int64_t n_z, int64_t n_w8,
+// Destination of the 8 consecutive entries starting at (row i, column j) of head h's D x D
+// block in the block-diagonal bf16 layout [..][H / P][128][128] (P = 128 / D heads per head
+// group); `lead` selects the leading index (group g for S_sum, nothing for W_l).  With
+// D = 128 this is the plain [..][H][D][D] index.
+__device__ __forceinline__ int64_t bdiag_index(int64_t lead, int H, int D, int h, int i, int j) {
+  const int P = 128 / D, hg = h / P, pp = h % P;
+  return ((lead * (H / P) + hg) * 128 + pp * D + i) * 128 + pp * D + j;
+}
+
+__global__ void __launch_bounds__(256) read_stage_kernel(int64_t n_s8, int64_t n_z, int64_t n_w8, int H, int D,
                                                          const float *__restrict__ Sf, const float *__restrict__ Sb,
                                                          const float *__restrict__ zf, const float *__restrict__ zb,
                                                          const float *__restrict__ wgl, __nv_bfloat16 *__restrict__ ssum,
                                                          float *__restrict__ zsum, __nv_bfloat16 *__restrict__ wl) {
   const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  const int64_t DD = (int64_t)D * D;
   if (i < n_s8) {
     const float4 *a = reinterpret_cast<const float4 *>(Sf + 8 * i), *b = reinterpret_cast<const float4 *>(Sb + 8 * i);
     const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
     const float f[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
                         a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
-    *reinterpret_cast<uint4 *>(ssum + 8 * i) = pack8(f);
+    const int64_t e = 8 * i, gh = e / DD, rem = e % DD;
+    *reinterpret_cast<uint4 *>(ssum + bdiag_index(gh / H, H, D, (int)(gh % H), (int)(rem / D), (int)(rem % D))) =
+        pack8(f);
   } else if (i < n_s8 + n_z) {
     const int64_t j = i - n_s8;
     zsum[j] = zf[j] + zb[j];
   } else if (i < n_s8 + n_z + n_w8) {
-    const int64_t j = i - n_s8 - n_z;
-    const float4 *a = reinterpret_cast<const float4 *>(wgl + 8 * j);
+    const int64_t e = 8 * (i - n_s8 - n_z), h = e / DD, rem = e % DD;
+    const float4 *a = reinterpret_cast<const float4 *>(wgl + e);
     const float4 a0 = a[0], a1 = a[1];
     const float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-    *reinterpret_cast<uint4 *>(wl + 8 * j) = pack8(f);
+    *reinterpret_cast<uint4 *>(wl + bdiag_index(0, H, D, (int)h, (int)(rem / D), (int)(rem % D))) = pack8(f);
   }
 }
 
@@ -374,8 +401,11 @@ struct alignas(16) Bars {
   // with S_sum (one fill per group and head): the normaliser z and the scalar-gate weights
   float zs[D], wg1[D];
   float gam[D];                 // gamma of the epilogue's current head (staged by the epilogue)
-  float den[2][2][BM], g1[2][2][BM];  // per accumulator set and column half: normaliser and scalar-gate logit
-  float ssq[2][BM];                   // the epilogue's sums of squares per column half
+  // per accumulator set and 32-column block of the row: shares of the normaliser (delta
+  // rule: of |q|^2) and of the scalar-gate logit; the epilogue's sums of squares.  A head
+  // of D features takes D / 32 consecutive blocks.
+  float den[2][4][BM], g1[2][4][BM];
+  float ssq[4][BM];
   uint64_t q_full[NQ], q_empty[NQ], gate_done[NQ], feat_full[NQ], den_full[2], acc_full[2], acc_empty[2];
   uint64_t s_full, s_empty, w_full, w_empty, drain;
   uint32_t tmem;
@@ -428,8 +458,10 @@ __device__ __forceinline__ bool read_item(const int32_t *__restrict__ tiles, int
 
 // DELTA: q/|q| features and no normaliser; FUSED: RMSNorm and the linear gate (GATE_MMA:
 // element-wise, G_l = D, on the tensor cores; otherwise the scalar gate, G_l = 1); AMAX:
-// also the per-head max |q| into amax_q (for the e4m3 quantisation that follows)
-template <bool DELTA, bool FUSED, bool GATE_MMA, bool AMAX>
+// also the per-head max |q| into amax_q (for the e4m3 quantisation that follows); NB: the
+// 32-column blocks of one head (D / 32: 4 for D = 128, whose halves of a row belong to one
+// head; 2 or 1 for the 128 / D heads of a head group of D = 64 or 32)
+template <bool DELTA, bool FUSED, bool GATE_MMA, bool AMAX, int NB>
 __global__ void __launch_bounds__(rd::THREADS, 1)
     read_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                    const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmO, Dims d,
@@ -441,6 +473,7 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
   using namespace rd;
   constexpr bool delta = DELTA, fused = FUSED, gate_mma = FUSED && GATE_MMA, scalar_gate = FUSED && !GATE_MMA;
   constexpr bool amax = AMAX;
+  static_assert(NB == 4 || NB == 2 || NB == 1, "32-column blocks per head");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   Bars *bars = reinterpret_cast<Bars *>(base + BAR_OFF);
@@ -455,7 +488,8 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
   const int64_t x1 = x0 + per < n_items ? x0 + per : n_items;
   if (x0 >= x1) return;  // block-uniform
   // range-check build: the last head's columns lie inside an output row (block-uniform)
-  if (!in_range(st, (int64_t)d.H * D - 1, out_stride, K_READ_TC, 5)) return;
+  if (!in_range(st, (int64_t)d.H * d.D - 1, out_stride, K_READ_TC, 5)) return;
+  const int Hg = d.H * d.D / D;  // head groups of 128 features (one head when D = 128)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NQ; ++s) {
@@ -513,7 +547,7 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
           ++nw;
           cur_w = it.h;
         }
-        const int key = it.g * d.H + it.h;
+        const int key = it.g * Hg + it.h;
         if (key != cur_s) {
           if (!mbar_wait(smem_u32(&bars->s_empty), (ns & 1) ^ 1, abort_flag, st, K_READ, 3)) break;
           const uint32_t sb = smem_u32(&bars->s_full);
@@ -543,7 +577,7 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
         ReadItem it;
         if (!read_item(tiles, n_tiles, d, st, x, it)) continue;
         const int s = k % NQ, a = k & 1;
-        const int key = it.g * d.H + it.h;
+        const int key = it.g * Hg + it.h;
         const bool new_w = gate_mma && it.h != cur_w, new_s = key != cur_s;
         // releases first: every MMA on the previous W_l / S_sum has been issued
         if (new_w && nw > 0) mma_commit(smem_u32(&bars->w_empty));
@@ -607,7 +641,7 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
       const int s = k % NQ, a = k & 1;
       // z (and the scalar-gate weights) of a new group come with its S_sum; the slot is
       // refilled only after the last item of the previous group has been handed over
-      const int key = it.g * d.H + it.h;
+      const int key = it.g * Hg + it.h;
       if (key != cur_s && (!delta || scalar_gate)) {
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full), ns & 1, abort_flag, st, K_READ, 15))) break;
         ++ns;
@@ -627,29 +661,31 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
       // (Each half reads only its own columns of the tile: the other half's thread may
       // already be writing its features over the rest.)
       uint32_t fr[HC / 2];
-      float2 den2 = make_float2(0.f, 0.f);
-      float gate1 = 0.f;
+      float2 den2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // per 32-column block
+      float gate1[2] = {0.f, 0.f};
       const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
 #pragma unroll
       for (int i = 0; i < HC / 8; ++i) {
-        const int cl = c0 / 8 + i;
+        const int cl = c0 / 8 + i, bk = i >> 2;  // 16-byte chunk, and its block in this half
         const uint4 raw = *reinterpret_cast<const uint4 *>(qt + swz_off(r, cl, BM));
         const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float2 xv = __bfloat1622float2(hp[e]);
           if (amax) qmax = fmaxf(qmax, fmaxf(fabsf(xv.x), fabsf(xv.y)));
+          // D = 128: one share per half row; otherwise one per 32-column block
+          const int ab = NB == 4 ? 0 : bk;
           if (scalar_gate) {
             const float2 wv = *reinterpret_cast<const float2 *>(&bars->wg1[cl * 8 + 2 * e]);
-            gate1 = fmaf(xv.x, wv.x, fmaf(xv.y, wv.y, gate1));
+            gate1[ab] = fmaf(xv.x, wv.x, fmaf(xv.y, wv.y, gate1[ab]));
           }
           if (delta) {
-            den2 = __ffma2_rn(xv, xv, den2);
+            den2[ab] = __ffma2_rn(xv, xv, den2[ab]);
           } else {
             // elu + 1 as max(x, 0) + 2^(min(x, 0) log2 e): no branch
             const float2 e2 = __fmul2_rn(make_float2(fminf(xv.x, 0.f), fminf(xv.y, 0.f)), l2e);
             xv = __fadd2_rn(make_float2(fmaxf(xv.x, 0.f), fmaxf(xv.y, 0.f)), make_float2(ex2f(e2.x), ex2f(e2.y)));
-            den2 = __ffma2_rn(xv, *reinterpret_cast<const float2 *>(&bars->zs[cl * 8 + 2 * e]), den2);
+            den2[ab] = __ffma2_rn(xv, *reinterpret_cast<const float2 *>(&bars->zs[cl * 8 + 2 * e]), den2[ab]);
             fr[i * 4 + e] = pack_bf16(xv.x, xv.y);
           }
         }
@@ -666,8 +702,16 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
           *reinterpret_cast<uint4 *>(qt + swz_off(r, c0 / 8 + i, BM)) =
               make_uint4(fr[i * 4], fr[i * 4 + 1], fr[i * 4 + 2], fr[i * 4 + 3]);
       }
-      bars->den[a][hf][r] = den2.x + den2.y;
-      bars->g1[a][hf][r] = gate1;
+      if constexpr (NB == 4) {
+        bars->den[a][hf][r] = den2[0].x + den2[0].y;
+        bars->g1[a][hf][r] = gate1[0];
+      } else {
+#pragma unroll
+        for (int bk = 0; bk < 2; ++bk) {
+          bars->den[a][2 * hf + bk][r] = den2[bk].x + den2[bk].y;
+          bars->g1[a][2 * hf + bk][r] = gate1[bk];
+        }
+      }
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->feat_full[s]));
@@ -728,34 +772,62 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
       // the previous item's stores have finished reading once all of them are here
       if (!named_bar_and(1, NT, got)) break;
       tc_fence_after();
+      // The row's two 32-column chunks (blocks 2hf and 2hf + 1) and the heads they belong
+      // to: D = 128, the row's one head over both halves; otherwise the NB blocks of each head.
+      auto head_sum = [&](const float (*arr)[BM], int b) {
+        const int b0 = (b / NB) * NB;
+        float t = 0.f;
+#pragma unroll
+        for (int j = 0; j < NB; ++j) t += arr[b0 + j][r];
+        return t;
+      };
       // ELU1: the normaliser phi(q).z; delta rule: |q|^2 (o = (q . S) / |q|)
-      const float den = bars->den[a][0][r] + bars->den[a][1][r];
-      const float gate1 = bars->g1[a][0][r] + bars->g1[a][1][r];
-      const float scale = delta ? (den > 0.f ? rsqrtf(den) : 0.f) : (den > 0.f ? 1.f / den : 0.f);
+      float scale[2], gs[2];
+      if constexpr (NB == 4) {
+        const float den = bars->den[a][0][r] + bars->den[a][1][r];
+        scale[0] = scale[1] = delta ? (den > 0.f ? rsqrtf(den) : 0.f) : (den > 0.f ? 1.f / den : 0.f);
+        gs[0] = gs[1] = fast_sigmoid(bars->g1[a][0][r] + bars->g1[a][1][r]);
+      } else {
+#pragma unroll
+        for (int bk = 0; bk < 2; ++bk) {
+          const float den = head_sum(bars->den[a], 2 * hf + bk);
+          scale[bk] = delta ? (den > 0.f ? rsqrtf(den) : 0.f) : (den > 0.f ? 1.f / den : 0.f);
+          gs[bk] = fast_sigmoid(head_sum(bars->g1[a], 2 * hf + bk));
+        }
+      }
       const uint32_t acc = tmem + lane_off + (uint32_t)a * 256 + (uint32_t)c0;
-      float rinv = 1.f;
+      float rinv[2] = {1.f, 1.f};
       if (fused) {
         uint32_t u0[32], u1[32];
         tmem_ld32(acc, u0);
         tmem_ld32(acc + 32, u1);
         tmem_wait_ld();
-        float2 ss2 = make_float2(0.f, 0.f);
+        float2 ss2 = make_float2(0.f, 0.f);  // .x: block 2hf, .y: block 2hf + 1
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float2 ab = make_float2(__uint_as_float(u0[i]), __uint_as_float(u1[i]));
           ss2 = __ffma2_rn(ab, ab, ss2);
         }
-        bars->ssq[hf][r] = ss2.x + ss2.y;
-        named_bar_sync(1, NT);  // both halves' sums of squares are in
-        rinv = rsqrtf((bars->ssq[0][r] + bars->ssq[1][r]) * (scale * scale) / (float)D + eps);
+        if constexpr (NB == 4) {
+          bars->ssq[hf][r] = ss2.x + ss2.y;
+          named_bar_sync(1, NT);  // both halves' sums of squares are in
+          rinv[0] = rinv[1] = rsqrtf((bars->ssq[0][r] + bars->ssq[1][r]) * (scale[0] * scale[0]) / (float)D + eps);
+        } else {
+          bars->ssq[2 * hf][r] = ss2.x;
+          bars->ssq[2 * hf + 1][r] = ss2.y;
+          named_bar_sync(1, NT);  // every block's sum of squares is in
+#pragma unroll
+          for (int bk = 0; bk < 2; ++bk)
+            rinv[bk] = rsqrtf(head_sum(bars->ssq, 2 * hf + bk) * (scale[bk] * scale[bk]) / (float)(32 * NB) + eps);
+        }
       }
-      const float f_row = scale * rinv;  // o / rms(o) = num * scale * rinv
-      const float f_out = out8 ? f_row / a8_scale[it.h] : f_row;
-      const float gs = fast_sigmoid(gate1);
       // this thread's 64 columns: bf16, box hf, chunks 0-7 of row r; e4m3, chunks 4hf .. 4hf+3
       uint8_t *srow = stage + (out8 ? 0 : hf * (BM * 128)) + r * 128;
 #pragma unroll
       for (int c = 0; c < HC; c += 32) {
+        const int bk = c >> 5;
+        const float f_row = scale[bk] * rinv[bk];  // o / rms(o) = num * scale * rinv
+        const float f_out = out8 ? f_row / a8_scale[it.h] : f_row;
         uint32_t u[32], ug[32];
         tmem_ld32(acc + c, u);
         if (gate_mma) tmem_ld32(acc + 128 + c, ug);
@@ -772,7 +844,7 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
               if (gate_mma) {
                 gl = make_float2(__uint_as_float(ug[v + e]), __uint_as_float(ug[v + e + 1]));  // sigmoid, in place
               } else {
-                gl = make_float2(gs, gs);
+                gl = make_float2(gs[bk], gs[bk]);
               }
               const float2 o = __fmul2_rn(__fmul2_rn(gl, gg[e >> 1]),
                                           __fmul2_rn(make_float2(__uint_as_float(u[v + e]), __uint_as_float(u[v + e + 1])), fo));
@@ -847,13 +919,16 @@ __global__ void __launch_bounds__(rd::THREADS, 1)
 
 }  // namespace
 
-bool linear_tc_supported(const Dims &d, vdn_dtype dt) { return dt == VDN_BF16 && d.D == 128; }
+// bf16 with D = 128, or D = 64 or 32 whose heads fill whole 128-feature groups
+bool linear_tc_supported(const Dims &d, vdn_dtype dt) {
+  return dt == VDN_BF16 && (d.D == 128 || ((d.D == 64 || d.D == 32) && (d.H * d.D) % 128 == 0));
+}
 
 cudaError_t launch_state_build_tc(const Dims &d, const void *k, const void *v, const void *kt, const void *vt,
                                   float *S, float *z, float *St, float *zt, char *ws, const WsPlan &p,
                                   cudaStream_t st) {
   using namespace sb;
-  const uint64_t HD = (uint64_t)d.H * D;
+  const uint64_t HD = (uint64_t)d.H * d.D;
   CUtensorMap mk, mv, mkt, mvt;
   uint64_t strides[1] = {HD * 2};
   uint32_t box[2] = {64, TK};
@@ -867,7 +942,7 @@ cudaError_t launch_state_build_tc(const Dims &d, const void *k, const void *v, c
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(state_build_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
   if (e != cudaSuccess) return e;
-  const int n_items = (d.F + 1) * d.H;
+  const int n_items = (d.F + 1) * (int)(HD / D);  // (frames + text) x head groups
   const int grid = n_items < 2 * sm_count() ? n_items : 2 * sm_count();  // persistent: two CTAs per SM
   state_build_tc_kernel<<<(unsigned)grid, THREADS, SMEM, st>>>(mk, mv, mkt, mvt, d, S, z, St, zt,
                                                                (DevStatus *)(ws + p.status));
@@ -883,8 +958,16 @@ cudaError_t launch_read_stage(const Dims &d, vdn_lin_kind kind, const float *Sf,
   const int64_t n_w8 = (wgl != nullptr && G_l == d.D) ? (int64_t)d.H * DD / 8 : 0;
   const int64_t n = n_s8 + n_z + n_w8;
   if (n == 0) return cudaSuccess;
+  if (d.D < 128) {
+    // the off-diagonal blocks of the head groups' 128 x 128 operands are zero
+    const size_t hd128 = (size_t)d.H * d.D * 128 * 2;
+    cudaError_t e = cudaSuccess;
+    if (n_s8 > 0) e = cudaMemsetAsync(ws + p.ssum, 0, (size_t)G * hd128, st);
+    if (e == cudaSuccess && n_w8 > 0) e = cudaMemsetAsync(ws + p.wl, 0, hd128, st);
+    if (e != cudaSuccess) return e;
+  }
   read_stage_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-      n_s8, n_z, n_w8, Sf, Sb, zf, zb, wgl, (__nv_bfloat16 *)(ws + p.ssum), (float *)(ws + p.zsum),
+      n_s8, n_z, n_w8, d.H, d.D, Sf, Sb, zf, zb, wgl, (__nv_bfloat16 *)(ws + p.ssum), (float *)(ws + p.zsum),
       (__nv_bfloat16 *)(ws + p.wl));
   return cudaGetLastError();
 }
@@ -893,7 +976,7 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
                            const float *gamma, float eps, char *ws, const WsPlan &p, cudaStream_t st,
                            const float *a8_scale, uint32_t *amax_q) {
   using namespace rd;
-  const uint64_t HD = (uint64_t)d.H * D;
+  const uint64_t HD = (uint64_t)d.H * d.D;
   const int G = host_group_count(d);
   const bool fused = wgl != nullptr;
   const bool gate_mma = fused && G_l == D;
@@ -906,12 +989,13 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
       return cudaErrorInvalidValue;
   }
   {
-    uint64_t dims[2] = {(uint64_t)D, (uint64_t)G * d.H * D}, strides[1] = {(uint64_t)D * 2};
+    // block-diagonal S_sum [G][head groups][128][128] and W_l [head groups][128][128]
+    uint64_t dims[2] = {(uint64_t)D, (uint64_t)G * HD}, strides[1] = {(uint64_t)D * 2};
     uint32_t box[2] = {64, (uint32_t)D};
     if (!encode_tmap(&ms, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.ssum, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
-    uint64_t dimsw[2] = {(uint64_t)D, (uint64_t)d.H * D};
+    uint64_t dimsw[2] = {(uint64_t)D, HD};
     if (!encode_tmap(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.wl, dimsw, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
@@ -929,7 +1013,7 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
       return cudaErrorInvalidValue;
   }
   const int n_tiles = host_tile_count(d);
-  const int64_t n_items = (int64_t)2 * n_tiles * d.H;
+  const int64_t n_items = (int64_t)2 * n_tiles * (int64_t)(HD / D);  // tile halves x head groups
   const int grid = (int)(n_items < sm_count() ? n_items : sm_count());  // persistent: one CTA per SM
   const float *zs = (const float *)(ws + p.zsum);
   const int32_t *tl = (const int32_t *)(ws + p.tiles);
@@ -942,16 +1026,23 @@ cudaError_t launch_read_tc(const Dims &d, vdn_lin_kind kind, const void *q, void
                                       n_tiles, n_items, a8_scale, amax_q, sp);
     return cudaGetLastError();
   };
+  if (d.D < 128) {
+    // heads of D = 64 or 32 in 128-feature head groups: the plain read (the layer applies the
+    // gates and RMSNorm in its own pass at these sizes)
+    if (fused || amax_q != nullptr) return cudaErrorInvalidValue;
+    if (d.D == 64) return delta ? go(read_tc_kernel<true, false, false, false, 2>) : go(read_tc_kernel<false, false, false, false, 2>);
+    return delta ? go(read_tc_kernel<true, false, false, false, 1>) : go(read_tc_kernel<false, false, false, false, 1>);
+  }
   if (amax_q != nullptr) {  // the max |q| by-product: the delta rule's gated layer only
     if (!(delta && gate_mma)) return cudaErrorInvalidValue;
-    return go(read_tc_kernel<true, true, true, true>);
+    return go(read_tc_kernel<true, true, true, true, 4>);
   }
   if (delta) {
-    if (!fused) return go(read_tc_kernel<true, false, false, false>);
-    return gate_mma ? go(read_tc_kernel<true, true, true, false>) : go(read_tc_kernel<true, true, false, false>);
+    if (!fused) return go(read_tc_kernel<true, false, false, false, 4>);
+    return gate_mma ? go(read_tc_kernel<true, true, true, false, 4>) : go(read_tc_kernel<true, true, false, false, 4>);
   }
-  if (!fused) return go(read_tc_kernel<false, false, false, false>);
-  return gate_mma ? go(read_tc_kernel<false, true, true, false>) : go(read_tc_kernel<false, true, false, false>);
+  if (!fused) return go(read_tc_kernel<false, false, false, false, 4>);
+  return gate_mma ? go(read_tc_kernel<false, true, true, false, 4>) : go(read_tc_kernel<false, true, false, false, 4>);
 }
 
 }  // namespace vdn

@@ -502,7 +502,14 @@ vdn_status layer_impl(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype
       ProfScope ps(K_SCAN, st);
       VDN_CUDA(launch_state_scan(d, kind, S, z, St, zt, beta, Sf, Sb, zf, zb, w, p, st), "scan launch");
     }
-    {
+    if (linear_tc_supported(d, act)) {
+      {
+        ProfScope ps(K_READ_STAGE, st);
+        VDN_CUDA(launch_read_stage(d, kind, Sf, Sb, zf, zb, nullptr, 0, w, p, st), "read staging");
+      }
+      ProfScope ps(K_READ_TC, st);
+      VDN_CUDA(launch_read_tc(d, kind, q, Ol, nullptr, 0, nullptr, 0.f, w, p, st), "read launch");
+    } else {
       ProfScope ps(K_READ, st);
       VDN_CUDA(launch_linear_read(d, kind, act, q, Sf, Sb, zf, zb, Ol, w, p, st), "read launch");
     }

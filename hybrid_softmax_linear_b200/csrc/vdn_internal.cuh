@@ -206,9 +206,12 @@ inline WsPlan plan_workspace(const vdn_shape &s, vdn_lin_kind kind, vdn_dtype dt
   p.splan = take((size_t)splan_ints(s.frames, (int)G) * 4);
   p.tscr = take((4 * G + 2 * (F + 1)) * 4);  // keys, order, count, first; mark, idx
   p.step_end = off;
-  p.ssum = take(G * H * D * D * 2);
+  // bf16 operands of the tensor-core read: per (group, 128-feature head group) a 128 x 128
+  // block-diagonal S_sum and W_l (one block per head: 128 / D heads per head group), so
+  // G * H * D * 128 entries (G * H * D * D when D = 128)
+  p.ssum = take(G * H * D * 128 * 2);
   p.zsum = take(G * H * D * 4);
-  p.wl = take(H * D * D * 2);
+  p.wl = take(H * D * 128 * 2);
   p.stage_end = off;
   size_t act = (dtype == VDN_F32) ? 4 : 2;
   // per-frame states: ELU1 S [F][H][D][D]; DELTA kbar [F][H][D] in S, vbar in z

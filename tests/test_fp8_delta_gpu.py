@@ -163,7 +163,8 @@ def test_config5_full_size_fp8_delta_sampled():
 
 @pytest.mark.parametrize("shape", [(1, 70, 5, 3, 2, 128),    # one frame (both anchors)
                                    (2, 40, 5, 0, 1, 128),    # two anchors, no text
-                                   (87, 20, 5, 8, 2, 128)])  # ragged last chunk
+                                   (87, 20, 5, 8, 2, 128),   # ragged last chunk
+                                   (17, 50, 3, 6, 2, 64)])   # D = 64: two heads per tensor-core head group
 def test_delta_layer_edge_shapes(shape):
     s = synth.Shape(*shape)
     inp = synth.make_inputs(s, "bf16", seed=31 + shape[0], with_beta=True)
