@@ -69,6 +69,9 @@ _SIGS = {
                                              _sz, _vp]),
     "vdn_linear_read": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                        _vp]),
+    "vdn_linear_branch_bwd_workspace_size": (_sz, [_SP]),
+    "vdn_linear_branch_bwd": (ctypes.c_int, [_SP, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                             _vp, _vp, _vp, _vp, _sz, _vp]),
     "vdn_hybrid_fuse": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _f32, _vp, _vp]),
     "vdn_out_proj": (ctypes.c_int, [_SP, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "vdn_out_proj_e4m3_workspace_size": (_sz, [_SP]),
@@ -204,6 +207,18 @@ def linear_state_scan(shape, kind, S, z, S_txt, z_txt, beta, S_fwd, S_bwd, z_fwd
 def linear_read(shape, kind, dtype, q, S_fwd, S_bwd, z_fwd, z_bwd, o_l, ws, stream=None):
     _check(lib().vdn_linear_read(ctypes.byref(Shape.of(shape)), kind, dtype, _p(q), _p(S_fwd), _p(S_bwd),
                                  _p(z_fwd), _p(z_bwd), _p(o_l), _p(ws), _nbytes(ws), _stream(stream)))
+
+
+def linear_branch_bwd_workspace_size(shape) -> int:
+    return lib().vdn_linear_branch_bwd_workspace_size(ctypes.byref(Shape.of(shape)))
+
+
+def linear_branch_bwd(shape, kind, dtype, q, k, v, kt, vt, do_l, dq, dk, dv, dkt, dvt, ws, stream=None):
+    """Gradients of sum(o_l * do_l) of the elu+1 linear branch with respect to q, k, v, kt, vt
+    (fp32 outputs; see vdn_linear_branch_bwd in include/vdn.h)."""
+    _check(lib().vdn_linear_branch_bwd(ctypes.byref(Shape.of(shape)), kind, dtype, _p(q), _p(k), _p(v), _p(kt),
+                                       _p(vt), _p(do_l), _p(dq), _p(dk), _p(dv), _p(dkt), _p(dvt), _p(ws),
+                                       _nbytes(ws), _stream(stream)))
 
 
 def hybrid_fuse(shape, dtype, q, o_s, o_l, w_gate_s, w_gate_l, G_l, gamma, eps, a, stream=None):

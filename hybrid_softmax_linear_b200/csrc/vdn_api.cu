@@ -197,6 +197,37 @@ vdn_status device_check() { return check_device(); }
 float softmax_scale_log2(float sm_scale, int D) { return scale_log2_of(sm_scale, D); }
 }  // namespace vdn
 
+namespace vdn {
+// workspace of the linear branch's backward: the step tables, then the per-frame states,
+// the groups' memories, and the per-row and per-group scratch
+struct LinBwdPlan {
+  WsPlan p;
+  size_t dnum, dden, dN, dZ, total;
+};
+LinBwdPlan plan_lin_bwd(const vdn_shape &s) {
+  LinBwdPlan b;
+  b.p = plan_workspace(s, VDN_LIN_ELU1, VDN_F32);
+  const size_t F = s.frames, H = s.heads, D = s.head_dim, Nv = (size_t)s.frames * s.tokens_per_frame;
+  const size_t G = (size_t)max_groups(s.frames, s.chunk_frames);
+  size_t off = b.p.step_end;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+  b.p.S = take(F * H * D * D * 4);
+  b.p.z = take(F * H * D * 4);
+  b.p.St = take(H * D * D * 4);
+  b.p.zt = take(H * D * 4);
+  b.p.Sf = take(G * H * D * D * 4);
+  b.p.Sb = take(G * H * D * D * 4);
+  b.p.zf = take(G * H * D * 4);
+  b.p.zb = take(G * H * D * 4);
+  b.dnum = take(Nv * H * D * 4);
+  b.dden = take(Nv * H * 4);
+  b.dN = take(G * H * D * D * 4);
+  b.dZ = take(G * H * D * 4);
+  b.total = off;
+  return b;
+}
+}  // namespace vdn
+
 extern "C" {
 
 int vdn_version(void) { return 100; }
@@ -341,6 +372,43 @@ vdn_status vdn_linear_read(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype 
     VDN_CUDA(launch_linear_read(d, kind, dtype, q, S_fwd, S_bwd, z_fwd, z_bwd, o_l, (char *)ws, p, st),
              "read launch");
   }
+  return ok();
+}
+
+size_t vdn_linear_branch_bwd_workspace_size(const vdn_shape *shape) {
+  if (check_shape(shape) != VDN_OK) return 0;
+  return plan_lin_bwd(*shape).total;
+}
+
+vdn_status vdn_linear_branch_bwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *q,
+                                 const void *k, const void *v, const void *kt, const void *vt, const float *do_l,
+                                 float *dq, float *dk, float *dv, float *dkt, float *dvt, void *ws, size_t ws_bytes,
+                                 vdn_stream stream) {
+  VDN_TRY(check_shape(shape));
+  VDN_TRY(check_kind(kind));
+  if (kind != VDN_LIN_ELU1) return fail(VDN_ERR_UNSUPPORTED, "the linear branch's backward is built for ELU1 only");
+  if (dtype != VDN_BF16) return fail(VDN_ERR_UNSUPPORTED, "the linear branch's backward takes bf16 inputs");
+  VDN_TRY(need(q, "q")); VDN_TRY(need(k, "k")); VDN_TRY(need(v, "v")); VDN_TRY(need(do_l, "do_l"));
+  VDN_TRY(need(dq, "dq")); VDN_TRY(need(dk, "dk")); VDN_TRY(need(dv, "dv"));
+  if (shape->text_tokens > 0) {
+    VDN_TRY(need(kt, "kt")); VDN_TRY(need(vt, "vt")); VDN_TRY(need(dkt, "dkt")); VDN_TRY(need(dvt, "dvt"));
+  }
+  const LinBwdPlan b = plan_lin_bwd(*shape);
+  VDN_TRY(check_ws(ws, ws_bytes, b.total));
+  VDN_TRY(check_device());
+  const Dims d = dims_of(*shape);
+  cudaStream_t st = (cudaStream_t)stream;
+  char *w = (char *)ws;
+  const WsPlan &p = b.p;
+  VDN_CUDA(launch_tables(d, w, p, st), "tables launch");
+  float *S = (float *)(w + p.S), *z = (float *)(w + p.z), *St = (float *)(w + p.St), *zt = (float *)(w + p.zt);
+  float *Sf = (float *)(w + p.Sf), *Sb = (float *)(w + p.Sb), *zf = (float *)(w + p.zf), *zb = (float *)(w + p.zb);
+  VDN_CUDA(launch_state_build(d, VDN_LIN_ELU1, VDN_BF16, k, v, kt, vt, S, z, St, zt, st), "state build launch");
+  VDN_CUDA(launch_state_scan(d, VDN_LIN_ELU1, S, z, St, zt, nullptr, Sf, Sb, zf, zb, w, p, st), "scan launch");
+  VDN_CUDA(launch_linear_bwd(d, q, k, v, kt, vt, do_l, Sf, Sb, zf, zb, (const int32_t *)(w + p.gtab),
+                             host_group_count(d), (float *)(w + b.dnum), (float *)(w + b.dden), (float *)(w + b.dN),
+                             (float *)(w + b.dZ), dq, dk, dv, dkt, dvt, st),
+           "linear branch backward launch");
   return ok();
 }
 

@@ -388,6 +388,13 @@ cudaError_t launch_softmax_tc_gated(const Dims &d, vdn_dtype dt, const void *q, 
                                     const void *kt, const void *vt, const float *scales, const float *w_gate_s,
                                     float sl2, void *a, char *ws, const WsPlan &p, cudaStream_t st, bool a8 = false);
 // per-head e4m3 quantisation of q, k (+ text), v (+ text); scales float[3][H]
+// backward of the elu+1 linear branch (CUDA cores, fp32): Sf..zb the groups' memories,
+// gtab the group table (G groups); dnum [N_v][H][D], dden [N_v][H], dN [G][H][D][D],
+// dZ [G][H][D] scratch
+cudaError_t launch_linear_bwd(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
+                              const void *vt, const float *dO, const float *Sf, const float *Sb, const float *zf,
+                              const float *zb, const int32_t *gtab, int G, float *dnum, float *dden, float *dN,
+                              float *dZ, float *dq, float *dk, float *dv, float *dkt, float *dvt, cudaStream_t st);
 cudaError_t launch_fp8_quant(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
                              const void *vt, void *q8, void *k8, void *v8, void *kt8, void *vt8, float *scales,
                              uint32_t *amax_bits, cudaStream_t st);

@@ -215,6 +215,27 @@ VDN_API vdn_status vdn_linear_read(const vdn_shape *shape, vdn_lin_kind kind, vd
                            const float *S_fwd, const float *S_bwd, const float *z_fwd, const float *z_bwd,
                            void *o_l, void *ws, size_t ws_bytes, vdn_stream stream);
 
+/* vdn_linear_branch_bwd — backward of the elu+1 linear branch (gradients of
+ * sum(o_l * do_l) over every video query row), for training the linear branch ([CARD]
+ * "Training"; [ART] 分阶段适配 A1/A2 train it, with the softmax branch frozen).  Recomputes
+ * the per-frame states and the groups' memories from k, v, kt, vt, then for every query row
+ * dq = (Num dnum + Den dden) * phi'(q) with dnum = do / den, dden = -(do . o) / den (0 where
+ * the normaliser is 0), and for every key row, with dS_f the sum of the groups' dNum =
+ * sum phi(q)^T dnum over the groups whose memory holds frame f (all groups for the text):
+ * dk = (dS_f v + dz_f) * phi'(k), dv = dS_f^T phi(k).  CUDA cores, fp32; every sum in a
+ * fixed order, so a call repeats bit for bit.
+ *   kind VDN_LIN_ELU1 and dtype VDN_BF16 only (VDN_ERR_UNSUPPORTED otherwise).
+ *   q, k, v [N_v][H][D] and kt, vt [L][H][D] bf16; do_l float [N_v][H][D];
+ *   dq, dk, dv float [N_v][H][D]; dkt, dvt float [L][H][D] (NULL allowed when L = 0).
+ *   All pointers device memory, 16-byte aligned, owned by the caller.
+ * ws: vdn_linear_branch_bwd_workspace_size(shape) bytes (tables, the states and memories,
+ * and per-row and per-group scratch). */
+VDN_API size_t vdn_linear_branch_bwd_workspace_size(const vdn_shape *shape);
+VDN_API vdn_status vdn_linear_branch_bwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_dtype dtype, const void *q,
+                                         const void *k, const void *v, const void *kt, const void *vt,
+                                         const float *do_l, float *dq, float *dk, float *dv, float *dkt, float *dvt,
+                                         void *ws, size_t ws_bytes, vdn_stream stream);
+
 /* ------------------------------------------------------------------ fuse
  * vdn_hybrid_fuse — per-branch gates and RMSNorm.  [ART] 独立门控，融合两条注意力分支.
  *   g_s = sigmoid(q_h . w_gate_s[h]);  g_l = sigmoid(q_h W_l[h]) (G_l = D: element-wise,

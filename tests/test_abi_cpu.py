@@ -121,6 +121,26 @@ def test_argument_checks_precede_cuda():
         assert L.vdn_debug_unset_flag_wait(256, 1 << 20, polls, None) == 1  # the test wait stays short
 
 
+def test_linear_branch_bwd_checks():
+    """The backward of the linear branch: ELU1 and bf16 only, text pointers required when
+    L > 0, workspace size reported without a device and checked before any launch."""
+    s = vdn.Shape(12, 40, 5, 6, 2, 64)
+    L = vdn.lib()
+    need = L.vdn_linear_branch_bwd_workspace_size(ctypes.byref(s))
+    assert need > 0 and need % 256 == 0
+    assert L.vdn_linear_branch_bwd_workspace_size(ctypes.byref(vdn.Shape(0, 40, 5, 6, 2, 64))) == 0
+    args = [16] * 11
+    st = L.vdn_linear_branch_bwd(ctypes.byref(s), vdn.DELTA, vdn.BF16, *args, 256, need, None)
+    assert st == 2  # delta rule: not built
+    st = L.vdn_linear_branch_bwd(ctypes.byref(s), vdn.ELU1, vdn.F32, *args, 256, need, None)
+    assert st == 2  # f32 inputs: not built
+    st = L.vdn_linear_branch_bwd(ctypes.byref(s), vdn.ELU1, vdn.BF16, 16, 16, 16, None, 16, 16, 16, 16, 16, 16, 16,
+                                 256, need, None)
+    assert st == 1 and b"kt" in L.vdn_last_error()
+    st = L.vdn_linear_branch_bwd(ctypes.byref(s), vdn.ELU1, vdn.BF16, *args, 256, need - 256, None)
+    assert st == 3  # workspace too small
+
+
 def test_noalloc_checks_match_the_workspace_entry_point():
     """The no-allocation softmax entry point rejects exactly what vdn_softmax_branch_fwd
     rejects, before any device work, and refuses shapes whose scratch exceeds its fixed

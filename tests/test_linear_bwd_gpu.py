@@ -1,0 +1,64 @@
+"""GPU parity of the linear branch's backward (vdn_linear_branch_bwd, elu+1, bf16 inputs,
+fp32 gradients) with the float64 backward oracle (oracle/vdn_oracle_bwd.py, pinned on the
+CPU by finite differences and autograd): dq, dk, dv and the text's dkt, dvt over every row,
+for each head size, with and without text, and bit-repeatability."""
+import numpy as np
+import pytest
+import torch
+
+import hybrid_softmax_linear_b200 as vdn
+from hybrid_softmax_linear_b200 import synth
+from hybrid_softmax_linear_b200.tensors import to_device, workspace
+from oracle import vdn_oracle_bwd as vb
+from _harness import oracle_inputs, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+# fp32 sums of at most a few thousand terms against float64: a few ulp of fp32, relative
+TOL = 1e-4
+
+
+def _run(s, inp, do_l):
+    H, D, Nv, L = s.heads, s.head_dim, s.n_video, s.text_tokens
+    d = {n: to_device(a) for n, a in inp.items()}
+    dO = torch.from_numpy(do_l).cuda()
+    dq, dk, dv = (torch.full((Nv, H, D), float("nan"), device="cuda") for _ in range(3))
+    dkt, dvt = (torch.full((max(L, 1), H, D), float("nan"), device="cuda") for _ in range(2))
+    ws = workspace(vdn.linear_branch_bwd_workspace_size(s))
+    vdn.workspace_init(ws)
+    vdn.linear_branch_bwd(s, vdn.ELU1, vdn.BF16, d["q"], d["k"], d["v"], d["kt"] if L else None,
+                          d["vt"] if L else None, dO, dq, dk, dv, dkt if L else None, dvt if L else None, ws)
+    vdn.check_device_status(ws)
+    return [t.cpu().numpy() for t in (dq, dk, dv, dkt, dvt)]
+
+
+@pytest.mark.parametrize("shape", [(13, 24, 5, 8, 2, 32),     # D = 32, ragged last chunk
+                                   (12, 40, 5, 6, 2, 64),     # D = 64
+                                   (9, 33, 3, 10, 2, 128),    # D = 128, odd T
+                                   (7, 20, 3, 0, 1, 64)])     # no text
+def test_linear_branch_bwd_matches_oracle(shape):
+    assert torch.cuda.is_available(), "GPU test needs a CUDA device"
+    s = synth.Shape(*shape)
+    F, T, C, L, H, D = shape
+    inp = synth.make_inputs(s, "bf16", seed=91 + F)
+    rng = np.random.default_rng(7 + F)
+    do_l = rng.standard_normal((s.n_video, H, D)).astype(np.float32)
+    dq, dk, dv, dkt, dvt = _run(s, inp, do_l)
+    o = oracle_inputs(inp)
+    rq, rk, rv, rkt, rvt = vb.linear_branch_bwd(o["q"], o["k"], o["v"], o["kt"], o["vt"], F, T, C,
+                                                do_l.astype(np.float64))
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        assert np.all(np.isfinite(got)), name
+        assert rel_l2(got, ref) < TOL, (name, rel_l2(got, ref))
+    if L:
+        assert rel_l2(dkt[:L], rkt) < TOL and rel_l2(dvt[:L], rvt) < TOL
+
+
+def test_linear_branch_bwd_repeats_bit_for_bit():
+    s = synth.Shape(12, 40, 5, 6, 2, 64)
+    inp = synth.make_inputs(s, "bf16", seed=5)
+    do_l = np.random.default_rng(3).standard_normal((s.n_video, 2, 64)).astype(np.float32)
+    a = _run(s, inp, do_l)
+    b = _run(s, inp, do_l)
+    for x, y in zip(a, b):
+        assert np.array_equal(x.view(np.uint32), y.view(np.uint32))
