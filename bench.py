@@ -169,12 +169,16 @@ class ClockSampler:
 
     def __init__(self, cuda_index: int):
         import threading
-        self.rows, self.proc, self.thread = [], None, None
-        self.stop_ev = threading.Event()
+        self.rows, self.proc, self.thread, self.skip = [], None, None, 0
+        self.stop_ev, self.first = threading.Event(), threading.Event()
         handle = self._nvml_handle(cuda_index)
         if handle is not None:
             self.thread = threading.Thread(target=self._loop, args=(handle,), daemon=True)
             self.thread.start()
+            # the first NVML reads can take longer than a short timed region: sample once
+            # before the region starts
+            self.first.wait(2.0)
+            self.skip = len(self.rows)  # samples taken before the region, left out of the summary
             return
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(cuda_index), f"--query-gpu={self.Q}",
@@ -208,12 +212,16 @@ class ClockSampler:
                                   pynvml.nvmlDeviceGetPowerUsage(h) / 1e3))
             except Exception:
                 break
+            finally:
+                self.first.set()
             self.stop_ev.wait(0.02)
 
     def stop(self) -> dict | None:
         if self.thread is not None:
             self.stop_ev.set()
             self.thread.join(timeout=5)
+            if len(self.rows) > self.skip:
+                self.rows = self.rows[self.skip:]
             if not self.rows:
                 return None
             sm = [r[0] for r in self.rows]
@@ -474,6 +482,74 @@ def extra_layer_timing(s, kind, cdt, d, beta, G_l, steps, warmup, dev, local_ran
            "per_kernel_ms_per_step": {k: round(v[0] / max(steps, 1), 4) for k, v in prof.items()},
            "clocks": clk}
     del ws, y
+    torch.cuda.empty_cache()
+    return out
+
+
+# FP32 FMA lanes of a B200: 148 SMs x 128 lanes, two flops per FMA, at the 1965 MHz maximum
+# SM clock; the peak of kernels that run their contractions on the CUDA cores.
+FP32_CUDA_CORE_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def linear_bwd_flops(s) -> dict:
+    """Algorithmic fp32 flops of the elu+1 linear branch's backward, per stage (matrix-vector
+    products with the D x D memories; the per-row scalars are not counted)."""
+    D2, H = s.head_dim * s.head_dim, s.heads
+    return {"state_build": (s.n_video + s.text_tokens) * H * 2 * D2,    # phi(k)^T v per key row
+            "lin_bwd_rows": s.n_video * H * 4 * D2,                      # num and dphi(q) per query row
+            "lin_bwd_groups": s.n_video * H * 2 * D2,                    # phi(q)^T dnum per query row
+            "lin_bwd_keys": (s.n_video + s.text_tokens) * H * 4 * D2}    # dS v and dS^T phi(k) per key row
+
+
+def linear_bwd_timing(s, d, steps, warmup, dev, local_rank):
+    """Times the elu+1 linear branch's backward (vdn_linear_branch_bwd: state rebuild in fp32,
+    scan, per-row, per-group and per-key-frame kernels) on this run's bf16 q, k, v with a
+    seeded N(0, 1) upstream gradient; fp32 gradients out."""
+    import torch
+    import hybrid_softmax_linear_b200 as vdn
+    from hybrid_softmax_linear_b200.tensors import workspace
+    H, D, L = s.heads, s.head_dim, s.text_tokens
+    gen = torch.Generator(device=dev).manual_seed(17)
+    do_l = torch.randn((s.n_video, H, D), generator=gen, dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(do_l) for _ in range(3))
+    dkt, dvt = (torch.empty((max(L, 1), H, D), dtype=torch.float32, device=dev) for _ in range(2))
+    ws = workspace(vdn.linear_branch_bwd_workspace_size(s), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vdn.linear_branch_bwd(s, vdn.ELU1, vdn.BF16, d["q"], d["k"], d["v"], d["kt"], d["vt"], do_l, dq, dk, dv,
+                              dkt, dvt, ws, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local_rank)
+    vdn.profile_begin(16 * max(steps, 1))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    prof = vdn.profile_end()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / max(steps, 1)
+    fl = linear_bwd_flops(s)
+    kernels = {}
+    for name, (tot, n) in prof.items():
+        avg = tot / max(n, 1)
+        k = {"ms_per_launch": avg, "launches": n}
+        if name in fl and avg > 0:
+            ach = fl[name] / (avg / 1e3) / 1e12
+            k.update({"bound": "alu", "achieved": ach, "peak": FP32_CUDA_CORE_TFLOPS, "unit": "TFLOP/s",
+                      "frac": ach / FP32_CUDA_CORE_TFLOPS, "algorithmic_tflop_per_launch": fl[name] / 1e12})
+        kernels[name] = k
+    out = {"entry_point": "vdn_linear_branch_bwd", "linear": "elu1", "inputs": "this run's bf16 q, k, v, kt, vt; "
+           "do_l ~ N(0, 1) fp32 (seed 17); fp32 gradients", "ms_per_step": ms,
+           "value": s.n_video / (ms / 1e3), "unit": UNIT, "steps": steps, "warmup": warmup,
+           "tflops": sum(fl.values()) / (ms / 1e3) / 1e12,
+           "peak_note": "fp32 FMA lanes: 148 SMs x 128 x 2 flops x 1965 MHz", "kernels": kernels, "clocks": clk}
+    del ws, do_l, dq, dk, dv, dkt, dvt
     torch.cuda.empty_cache()
     return out
 
@@ -756,6 +832,7 @@ def run_ours(args, rank, world, local_rank):
         extra["e4m3_projection"] = extra_layer_timing(s, vdn.DELTA, vdn.E4M3_PROJ, d, beta.contiguous(), G_l,
                                                       args.steps, 2, dev, local_rank, peaks, ratio5)
         line["config5_extra"] = extra
+        line["linear_bwd_extra"] = linear_bwd_timing(s, d, args.steps, 2, dev, local_rank)
     line["pages_context"] = PAGES_CONTEXT
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg, inp, args.cpu_rows)
@@ -773,7 +850,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=16, help="query rows per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense-ref", action="store_true", help="skip the dense cuDNN SDPA comparator")
-    ap.add_argument("--no-extra", action="store_true", help="skip the extra e4m3 configuration timings")
+    ap.add_argument("--no-extra", action="store_true", help="skip the extra timings (the e4m3 configuration, the linear branch's backward)")
     ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
                     help="replicas: one video per GPU (weak scaling); heads: one video split by heads (strong)")
     args = ap.parse_args()

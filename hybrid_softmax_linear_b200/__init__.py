@@ -94,10 +94,10 @@ _SIGS = {
     "vdn_profile_end": (ctypes.c_int, [_vp, _vp, _i32]),
 }
 
-PROF_KERNELS = 16
+PROF_KERNELS = 19
 KERNEL_NAMES = {1: "tables", 2: "softmax_simt", 3: "softmax_tc", 4: "state_build", 5: "scan", 6: "read", 7: "fuse",
                 8: "out_proj_simt", 9: "out_proj_tc", 10: "fp8_quant", 11: "delta_stats", 13: "state_build_tc",
-                14: "read_stage", 15: "read_tc"}
+                14: "read_stage", 15: "read_tc", 16: "lin_bwd_rows", 17: "lin_bwd_groups", 18: "lin_bwd_keys"}
 
 
 def lib() -> ctypes.CDLL:
@@ -342,7 +342,7 @@ def check_device_status(ws, stream=None):
 
 
 def profile_begin(max_launches: int = 4096):
-    """Start per-kernel CUDA-event timing of vdn_hybrid_attn_fwd calls."""
+    """Start per-kernel CUDA-event timing of the entry points' launches."""
     _check(lib().vdn_profile_begin(max_launches))
 
 

@@ -203,36 +203,41 @@ __global__ void __launch_bounds__(BT) lin_bwd_keys_kernel(Dims d, const __nv_bfl
 }
 
 template <int D>
-cudaError_t lin_bwd_t(const Dims &d, const void *q, const void *k, const void *v, const void *kt, const void *vt,
-                      const float *dO, const float *Sf, const float *Sb, const float *zf, const float *zb,
-                      const int32_t *gtab, int G, float *dnum, float *dden, float *dN, float *dZ, float *dq,
-                      float *dk, float *dv, float *dkt, float *dvt, cudaStream_t st) {
+cudaError_t lin_bwd_t(const Dims &d, int stage, const void *q, const void *k, const void *v, const void *kt,
+                      const void *vt, const float *dO, const float *Sf, const float *Sb, const float *zf,
+                      const float *zb, const int32_t *gtab, int G, float *dnum, float *dden, float *dN, float *dZ,
+                      float *dq, float *dk, float *dv, float *dkt, float *dvt, cudaStream_t st) {
   constexpr int RS = BT / D;
-  const size_t smem_rows = (size_t)(2 * D * D + D + 4 * RS * D) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(lin_bwd_rows_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_rows);
-  if (e != cudaSuccess) return e;
-  lin_bwd_rows_kernel<D><<<dim3(G, d.H), BT, smem_rows, st>>>(d, (const __nv_bfloat16 *)q, dO, Sf, Sb, zf, zb, gtab, dq,
-                                                               dnum, dden);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  lin_bwd_dnum_kernel<D><<<dim3(G, d.H), BT, 0, st>>>(d, (const __nv_bfloat16 *)q, dnum, dden, gtab, dN, dZ);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t smem_keys = (size_t)(2 * D * D + D + 2 * RS * D) * sizeof(float);
-  e = cudaFuncSetAttribute(lin_bwd_keys_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_keys);
-  if (e != cudaSuccess) return e;
-  lin_bwd_keys_kernel<D><<<dim3(d.F + 1, d.H), BT, smem_keys, st>>>(
-      d, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)kt, (const __nv_bfloat16 *)vt, dN,
-      dZ, gtab, G, dk, dv, dkt, dvt);
+  cudaError_t e = cudaSuccess;
+  if (stage == 0) {
+    const size_t smem_rows = (size_t)(2 * D * D + D + 4 * RS * D) * sizeof(float);
+    e = cudaFuncSetAttribute(lin_bwd_rows_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_rows);
+    if (e != cudaSuccess) return e;
+    lin_bwd_rows_kernel<D><<<dim3(G, d.H), BT, smem_rows, st>>>(d, (const __nv_bfloat16 *)q, dO, Sf, Sb, zf, zb,
+                                                                 gtab, dq, dnum, dden);
+  } else if (stage == 1) {
+    lin_bwd_dnum_kernel<D><<<dim3(G, d.H), BT, 0, st>>>(d, (const __nv_bfloat16 *)q, dnum, dden, gtab, dN, dZ);
+  } else if (stage == 2) {
+    const size_t smem_keys = (size_t)(2 * D * D + D + 2 * RS * D) * sizeof(float);
+    e = cudaFuncSetAttribute(lin_bwd_keys_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_keys);
+    if (e != cudaSuccess) return e;
+    lin_bwd_keys_kernel<D><<<dim3(d.F + 1, d.H), BT, smem_keys, st>>>(
+        d, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)kt, (const __nv_bfloat16 *)vt,
+        dN, dZ, gtab, G, dk, dv, dkt, dvt);
+  } else {
+    return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_linear_bwd(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
+cudaError_t launch_linear_bwd(const Dims &d, int stage, const void *q, const void *k, const void *v, const void *kt,
                               const void *vt, const float *dO, const float *Sf, const float *Sb, const float *zf,
                               const float *zb, const int32_t *gtab, int G, float *dnum, float *dden, float *dN,
                               float *dZ, float *dq, float *dk, float *dv, float *dkt, float *dvt, cudaStream_t st) {
 #define VDN_LB(DD) \
-  return lin_bwd_t<DD>(d, q, k, v, kt, vt, dO, Sf, Sb, zf, zb, gtab, G, dnum, dden, dN, dZ, dq, dk, dv, dkt, dvt, st)
+  return lin_bwd_t<DD>(d, stage, q, k, v, kt, vt, dO, Sf, Sb, zf, zb, gtab, G, dnum, dden, dN, dZ, dq, dk, dv, dkt, dvt, st)
   if (d.D == 32) VDN_LB(32);
   if (d.D == 64) VDN_LB(64);
   if (d.D == 128) VDN_LB(128);

@@ -403,12 +403,22 @@ vdn_status vdn_linear_branch_bwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_
   VDN_CUDA(launch_tables(d, w, p, st), "tables launch");
   float *S = (float *)(w + p.S), *z = (float *)(w + p.z), *St = (float *)(w + p.St), *zt = (float *)(w + p.zt);
   float *Sf = (float *)(w + p.Sf), *Sb = (float *)(w + p.Sb), *zf = (float *)(w + p.zf), *zb = (float *)(w + p.zb);
-  VDN_CUDA(launch_state_build(d, VDN_LIN_ELU1, VDN_BF16, k, v, kt, vt, S, z, St, zt, st), "state build launch");
-  VDN_CUDA(launch_state_scan(d, VDN_LIN_ELU1, S, z, St, zt, nullptr, Sf, Sb, zf, zb, w, p, st), "scan launch");
-  VDN_CUDA(launch_linear_bwd(d, q, k, v, kt, vt, do_l, Sf, Sb, zf, zb, (const int32_t *)(w + p.gtab),
-                             host_group_count(d), (float *)(w + b.dnum), (float *)(w + b.dden), (float *)(w + b.dN),
-                             (float *)(w + b.dZ), dq, dk, dv, dkt, dvt, st),
-           "linear branch backward launch");
+  {
+    ProfScope ps(K_STATE, st);
+    VDN_CUDA(launch_state_build(d, VDN_LIN_ELU1, VDN_BF16, k, v, kt, vt, S, z, St, zt, st), "state build launch");
+  }
+  {
+    ProfScope ps(K_SCAN, st);
+    VDN_CUDA(launch_state_scan(d, VDN_LIN_ELU1, S, z, St, zt, nullptr, Sf, Sb, zf, zb, w, p, st), "scan launch");
+  }
+  static const int kids[3] = {K_LIN_BWD_ROWS, K_LIN_BWD_GROUPS, K_LIN_BWD_KEYS};
+  for (int stage = 0; stage < 3; ++stage) {
+    ProfScope ps(kids[stage], st);
+    VDN_CUDA(launch_linear_bwd(d, stage, q, k, v, kt, vt, do_l, Sf, Sb, zf, zb, (const int32_t *)(w + p.gtab),
+                               host_group_count(d), (float *)(w + b.dnum), (float *)(w + b.dden),
+                               (float *)(w + b.dN), (float *)(w + b.dZ), dq, dk, dv, dkt, dvt, st),
+             "linear branch backward launch");
+  }
   return ok();
 }
 

@@ -259,7 +259,8 @@ struct DevStatus {
 enum KernelId : uint32_t {
   K_TABLES = 1, K_SOFTMAX_SIMT = 2, K_SOFTMAX_TC = 3, K_STATE = 4, K_SCAN = 5, K_READ = 6,
   K_FUSE = 7, K_GEMM_SIMT = 8, K_GEMM_TC = 9, K_QUANT = 10, K_DELTA = 11, K_DEBUG_WAIT = 12,
-  K_STATE_TC = 13, K_READ_STAGE = 14, K_READ_TC = 15,
+  K_STATE_TC = 13, K_READ_STAGE = 14, K_READ_TC = 15, K_LIN_BWD_ROWS = 16, K_LIN_BWD_GROUPS = 17,
+  K_LIN_BWD_KEYS = 18,
 };
 
 __device__ __forceinline__ void report(DevStatus *st, uint32_t code, uint32_t where, uint32_t detail) {
@@ -391,7 +392,8 @@ cudaError_t launch_softmax_tc_gated(const Dims &d, vdn_dtype dt, const void *q, 
 // backward of the elu+1 linear branch (CUDA cores, fp32): Sf..zb the groups' memories,
 // gtab the group table (G groups); dnum [N_v][H][D], dden [N_v][H], dN [G][H][D][D],
 // dZ [G][H][D] scratch
-cudaError_t launch_linear_bwd(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
+// stage 0: per-row dq, dnum, dden; 1: per-group dNum, dDen; 2: per-key-frame dk, dv
+cudaError_t launch_linear_bwd(const Dims &d, int stage, const void *q, const void *k, const void *v, const void *kt,
                               const void *vt, const float *dO, const float *Sf, const float *Sb, const float *zf,
                               const float *zb, const int32_t *gtab, int G, float *dnum, float *dden, float *dN,
                               float *dZ, float *dq, float *dk, float *dv, float *dkt, float *dvt, cudaStream_t st);

@@ -359,14 +359,16 @@ VDN_API vdn_status vdn_check_device_status(void *ws, size_t ws_bytes, vdn_stream
 VDN_API vdn_status vdn_debug_unset_flag_wait(void *ws, size_t ws_bytes, uint32_t max_polls, vdn_stream stream);
 
 /* ------------------------------------------------------------------ kernel timing
- * Per-kernel device timing of vdn_hybrid_attn_fwd with CUDA events recorded on the
- * launching stream around each kernel.  vdn_profile_begin enables recording (host state
+ * Per-kernel device timing of the entry points (the layer, its steps and the linear
+ * branch's backward) with CUDA events recorded on the launching stream around each kernel.  vdn_profile_begin enables recording (host state
  * of the calling process, up to max_launches launches); vdn_profile_end waits for the
  * recorded events, writes per kernel id k < n the summed milliseconds ms[k] and launch
  * count launches[k], and disables recording.  Kernel ids: 1 tables, 2 softmax (CUDA
  * cores), 3 softmax (tensor cores), 4 state build, 5 scan, 6 read, 7 fuse, 8 projection
- * (CUDA cores), 9 projection (tensor cores), 10 fp8 quantisation, 11 delta statistics. */
-#define VDN_PROF_KERNELS 16
+ * (CUDA cores), 9 projection (tensor cores), 10 fp8 quantisation, 11 delta statistics,
+ * 13 state build (tensor cores), 14 read staging, 15 read (tensor cores), 16-18 the linear
+ * branch's backward (per-row dq, per-group dNum/dDen, per-key-frame dk/dv). */
+#define VDN_PROF_KERNELS 19
 VDN_API vdn_status vdn_profile_begin(int32_t max_launches);
 VDN_API vdn_status vdn_profile_end(float *ms, int32_t *launches, int32_t n);
 

@@ -127,3 +127,34 @@ def test_reference_arm_prints_the_contract_line_on_rank_0_only():
     assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert _bench_reference({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_clock_sampler_summarises_only_the_timed_region(monkeypatch):
+    """The sampler takes one NVML reading before the timed region starts (the first reads
+    can outlast a short region) and leaves it out of the summary; reasons decode from the
+    event-reason bits.  NVML is a fake here: nothing on a GPU is read or set."""
+    import sys
+    import time
+    import types
+    fake = types.ModuleType("pynvml")
+    fake.NVML_CLOCK_SM = 0
+    fake.nvmlInit = lambda: None
+    fake.nvmlDeviceGetHandleByUUID = lambda uuid: object()
+    clock = iter([400] + [1900] * 1000)  # an idle reading first, then clocks under load
+
+    def get_clock(h, kind):
+        time.sleep(0.03)
+        return next(clock)
+    fake.nvmlDeviceGetClockInfo = get_clock
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, kind: 1965
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x4  # sw_power_cap
+    fake.nvmlDeviceGetPowerUsage = lambda h: 700_000
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda i: types.SimpleNamespace(uuid="0"))
+    sampler = bench.ClockSampler(0)
+    assert sampler.skip >= 1
+    time.sleep(0.2)
+    got = sampler.stop()
+    assert got["source"] == "nvml" and got["samples"] >= 2
+    assert got["sm_mhz"] == 1900 and got["sm_max_mhz"] == 1965
+    assert got["reasons"] == ["sw_power_cap"] and got["power_w_max"] == 700.0
