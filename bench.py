@@ -491,17 +491,21 @@ def extra_layer_timing(s, kind, cdt, d, beta, G_l, steps, warmup, dev, local_ran
 FP32_CUDA_CORE_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def linear_bwd_flops(s) -> dict:
-    """Algorithmic fp32 flops of the elu+1 linear branch's backward, per stage (matrix-vector
-    products with the D x D memories; the per-row scalars are not counted)."""
-    D2, H = s.head_dim * s.head_dim, s.heads
-    return {"state_build": (s.n_video + s.text_tokens) * H * 2 * D2,    # phi(k)^T v per key row
-            "lin_bwd_rows": s.n_video * H * 4 * D2,                      # num and dphi(q) per query row
-            "lin_bwd_groups": s.n_video * H * 2 * D2,                    # phi(q)^T dnum per query row
-            "lin_bwd_keys": (s.n_video + s.text_tokens) * H * 4 * D2}    # dS v and dS^T phi(k) per key row
+def linear_bwd_work(s) -> dict:
+    """Algorithmic work of the elu+1 linear branch's backward per stage: fp32 flops of the
+    matrix-vector products with the D x D memories (per-row scalars not counted), or, for
+    the per-group sums, the bytes they must move."""
+    import hybrid_softmax_linear_b200 as vdn
+    D2, H, F = s.head_dim * s.head_dim, s.heads, s.frames
+    G = len(vdn.mask_layout_build(s)[1])
+    return {"state_build": ("flops", (s.n_video + s.text_tokens) * H * 2 * D2),  # phi(k)^T v per key row
+            "lin_bwd_rows": ("flops", s.n_video * H * 4 * D2),                   # num and dphi(q) per query row
+            "lin_bwd_frames": ("flops", s.n_video * H * 2 * D2),                 # phi(q)^T dnum per query row
+            "lin_bwd_keys": ("flops", (s.n_video + s.text_tokens) * H * 4 * D2),  # dS v and dS^T phi(k) per key row
+            "lin_bwd_groups": ("bytes", (F + G) * H * D2 * 4)}                   # frame sums in, group sums out
 
 
-def linear_bwd_timing(s, d, steps, warmup, dev, local_rank):
+def linear_bwd_timing(s, d, steps, warmup, dev, local_rank, peaks):
     """Times the elu+1 linear branch's backward (vdn_linear_branch_bwd: state rebuild in fp32,
     scan, per-row, per-group and per-key-frame kernels) on this run's bf16 q, k, v with a
     seeded N(0, 1) upstream gradient; fp32 gradients out."""
@@ -534,21 +538,30 @@ def linear_bwd_timing(s, d, steps, warmup, dev, local_rank):
     prof = vdn.profile_end()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / max(steps, 1)
-    fl = linear_bwd_flops(s)
+    work = linear_bwd_work(s)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     kernels = {}
     for name, (tot, n) in prof.items():
         avg = tot / max(n, 1)
         k = {"ms_per_launch": avg, "launches": n}
-        if name in fl and avg > 0:
-            ach = fl[name] / (avg / 1e3) / 1e12
-            k.update({"bound": "alu", "achieved": ach, "peak": FP32_CUDA_CORE_TFLOPS, "unit": "TFLOP/s",
-                      "frac": ach / FP32_CUDA_CORE_TFLOPS, "algorithmic_tflop_per_launch": fl[name] / 1e12})
+        if name in work and avg > 0:
+            kind, amount = work[name]
+            if kind == "flops":
+                ach = amount / (avg / 1e3) / 1e12
+                k.update({"bound": "alu", "achieved": ach, "peak": FP32_CUDA_CORE_TFLOPS, "unit": "TFLOP/s",
+                          "frac": ach / FP32_CUDA_CORE_TFLOPS, "algorithmic_tflop_per_launch": amount / 1e12})
+            else:
+                ach = amount / (avg / 1e3) / 1e9
+                k.update({"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                          "algorithmic_bytes_per_launch": amount})
         kernels[name] = k
+    flops = sum(a for kind, a in work.values() if kind == "flops")
     out = {"entry_point": "vdn_linear_branch_bwd", "linear": "elu1", "inputs": "this run's bf16 q, k, v, kt, vt; "
            "do_l ~ N(0, 1) fp32 (seed 17); fp32 gradients", "ms_per_step": ms,
            "value": s.n_video / (ms / 1e3), "unit": UNIT, "steps": steps, "warmup": warmup,
-           "tflops": sum(fl.values()) / (ms / 1e3) / 1e12,
-           "peak_note": "fp32 FMA lanes: 148 SMs x 128 x 2 flops x 1965 MHz", "kernels": kernels, "clocks": clk}
+           "tflops": flops / (ms / 1e3) / 1e12,
+           "peak_note": "fp32 FMA lanes: 148 SMs x 128 x 2 flops x 1965 MHz; the per-group sums against the "
+                        "measured HBM copy rate", "kernels": kernels, "clocks": clk}
     del ws, do_l, dq, dk, dv, dkt, dvt
     torch.cuda.empty_cache()
     return out
@@ -832,7 +845,7 @@ def run_ours(args, rank, world, local_rank):
         extra["e4m3_projection"] = extra_layer_timing(s, vdn.DELTA, vdn.E4M3_PROJ, d, beta.contiguous(), G_l,
                                                       args.steps, 2, dev, local_rank, peaks, ratio5)
         line["config5_extra"] = extra
-        line["linear_bwd_extra"] = linear_bwd_timing(s, d, args.steps, 2, dev, local_rank)
+        line["linear_bwd_extra"] = linear_bwd_timing(s, d, args.steps, 2, dev, local_rank, peaks)
     line["pages_context"] = PAGES_CONTEXT
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg, inp, args.cpu_rows)

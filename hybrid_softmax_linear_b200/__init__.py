@@ -94,10 +94,11 @@ _SIGS = {
     "vdn_profile_end": (ctypes.c_int, [_vp, _vp, _i32]),
 }
 
-PROF_KERNELS = 19
+PROF_KERNELS = 20
 KERNEL_NAMES = {1: "tables", 2: "softmax_simt", 3: "softmax_tc", 4: "state_build", 5: "scan", 6: "read", 7: "fuse",
                 8: "out_proj_simt", 9: "out_proj_tc", 10: "fp8_quant", 11: "delta_stats", 13: "state_build_tc",
-                14: "read_stage", 15: "read_tc", 16: "lin_bwd_rows", 17: "lin_bwd_groups", 18: "lin_bwd_keys"}
+                14: "read_stage", 15: "read_tc", 16: "lin_bwd_rows", 17: "lin_bwd_frames", 18: "lin_bwd_keys",
+                19: "lin_bwd_groups"}
 
 
 def lib() -> ctypes.CDLL:

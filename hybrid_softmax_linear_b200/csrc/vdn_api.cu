@@ -401,23 +401,31 @@ vdn_status vdn_linear_branch_bwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_
   char *w = (char *)ws;
   const WsPlan &p = b.p;
   VDN_CUDA(launch_tables(d, w, p, st), "tables launch");
-  float *S = (float *)(w + p.S), *z = (float *)(w + p.z), *St = (float *)(w + p.St), *zt = (float *)(w + p.zt);
-  float *Sf = (float *)(w + p.Sf), *Sb = (float *)(w + p.Sb), *zf = (float *)(w + p.zf), *zb = (float *)(w + p.zb);
+  LinBwdArgs a{};
+  a.d = d;
+  a.q = q; a.k = k; a.v = v; a.kt = kt; a.vt = vt; a.dO = do_l;
+  a.S = (float *)(w + p.S); a.z = (float *)(w + p.z); a.St = (float *)(w + p.St); a.zt = (float *)(w + p.zt);
+  a.Sf = (float *)(w + p.Sf); a.Sb = (float *)(w + p.Sb); a.zf = (float *)(w + p.zf); a.zb = (float *)(w + p.zb);
+  a.ftab = (const int32_t *)(w + p.ftab); a.gtab = (const int32_t *)(w + p.gtab);
+  a.G = host_group_count(d);
+  a.dnum = (float *)(w + b.dnum); a.dden = (float *)(w + b.dden);
+  a.part = a.S; a.zpart = a.z;  // the per-frame states are dead once the scan has read them
+  a.dN = (float *)(w + b.dN); a.dZ = (float *)(w + b.dZ);
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dkt = dkt; a.dvt = dvt;
   {
     ProfScope ps(K_STATE, st);
-    VDN_CUDA(launch_state_build(d, VDN_LIN_ELU1, VDN_BF16, k, v, kt, vt, S, z, St, zt, st), "state build launch");
+    VDN_CUDA(launch_linear_bwd(a, LIN_BWD_STATE, st), "state rebuild launch");
   }
   {
     ProfScope ps(K_SCAN, st);
-    VDN_CUDA(launch_state_scan(d, VDN_LIN_ELU1, S, z, St, zt, nullptr, Sf, Sb, zf, zb, w, p, st), "scan launch");
+    VDN_CUDA(launch_state_scan(d, VDN_LIN_ELU1, a.S, a.z, a.St, a.zt, nullptr, a.Sf, a.Sb, a.zf, a.zb, w, p, st),
+             "scan launch");
   }
-  static const int kids[3] = {K_LIN_BWD_ROWS, K_LIN_BWD_GROUPS, K_LIN_BWD_KEYS};
-  for (int stage = 0; stage < 3; ++stage) {
-    ProfScope ps(kids[stage], st);
-    VDN_CUDA(launch_linear_bwd(d, stage, q, k, v, kt, vt, do_l, Sf, Sb, zf, zb, (const int32_t *)(w + p.gtab),
-                               host_group_count(d), (float *)(w + b.dnum), (float *)(w + b.dden),
-                               (float *)(w + b.dN), (float *)(w + b.dZ), dq, dk, dv, dkt, dvt, st),
-             "linear branch backward launch");
+  static const int stages[4] = {LIN_BWD_ROWS, LIN_BWD_FRAMES, LIN_BWD_GROUPS, LIN_BWD_KEYS};
+  static const int kids[4] = {K_LIN_BWD_ROWS, K_LIN_BWD_FRAMES, K_LIN_BWD_GROUPS, K_LIN_BWD_KEYS};
+  for (int i = 0; i < 4; ++i) {
+    ProfScope ps(kids[i], st);
+    VDN_CUDA(launch_linear_bwd(a, stages[i], st), "linear branch backward launch");
   }
   return ok();
 }

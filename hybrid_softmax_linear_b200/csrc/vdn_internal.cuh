@@ -259,8 +259,8 @@ struct DevStatus {
 enum KernelId : uint32_t {
   K_TABLES = 1, K_SOFTMAX_SIMT = 2, K_SOFTMAX_TC = 3, K_STATE = 4, K_SCAN = 5, K_READ = 6,
   K_FUSE = 7, K_GEMM_SIMT = 8, K_GEMM_TC = 9, K_QUANT = 10, K_DELTA = 11, K_DEBUG_WAIT = 12,
-  K_STATE_TC = 13, K_READ_STAGE = 14, K_READ_TC = 15, K_LIN_BWD_ROWS = 16, K_LIN_BWD_GROUPS = 17,
-  K_LIN_BWD_KEYS = 18,
+  K_STATE_TC = 13, K_READ_STAGE = 14, K_READ_TC = 15, K_LIN_BWD_ROWS = 16, K_LIN_BWD_FRAMES = 17,
+  K_LIN_BWD_KEYS = 18, K_LIN_BWD_GROUPS = 19,
 };
 
 __device__ __forceinline__ void report(DevStatus *st, uint32_t code, uint32_t where, uint32_t detail) {
@@ -389,14 +389,29 @@ cudaError_t launch_softmax_tc_gated(const Dims &d, vdn_dtype dt, const void *q, 
                                     const void *kt, const void *vt, const float *scales, const float *w_gate_s,
                                     float sl2, void *a, char *ws, const WsPlan &p, cudaStream_t st, bool a8 = false);
 // per-head e4m3 quantisation of q, k (+ text), v (+ text); scales float[3][H]
-// backward of the elu+1 linear branch (CUDA cores, fp32): Sf..zb the groups' memories,
-// gtab the group table (G groups); dnum [N_v][H][D], dden [N_v][H], dN [G][H][D][D],
-// dZ [G][H][D] scratch
-// stage 0: per-row dq, dnum, dden; 1: per-group dNum, dDen; 2: per-key-frame dk, dv
-cudaError_t launch_linear_bwd(const Dims &d, int stage, const void *q, const void *k, const void *v, const void *kt,
-                              const void *vt, const float *dO, const float *Sf, const float *Sb, const float *zf,
-                              const float *zb, const int32_t *gtab, int G, float *dnum, float *dden, float *dN,
-                              float *dZ, float *dq, float *dk, float *dv, float *dkt, float *dvt, cudaStream_t st);
+// Backward of the elu+1 linear branch (CUDA cores, fp32), launched stage by stage (the
+// forward's scan runs between the state rebuild and the row stage).
+enum LinBwdStage : int {
+  LIN_BWD_STATE = 0,   // per-frame and text states S, z, St, zt in fp32
+  LIN_BWD_ROWS = 1,    // per query row: dq, dnum, dden
+  LIN_BWD_FRAMES = 2,  // per query frame: sum of phi(q)^T dnum and phi(q) dden (part, zpart)
+  LIN_BWD_GROUPS = 3,  // per group: dN, dZ from the frame sums
+  LIN_BWD_KEYS = 4,    // per key frame and the text: dk, dv, dkt, dvt
+};
+struct LinBwdArgs {
+  Dims d;
+  const void *q, *k, *v, *kt, *vt;  // bf16 [rows][H][D]
+  const float *dO;
+  float *S, *z, *St, *zt;           // [F][H][D][D], [F][H][D], [H][D][D], [H][D]
+  float *Sf, *Sb, *zf, *zb;         // group memories [G][H][D][D], [G][H][D]
+  const int32_t *ftab, *gtab;
+  int G;
+  float *dnum, *dden;               // [Nv][H][D], [Nv][H]
+  float *part, *zpart;              // [F][H][D][D], [F][H][D]
+  float *dN, *dZ;                   // [G][H][D][D], [G][H][D]
+  float *dq, *dk, *dv, *dkt, *dvt;
+};
+cudaError_t launch_linear_bwd(const LinBwdArgs &a, int stage, cudaStream_t st);
 cudaError_t launch_fp8_quant(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
                              const void *vt, void *q8, void *k8, void *v8, void *kt8, void *vt8, float *scales,
                              uint32_t *amax_bits, cudaStream_t st);

@@ -366,9 +366,10 @@ VDN_API vdn_status vdn_debug_unset_flag_wait(void *ws, size_t ws_bytes, uint32_t
  * count launches[k], and disables recording.  Kernel ids: 1 tables, 2 softmax (CUDA
  * cores), 3 softmax (tensor cores), 4 state build, 5 scan, 6 read, 7 fuse, 8 projection
  * (CUDA cores), 9 projection (tensor cores), 10 fp8 quantisation, 11 delta statistics,
- * 13 state build (tensor cores), 14 read staging, 15 read (tensor cores), 16-18 the linear
- * branch's backward (per-row dq, per-group dNum/dDen, per-key-frame dk/dv). */
-#define VDN_PROF_KERNELS 19
+ * 13 state build (tensor cores), 14 read staging, 15 read (tensor cores), and the linear
+ * branch's backward: 16 per query row (dq), 17 per-frame gradient sums, 18 per key row
+ * (dk, dv), 19 per-group gradient sums (its state rebuild and scan count as 4 and 5). */
+#define VDN_PROF_KERNELS 20
 VDN_API vdn_status vdn_profile_begin(int32_t max_launches);
 VDN_API vdn_status vdn_profile_end(float *ms, int32_t *launches, int32_t n);
 
