@@ -92,7 +92,7 @@ template <int D>
 __device__ __forceinline__ void tile_mma2(const float *A1, const float *B1, const float *A2, const float *B2, int ty,
                                           int tx, float2 (&acc1)[4][Lay<D>::NP], float2 (&acc2)[4][Lay<D>::NP]) {
   using L = Lay<D>;
-#pragma unroll 1
+#pragma unroll 2
   for (int k0 = 0; k0 < D; k0 += 4) {
     float a1[4][4], a2[4][4];
 #pragma unroll
@@ -121,31 +121,45 @@ __device__ __forceinline__ void tile_mma2(const float *A1, const float *B1, cons
   }
 }
 
-// n (<= 64) bf16 rows of D features (row stride `stride` elements) into a [64][LD] tile as
-// float, phi applied when PHI; rows n..63 are zero.
+// A 64-row tile of bf16 rows of D features moves in two steps, so that its global loads can
+// be in flight while the previous tile is being multiplied: fetch_tile reads n (<= 64) rows
+// (row stride `stride` elements) into registers, 16 bytes per piece; put_tile converts them
+// to float (phi applied when PHI) into a [64][LD] tile in shared memory, rows n..63 zero.
+template <int D>
+struct TileRegs {
+  static constexpr int PER_ROW = D / 8;               // 16-byte pieces per row
+  static constexpr int N = BM * PER_ROW / BT;         // pieces per thread (exact for D >= 32)
+  uint4 r[N];
+};
+
+template <int D>
+__device__ __forceinline__ void fetch_tile(const __nv_bfloat16 *__restrict__ src, int64_t stride, int n,
+                                           TileRegs<D> &x, int t) {
+  constexpr int PR = TileRegs<D>::PER_ROW;
+#pragma unroll
+  for (int u = 0; u < TileRegs<D>::N; ++u) {
+    const int e = t + u * BT, row = e / PR;
+    x.r[u] = row < n ? *reinterpret_cast<const uint4 *>(src + row * stride + (e % PR) * 8) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 template <int D, bool PHI>
-__device__ __forceinline__ void load_tile(const __nv_bfloat16 *__restrict__ src, int64_t stride, int n, float *dst,
-                                          int t) {
+__device__ __forceinline__ void put_tile(const TileRegs<D> &x, int n, float *dst, int t) {
   using L = Lay<D>;
-  constexpr int PER_ROW = D / 8;  // 16-byte pieces per row
-  for (int e = t; e < BM * PER_ROW; e += BT) {
-    const int row = e / PER_ROW, c8 = (e % PER_ROW) * 8;
-    float x[8];
-    if (row < n) {
-      const uint4 raw = *reinterpret_cast<const uint4 *>(src + row * stride + c8);
-      const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+  constexpr int PR = TileRegs<D>::PER_ROW;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(p2[i]);
-        x[2 * i] = PHI ? phi1(f.x) : f.x;
-        x[2 * i + 1] = PHI ? phi1(f.y) : f.y;
-      }
-    } else {
+  for (int u = 0; u < TileRegs<D>::N; ++u) {
+    const int e = t + u * BT, row = e / PR, c8 = (e % PR) * 8;
+    float y[8];
+    const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&x.r[u]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(p2[i]);
+      y[2 * i] = PHI && row < n ? phi1(f.x) : f.x;  // a dead row was fetched as zeros and stays zero
+      y[2 * i + 1] = PHI && row < n ? phi1(f.y) : f.y;
     }
-    st_vec<4>(dst + row * L::LD + c8, x);
-    st_vec<4>(dst + row * L::LD + c8 + 4, x + 4);
+    st_vec<4>(dst + row * L::LD + c8, y);
+    st_vec<4>(dst + row * L::LD + c8 + 4, y + 4);
   }
 }
 
@@ -332,10 +346,27 @@ __global__ void __launch_bounds__(BT, 1) lin_bwd_rows_kernel(Dims d, const __nv_
   for (int e = t; e < D; e += BT) Den[e] = zf[((int64_t)g * d.H + h) * D + e] + zb[((int64_t)g * d.H + h) * D + e];
   __syncthreads();
   const int64_t fr0 = (int64_t)f * d.T;
+  const __nv_bfloat16 *qb = q + fr0 * HD + (int64_t)h * D;
+  TileRegs<D> rq;
+  fetch_tile<D>(qb, HD, min(BM, d.T), rq, t);
   for (int m0 = 0; m0 < d.T; m0 += BM) {
     const int n = min(BM, d.T - m0);
-    load_tile<D, true>(q + (fr0 + m0) * HD + (int64_t)h * D, HD, n, P, t);
+    put_tile<D, true>(rq, n, P, t);
     __syncthreads();
+    // this tile's dO and the next tile's q are in flight while den and num are computed
+    float go[4][L::CPT];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int row = ty * 4 + r;
+#pragma unroll
+      for (int c = 0; c < L::CPT; ++c) go[r][c] = 0.f;
+      if (row < n) {
+#pragma unroll
+        for (int v = 0; v < L::NV; ++v)
+          ld_vec<L::VW>(dO + (fr0 + m0 + row) * HD + (int64_t)h * D + L::col(tx, v), go[r] + v * L::VW);
+      }
+    }
+    if (m0 + BM < d.T) fetch_tile<D>(qb + (int64_t)(m0 + BM) * HD, HD, min(BM, d.T - m0 - BM), rq, t);
     {  // den partials over quarters of the features: row t / 4, quarter t % 4
       const int row = t >> 2, qq = t & 3;
       const float *pr = P + row * L::LD + qq * (D / 4), *dr = Den + qq * (D / 4);
@@ -365,16 +396,13 @@ __global__ void __launch_bounds__(BT, 1) lin_bwd_rows_kernel(Dims d, const __nv_
       float dot = 0.f;
 #pragma unroll
       for (int v = 0; v < L::NV; ++v) {
-        float go[L::VW], dn[L::VW];
-#pragma unroll
-        for (int c = 0; c < L::VW; ++c) go[c] = 0.f;
-        if (live) ld_vec<L::VW>(dO + gb + L::col(tx, v), go);
+        float dn[L::VW];
 #pragma unroll
         for (int c = 0; c < L::VW; ++c) {
           const int ci = v * L::VW + c;
           const float o = pick(acc[r][ci >> 1], ci) * inv;
-          dot = fmaf(go[c], o, dot);
-          dn[c] = go[c] * inv;
+          dot = fmaf(go[r][ci], o, dot);
+          dn[c] = go[r][ci] * inv;
         }
         st_vec<L::VW>(DN + row * L::LD + L::col(tx, v), dn);
         if (live) st_vec<L::VW>(dnum_out + gb + L::col(tx, v), dn);
@@ -456,20 +484,42 @@ __global__ void __launch_bounds__(BT, 1) lin_bwd_keys_kernel(Dims d, const __nv_
   using L = Lay<D>;
   extern __shared__ __align__(16) float sm[];
   float *dS = sm, *dST = dS + D * L::LD, *Vs = dST + D * L::LD, *PK = Vs + BM * L::LD, *dz = PK + BM * L::LD;
+  unsigned char *held = reinterpret_cast<unsigned char *>(dz + D);  // [G]: group g's memory holds fk
   const int fk = blockIdx.x, h = blockIdx.y, t = threadIdx.x, ty = t >> 4, tx = t & 15;
   const bool text = fk == d.F;
   const int64_t DD = (int64_t)D * D, HD = (int64_t)d.H * D;
-  auto holds = [&](int g) {
+  const int ntok = text ? d.L : d.T;
+  const __nv_bfloat16 *kb = (text ? kt : k + (int64_t)fk * d.T * HD) + (int64_t)h * D;
+  const __nv_bfloat16 *vb = (text ? vt : v + (int64_t)fk * d.T * HD) + (int64_t)h * D;
+  float *dkb = (text ? dkt : dk + (int64_t)fk * d.T * HD) + (int64_t)h * D;
+  float *dvb = (text ? dvt : dv + (int64_t)fk * d.T * HD) + (int64_t)h * D;
+  TileRegs<D> rk, rv;  // the first tile's loads are in flight during the gather
+  fetch_tile<D>(kb, HD, min(BM, ntok), rk, t);
+  fetch_tile<D>(vb, HD, min(BM, ntok), rv, t);
+  for (int g = t; g < G; g += BT) {
     const int32_t *r = gtab + g * 16;
-    return text || (fk >= r[12] && fk < r[13]) || (fk >= r[14] && fk < r[15]);
-  };
+    held[g] = (text || (fk >= r[12] && fk < r[13]) || (fk >= r[14] && fk < r[15])) ? 1 : 0;
+  }
+  __syncthreads();
+  // loads of 8 groups at a time, added in group order
+  constexpr int GB = 8;
   for (int e = t; e < D * D / 4; e += BT) {
     const int i = e % D, j0 = 4 * (e / D);
     float s[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int g = 0; g < G; ++g) {
-      if (!holds(g)) continue;
-      const float4 x = *reinterpret_cast<const float4 *>(dN + ((int64_t)g * d.H + h) * DD + i * D + j0);
-      s[0] += x.x; s[1] += x.y; s[2] += x.z; s[3] += x.w;
+    for (int g0 = 0; g0 < G; g0 += GB) {
+      float4 x[GB];
+#pragma unroll
+      for (int u = 0; u < GB; ++u) {
+        const int g = g0 + u;
+        x[u] = (g < G && held[g]) ? *reinterpret_cast<const float4 *>(dN + ((int64_t)g * d.H + h) * DD + i * D + j0)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < GB; ++u) {
+        if (g0 + u < G && held[g0 + u]) {
+          s[0] += x[u].x; s[1] += x[u].y; s[2] += x[u].z; s[3] += x[u].w;
+        }
+      }
     }
     st_vec<4>(dS + i * L::LD + j0, s);
 #pragma unroll
@@ -478,20 +528,18 @@ __global__ void __launch_bounds__(BT, 1) lin_bwd_keys_kernel(Dims d, const __nv_
   for (int e = t; e < D; e += BT) {
     float s = 0.f;
     for (int g = 0; g < G; ++g)
-      if (holds(g)) s += dZ[((int64_t)g * d.H + h) * D + e];
+      if (held[g]) s += dZ[((int64_t)g * d.H + h) * D + e];
     dz[e] = s;
   }
-  __syncthreads();
-  const int ntok = text ? d.L : d.T;
-  const __nv_bfloat16 *kb = (text ? kt : k + (int64_t)fk * d.T * HD) + (int64_t)h * D;
-  const __nv_bfloat16 *vb = (text ? vt : v + (int64_t)fk * d.T * HD) + (int64_t)h * D;
-  float *dkb = (text ? dkt : dk + (int64_t)fk * d.T * HD) + (int64_t)h * D;
-  float *dvb = (text ? dvt : dv + (int64_t)fk * d.T * HD) + (int64_t)h * D;
   for (int m0 = 0; m0 < ntok; m0 += BM) {
     const int n = min(BM, ntok - m0);
-    load_tile<D, true>(kb + (int64_t)m0 * HD, HD, n, PK, t);
-    load_tile<D, false>(vb + (int64_t)m0 * HD, HD, n, Vs, t);
+    put_tile<D, true>(rk, n, PK, t);
+    put_tile<D, false>(rv, n, Vs, t);
     __syncthreads();
+    if (m0 + BM < ntok) {
+      fetch_tile<D>(kb + (int64_t)(m0 + BM) * HD, HD, min(BM, ntok - m0 - BM), rk, t);
+      fetch_tile<D>(vb + (int64_t)(m0 + BM) * HD, HD, min(BM, ntok - m0 - BM), rv, t);
+    }
     float2 a1[4][L::NP], a2[4][L::NP];
 #pragma unroll
     for (int r = 0; r < 4; ++r)
@@ -555,7 +603,7 @@ cudaError_t lin_bwd_t(const LinBwdArgs &a, int stage, cudaStream_t st) {
       lin_bwd_group_sum_kernel<D><<<dim3(a.G, d.H), BT, 0, st>>>(d, a.part, a.zpart, a.gtab, a.dN, a.dZ);
       break;
     case LIN_BWD_KEYS: {
-      const size_t smem = (size_t)(2 * D * L::LD + 2 * BM * L::LD + D) * sizeof(float);
+      const size_t smem = (size_t)(2 * D * L::LD + 2 * BM * L::LD + D) * sizeof(float) + (size_t)((a.G + 15) & ~15);
       e = cudaFuncSetAttribute(lin_bwd_keys_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
       lin_bwd_keys_kernel<D><<<dim3(d.F + 1, d.H), BT, smem, st>>>(

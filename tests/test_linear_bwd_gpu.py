@@ -35,7 +35,11 @@ def _run(s, inp, do_l):
 @pytest.mark.parametrize("shape", [(13, 24, 5, 8, 2, 32),     # D = 32, ragged last chunk
                                    (12, 40, 5, 6, 2, 64),     # D = 64
                                    (9, 33, 3, 10, 2, 128),    # D = 128, odd T
-                                   (7, 20, 3, 0, 1, 64)])     # no text
+                                   (7, 20, 3, 0, 1, 64),      # no text
+                                   # several 64-row tiles and 32-row chunks per frame and in the
+                                   # text, each with a ragged last one
+                                   (6, 150, 2, 70, 2, 128),
+                                   (5, 130, 2, 40, 3, 32)])
 def test_linear_branch_bwd_matches_oracle(shape):
     assert torch.cuda.is_available(), "GPU test needs a CUDA device"
     s = synth.Shape(*shape)
