@@ -567,6 +567,24 @@ def linear_bwd_timing(s, d, steps, warmup, dev, local_rank, peaks):
     return out
 
 
+def run_linear_bwd_only(args, local_rank):
+    """The linear branch's backward alone at one configuration's shapes and inputs (an elu+1,
+    bf16 configuration), for profiling it without the rest of the layer."""
+    import torch
+    from hybrid_softmax_linear_b200.tensors import to_device
+    w = synth.CONFIGS[args.config]
+    if w.linear != "elu1" or w.dtype != "bf16" or w.softmax_fp8:
+        raise SystemExit(f"--linear-bwd-only needs an elu+1 bf16 configuration, not {w.name}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inp = synth.workload_inputs(args.config, 0)
+    d = {n: to_device(inp[n], dev) for n in ("q", "k", "v", "kt", "vt")}
+    peaks, _ = load_peaks()
+    out = linear_bwd_timing(w.shape, d, args.steps, args.warmup, dev, local_rank, peaks)
+    out["config"] = workload_config(args.config)
+    print(json.dumps(out), flush=True)
+
+
 def run_split(args, rank, world, local_rank):
     """One video's layer split by heads over the ranks (strong scaling): each rank runs its
     heads through both branches and the fuse, multiplies its part of A by the matching
@@ -866,12 +884,17 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the extra timings (the e4m3 configuration, the linear branch's backward)")
     ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
                     help="replicas: one video per GPU (weak scaling); heads: one video split by heads (strong)")
+    ap.add_argument("--linear-bwd-only", action="store_true",
+                    help="time only the elu+1 linear branch's backward at --config (one GPU; prints its own line)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.linear_bwd_only:
+        run_linear_bwd_only(args, local_rank)
         return
     import datetime
     import torch

@@ -158,3 +158,16 @@ def test_clock_sampler_summarises_only_the_timed_region(monkeypatch):
     assert got["source"] == "nvml" and got["samples"] >= 2
     assert got["sm_mhz"] == 1900 and got["sm_max_mhz"] == 1965
     assert got["reasons"] == ["sw_power_cap"] and got["power_w_max"] == 700.0
+
+
+def test_linear_bwd_only_refuses_configurations_without_an_elu1_bf16_branch(monkeypatch):
+    """--linear-bwd-only times the elu+1 backward; a delta-rule or e4m3 configuration is
+    refused on the host before any device work."""
+    import sys
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--linear-bwd-only", "--config", "5"])
+    try:
+        bench.main()
+    except SystemExit as e:
+        assert "elu+1 bf16" in str(e.code)
+    else:
+        raise AssertionError("configuration 5 was accepted")
