@@ -32,18 +32,6 @@ __device__ __forceinline__ uint32_t swz_off(int r, int cl, int box_rows) {
   return (uint32_t)((cl >> 3) * box_rows * 128 + r * 128 + ((((cl & 7) ^ (r & 7))) << 4));
 }
 
-// phi(x) = elu(x) + 1 without a branch: max(x, 0) + e^min(x, 0) is x + 1 for x > 0 (e^0 = 1
-// exactly) and e^x otherwise, and keeps the warp converged whatever the signs
-__device__ __forceinline__ float phi_fast(float x) { return fmaxf(x, 0.f) + __expf(fminf(x, 0.f)); }
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
-  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 x = __bfloat1622float2(h[i]);
-    f[2 * i] = x.x; f[2 * i + 1] = x.y;
-  }
-}
 __device__ __forceinline__ uint4 pack8(const float *f) {
   uint4 u;
   u.x = pack_bf16(f[0], f[1]); u.y = pack_bf16(f[2], f[3]); u.z = pack_bf16(f[4], f[5]); u.w = pack_bf16(f[6], f[7]);
