@@ -603,7 +603,7 @@ cudaError_t lin_bwd_t(const LinBwdArgs &a, int stage, cudaStream_t st) {
       lin_bwd_group_sum_kernel<D><<<dim3(a.G, d.H), BT, 0, st>>>(d, a.part, a.zpart, a.gtab, a.dN, a.dZ);
       break;
     case LIN_BWD_KEYS: {
-      const size_t smem = (size_t)(2 * D * L::LD + 2 * BM * L::LD + D) * sizeof(float) + (size_t)((a.G + 15) & ~15);
+      const size_t smem = linear_bwd_keys_smem(D, a.G);
       e = cudaFuncSetAttribute(lin_bwd_keys_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
       lin_bwd_keys_kernel<D><<<dim3(d.F + 1, d.H), BT, smem, st>>>(
@@ -618,6 +618,13 @@ cudaError_t lin_bwd_t(const LinBwdArgs &a, int stage, cudaStream_t st) {
 }
 
 }  // namespace
+
+size_t linear_bwd_keys_smem(int D, int G) {
+  const size_t g = (size_t)((G + 15) & ~15);
+  if (D == 32) return (size_t)(2 * D * Lay<32>::LD + 2 * BM * Lay<32>::LD + D) * sizeof(float) + g;
+  if (D == 64) return (size_t)(2 * D * Lay<64>::LD + 2 * BM * Lay<64>::LD + D) * sizeof(float) + g;
+  return (size_t)(2 * D * Lay<128>::LD + 2 * BM * Lay<128>::LD + D) * sizeof(float) + g;
+}
 
 cudaError_t launch_linear_bwd(const LinBwdArgs &a, int stage, cudaStream_t st) {
   if (a.d.D == 32) return lin_bwd_t<32>(a, stage, st);

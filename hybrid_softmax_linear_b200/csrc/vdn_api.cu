@@ -388,6 +388,10 @@ vdn_status vdn_linear_branch_bwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_
   VDN_TRY(check_kind(kind));
   if (kind != VDN_LIN_ELU1) return fail(VDN_ERR_UNSUPPORTED, "the linear branch's backward is built for ELU1 only");
   if (dtype != VDN_BF16) return fail(VDN_ERR_UNSUPPORTED, "the linear branch's backward takes bf16 inputs");
+  const int G = host_group_count(dims_of(*shape));
+  if (linear_bwd_keys_smem(shape->head_dim, G) > MAX_DYN_SMEM)
+    return fail(VDN_ERR_UNSUPPORTED, "%d groups: the backward's key kernel keeps one flag per group in shared "
+                "memory, which this many groups overflow", G);
   VDN_TRY(need(q, "q")); VDN_TRY(need(k, "k")); VDN_TRY(need(v, "v")); VDN_TRY(need(do_l, "do_l"));
   VDN_TRY(need(dq, "dq")); VDN_TRY(need(dk, "dk")); VDN_TRY(need(dv, "dv"));
   if (shape->text_tokens > 0) {
@@ -407,7 +411,7 @@ vdn_status vdn_linear_branch_bwd(const vdn_shape *shape, vdn_lin_kind kind, vdn_
   a.S = (float *)(w + p.S); a.z = (float *)(w + p.z); a.St = (float *)(w + p.St); a.zt = (float *)(w + p.zt);
   a.Sf = (float *)(w + p.Sf); a.Sb = (float *)(w + p.Sb); a.zf = (float *)(w + p.zf); a.zb = (float *)(w + p.zb);
   a.ftab = (const int32_t *)(w + p.ftab); a.gtab = (const int32_t *)(w + p.gtab);
-  a.G = host_group_count(d);
+  a.G = G;
   a.dnum = (float *)(w + b.dnum); a.dden = (float *)(w + b.dden);
   a.part = a.S; a.zpart = a.z;  // the per-frame states are dead once the scan has read them
   a.dN = (float *)(w + b.dN); a.dZ = (float *)(w + b.dZ);

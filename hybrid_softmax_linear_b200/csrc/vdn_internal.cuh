@@ -412,6 +412,10 @@ struct LinBwdArgs {
   float *dq, *dk, *dv, *dkt, *dvt;
 };
 cudaError_t launch_linear_bwd(const LinBwdArgs &a, int stage, cudaStream_t st);
+// Dynamic shared memory of the backward's key kernel: the D x D gradient and its transpose,
+// two 64-row tiles, and one flag per group.
+size_t linear_bwd_keys_smem(int D, int G);
+constexpr size_t MAX_DYN_SMEM = 232448;  // per block, sm_100 (227 KB)
 cudaError_t launch_fp8_quant(const Dims &d, const void *q, const void *k, const void *v, const void *kt,
                              const void *vt, void *q8, void *k8, void *v8, void *kt8, void *vt8, float *scales,
                              uint32_t *amax_bits, cudaStream_t st);

@@ -228,6 +228,9 @@ VDN_API vdn_status vdn_linear_read(const vdn_shape *shape, vdn_lin_kind kind, vd
  *   q, k, v [N_v][H][D] and kt, vt [L][H][D] bf16; do_l float [N_v][H][D];
  *   dq, dk, dv float [N_v][H][D]; dkt, dvt float [L][H][D] (NULL allowed when L = 0).
  *   All pointers device memory, 16-byte aligned, owned by the caller.
+ *   Layouts with more groups than the key kernel's shared memory can flag (29184 at
+ *   D = 128; only one-frame chunks over tens of thousands of frames get there) give
+ *   VDN_ERR_UNSUPPORTED before any device work.
  * ws: vdn_linear_branch_bwd_workspace_size(shape) bytes (tables, the states and memories,
  * and per-row and per-group scratch). */
 VDN_API size_t vdn_linear_branch_bwd_workspace_size(const vdn_shape *shape);

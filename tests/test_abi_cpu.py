@@ -139,6 +139,11 @@ def test_linear_branch_bwd_checks():
     assert st == 1 and b"kt" in L.vdn_last_error()
     st = L.vdn_linear_branch_bwd(ctypes.byref(s), vdn.ELU1, vdn.BF16, *args, 256, need - 256, None)
     assert st == 3  # workspace too small
+    # one-frame chunks give one group per frame; the key kernel's per-group flags overflow
+    # its shared memory past 29184 groups at D = 128, refused before any device work
+    big = vdn.Shape(30000, 1, 1, 0, 1, 128)
+    st = L.vdn_linear_branch_bwd(ctypes.byref(big), vdn.ELU1, vdn.BF16, *args, 256, 1 << 40, None)
+    assert st == 2 and b"groups" in L.vdn_last_error()
 
 
 def test_noalloc_checks_match_the_workspace_entry_point():
