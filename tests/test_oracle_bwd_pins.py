@@ -107,6 +107,21 @@ def test_branch_gradients_match_finite_differences(F, T, C, L, H, D, G_l):
     _check_fd(delta, inp, dict(zip(names + ("beta",), g)), names + ("beta",))
 
 
+def test_linear_branch_gradients_are_per_head():
+    """The linear branch mixes no heads, so its gradients for all heads at once equal those of
+    each one-head slice of the inputs (what the full-size GPU check relies on); a head or
+    feature axis mixed up anywhere in the backward breaks this."""
+    F, T, C, L, H, D = 9, 6, 2, 4, 3, 8
+    inp = _inputs(F, T, L, H, D, None, seed=12)
+    do = np.random.default_rng(13).standard_normal((F * T, H, D))
+    names = ("q", "k", "v", "kt", "vt")
+    whole = vb.linear_branch_bwd(*(inp[n] for n in names), F, T, C, do)
+    for h in range(H):
+        one = vb.linear_branch_bwd(*(inp[n][:, h:h + 1] for n in names), F, T, C, do[:, h:h + 1])
+        for a, b in zip(whole, one):
+            np.testing.assert_allclose(a[:, h:h + 1], b, rtol=1e-12, atol=1e-14)
+
+
 @pytest.mark.parametrize("G_l", [None, 1])
 def test_fuse_gradients_match_finite_differences(G_l):
     H, D, n = 2, 4, 5
