@@ -289,6 +289,28 @@ def oracle_sample(cfg: int, inp: dict, n_rows: int, seed: int = 11) -> dict:
             "t_states_s": round(t1 - t0, 3), "t_rows_s": round(t2 - t1, 3)}
 
 
+def oracle_bwd_sample(s, inp: dict, heads: int = 1, seed: int = 23) -> dict:
+    """Time the float64 backward oracle of the elu+1 linear branch on a bounded sample: the
+    first `heads` heads of the workload, every row (the branch mixes no heads, so a head
+    slice is a whole problem).  Extrapolates to video tokens/s of all heads."""
+    from oracle import vdn_oracle_bwd as vb
+    F, T, C, H, D = s.frames, s.tokens_per_frame, s.chunk_frames, s.heads, s.head_dim
+    o = {n: (synth.bf16_bits_to_f32(inp[n][:, :heads]) if inp[n].dtype == np.uint16 else inp[n][:, :heads])
+         for n in ("q", "k", "v", "kt", "vt")}
+    do_l = np.random.default_rng(seed).standard_normal((s.n_video, heads, D))
+    t0 = time.perf_counter()
+    vb.linear_branch_bwd(o["q"], o["k"], o["v"], o["kt"], o["vt"], F, T, C, do_l)
+    t = (time.perf_counter() - t0) * H / heads
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        cores = len(os.sched_getaffinity(0))
+    return {"value": s.n_video / t, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"the float64 backward oracle on {heads} of {H} heads, every row; extrapolated x{H / heads:g}",
+            "t_sample_s": round(t * heads / H, 3)}
+
+
 def dense_reference(s, dev, iters: int = 10, warmup: int = 3) -> dict:
     """The dense full-attention layer on the same shapes, through library kernels: torch SDPA
     with the cuDNN backend (Q [1,H,N_v,D], K/V [1,H,N_v+L,D], no mask, bf16), plus one bf16
@@ -505,7 +527,7 @@ def linear_bwd_work(s) -> dict:
             "lin_bwd_groups": ("bytes", (F + G) * H * D2 * 4)}                   # frame sums in, group sums out
 
 
-def linear_bwd_timing(s, d, steps, warmup, dev, local_rank, peaks):
+def linear_bwd_timing(s, d, steps, warmup, dev, local_rank, peaks, inp=None):
     """Times the elu+1 linear branch's backward (vdn_linear_branch_bwd: state rebuild in fp32,
     scan, per-row, per-group and per-key-frame kernels) on this run's bf16 q, k, v with a
     seeded N(0, 1) upstream gradient; fp32 gradients out."""
@@ -564,6 +586,8 @@ def linear_bwd_timing(s, d, steps, warmup, dev, local_rank, peaks):
                         "measured HBM copy rate", "kernels": kernels, "clocks": clk}
     del ws, do_l, dq, dk, dv, dkt, dvt
     torch.cuda.empty_cache()
+    if inp is not None:
+        out["cpu_baseline"] = oracle_bwd_sample(s, inp)
     return out
 
 
@@ -580,7 +604,8 @@ def run_linear_bwd_only(args, local_rank):
     inp = synth.workload_inputs(args.config, 0)
     d = {n: to_device(inp[n], dev) for n in ("q", "k", "v", "kt", "vt")}
     peaks, _ = load_peaks()
-    out = linear_bwd_timing(w.shape, d, args.steps, args.warmup, dev, local_rank, peaks)
+    out = linear_bwd_timing(w.shape, d, args.steps, args.warmup, dev, local_rank, peaks,
+                            None if args.no_cpu_baseline else inp)
     out["config"] = workload_config(args.config)
     print(json.dumps(out), flush=True)
 
@@ -863,7 +888,8 @@ def run_ours(args, rank, world, local_rank):
         extra["e4m3_projection"] = extra_layer_timing(s, vdn.DELTA, vdn.E4M3_PROJ, d, beta.contiguous(), G_l,
                                                       args.steps, 2, dev, local_rank, peaks, ratio5)
         line["config5_extra"] = extra
-        line["linear_bwd_extra"] = linear_bwd_timing(s, d, args.steps, 2, dev, local_rank, peaks)
+        line["linear_bwd_extra"] = linear_bwd_timing(s, d, args.steps, 2, dev, local_rank, peaks,
+                                                     None if args.no_cpu_baseline else inp)
     line["pages_context"] = PAGES_CONTEXT
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg, inp, args.cpu_rows)

@@ -171,3 +171,13 @@ def test_linear_bwd_only_refuses_configurations_without_an_elu1_bf16_branch(monk
         assert "elu+1 bf16" in str(e.code)
     else:
         raise AssertionError("configuration 5 was accepted")
+
+
+def test_backward_cpu_baseline_times_a_head_sample_of_the_oracle():
+    """The backward leg's CPU baseline runs the float64 backward oracle on a head slice and
+    scales by the head count; it reports the contract's keys."""
+    w = synth.CONFIGS[1]
+    inp = synth.workload_inputs(1)
+    got = bench.oracle_bwd_sample(w.shape, inp, heads=1)
+    assert got["kind"] == "oracle" and got["unit"] == bench.UNIT and got["cores"] >= 1
+    assert got["value"] > 0 and f"1 of {w.shape.heads} heads" in got["sample"]
