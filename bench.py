@@ -528,9 +528,11 @@ def linear_bwd_work(s) -> dict:
 
 
 def linear_bwd_timing(s, d, steps, warmup, dev, local_rank, peaks, inp=None):
-    """Times the elu+1 linear branch's backward (vdn_linear_branch_bwd: state rebuild in fp32,
-    scan, per-row, per-group and per-key-frame kernels) on this run's bf16 q, k, v with a
-    seeded N(0, 1) upstream gradient; fp32 gradients out."""
+    """Times the elu+1 linear branch's backward (vdn_linear_branch_bwd: fp32 state rebuild,
+    scan, per-row kernel, per-frame and per-group gradient sums, per-key-frame kernel) on this
+    run's bf16 q, k, v with a seeded N(0, 1) upstream gradient; fp32 gradients out.  With
+    `inp` (the host copies of the inputs) it also times the float64 backward oracle on a
+    head sample as the CPU baseline."""
     import torch
     import hybrid_softmax_linear_b200 as vdn
     from hybrid_softmax_linear_b200.tensors import workspace
